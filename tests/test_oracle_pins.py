@@ -1,0 +1,345 @@
+"""Pins for the oracle: checks against things other than the oracle itself.
+
+Each test ties one part of the oracle to a fixed point: the number-format
+definitions (cross-checked with torch's casts), closed forms, hand-computed
+values, invariants of the method, a library attention routine, brute force on
+tiny inputs, and the KV-state sizing figures printed on the vLLM page.
+"""
+
+import itertools
+import json
+import math
+import os
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+import oracle.dsv4_oracle as O
+
+RNG = np.random.default_rng(1234)
+
+
+# ----------------------------------------------------------------- codecs
+def test_e4m3_decode_all_codes_match_library():
+    codes = np.arange(256, dtype=np.uint8)
+    lib = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    ours = O.e4m3_decode(codes)
+    nan = np.isnan(lib)
+    assert np.array_equal(np.isnan(ours), nan)
+    assert np.array_equal(ours[~nan], lib[~nan])
+    assert set(np.flatnonzero(nan)) == {0x7F, 0xFF}
+    assert ours[0x7E] == 448.0 and ours[0x01] == 2.0 ** -9 and ours[0x08] == 2.0 ** -6
+
+
+def _fp32_cases(n):
+    vals = O.E4M3_VALUES[:0x7F]
+    mids = (vals[1:] + vals[:-1]) / 2  # exact ties
+    x = np.concatenate([
+        RNG.standard_normal(n) * 40.0,
+        RNG.standard_normal(n) * 0.01,             # subnormal range
+        RNG.uniform(-448, 448, n),
+        mids, -mids, vals, -vals,
+        np.nextafter(mids.astype(np.float32), np.float32(np.inf)),
+        np.nextafter(mids.astype(np.float32), np.float32(-np.inf)),
+    ]).astype(np.float32)
+    return x
+
+
+def test_e4m3_encode_matches_library_in_range():
+    x = _fp32_cases(300_000)
+    lib = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(O.e4m3_encode(x), lib)
+
+
+def test_e4m3_encode_saturates_and_keeps_zero_sign():
+    x = np.array([448.0, 449.0, 464.0, 1e30, -500.0, -1e-30, 1e-30, 0.0, -0.0], np.float32)
+    got = O.e4m3_encode(x)
+    assert list(got) == [0x7E, 0x7E, 0x7E, 0x7E, 0xFE, 0x80, 0x00, 0x00, 0x80]
+
+
+def test_bf16_encode_matches_library():
+    x = np.concatenate([RNG.standard_normal(200_000) * 10 ** RNG.uniform(-8, 8, 200_000),
+                        (np.arange(1, 5000) * 2.0 ** -8 + 1.0 + 2.0 ** -9)]).astype(np.float32)
+    lib = torch.from_numpy(x).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(O.bf16_encode(x), lib)
+    assert np.array_equal(O.bf16_decode(lib), torch.from_numpy(lib.view(np.int16)).view(torch.bfloat16).double().numpy())
+
+
+def test_fp8_store_scale_and_roundtrip():
+    x = RNG.standard_normal(512) * 3.0
+    codes, scale, dec = O.store(x, "fp8")
+    amax = np.float32(np.max(np.abs(np.float32(x))))
+    assert scale == np.float32(amax / np.float32(448.0))
+    assert O.E4M3_VALUES[codes[np.argmax(np.abs(x))] & 0x7F] == 448.0
+    # e4m3 keeps 3 mantissa bits: relative error <= 2^-4 above the subnormal range
+    big = np.abs(x) > 2.0 ** -6 * float(scale)
+    assert np.all(np.abs(dec[big] - x[big]) <= 2.0 ** -4 * np.abs(x[big]) + 1e-12)
+    codes0, scale0, dec0 = O.store(np.zeros(8), "fp8")
+    assert scale0 == 1.0 and np.all(codes0 == 0) and np.all(dec0 == 0)
+
+
+# ----------------------------------------------------------------- pool / norm / rope
+def test_gated_pool_closed_forms():
+    kv = RNG.standard_normal((4, 6))
+    # equal logits -> arithmetic mean
+    assert np.allclose(O.gated_pool(kv, np.zeros((4, 6))), kv.mean(axis=0), atol=1e-15)
+    # one token 60 above the rest -> that token, to within e^-60
+    g = RNG.standard_normal((4, 6))
+    g[2] += 60.0 + (g.max(axis=0) - g[2])
+    assert np.max(np.abs(O.gated_pool(kv, g) - kv[2])) <= 4 * math.exp(-60) * np.max(np.abs(kv))
+    # m = 1 -> identity
+    assert np.allclose(O.gated_pool(kv[:1], g[:1]), kv[0], atol=0)
+    # two tokens: hand-computed softmax weight
+    kv2 = np.array([[1.0], [3.0]])
+    g2 = np.array([[0.0], [math.log(3.0)]])  # weights 1/4, 3/4
+    assert abs(O.gated_pool(kv2, g2)[0] - (0.25 * 1 + 0.75 * 3)) < 1e-15
+    # scalar gate (G = 1) is the broadcast of a per-channel gate
+    gs = RNG.standard_normal((4, 1))
+    assert np.allclose(O.gated_pool(kv, gs), O.gated_pool(kv, np.repeat(gs, 6, axis=1)), atol=1e-15)
+    # channels are independent: permuting channels permutes the output
+    perm = RNG.permutation(6)
+    assert np.allclose(O.gated_pool(kv[:, perm], g[:, perm]), O.gated_pool(kv, g)[perm])
+
+
+def test_rms_norm_closed_forms():
+    x = np.array([3.0, 4.0])
+    assert np.allclose(O.rms_norm(x, np.ones(2), 0.0), x / math.sqrt(12.5), atol=1e-15)
+    y = RNG.standard_normal(512)
+    out = O.rms_norm(y, np.full(512, 2.5), 1e-6)
+    assert abs(np.sqrt(np.mean(out ** 2)) - 2.5 * math.sqrt(np.mean(y ** 2) / (np.mean(y ** 2) + 1e-6))) < 1e-12
+    assert np.allclose(O.rms_norm(7.0 * y, np.ones(512), 0.0), O.rms_norm(y, np.ones(512), 0.0), atol=1e-13)
+    g = RNG.standard_normal(512)
+    assert np.allclose(O.rms_norm(y, g, 0.0), O.rms_norm(y, np.ones(512), 0.0) * g, atol=1e-14)
+
+
+def test_rope_hand_example():
+    # D = 6, r = 4: dims 0,1 untouched; pairs (2,3) by pos*1, (4,5) by pos*10000^(-1/2)
+    x = np.array([5.0, -7.0, 1.0, 0.0, 0.0, 1.0])
+    y = O.apply_rope(x, 1, 4, 10000.0)
+    want = np.array([5.0, -7.0, math.cos(1.0), math.sin(1.0), -math.sin(0.01), math.cos(0.01)])
+    assert np.allclose(y, want, atol=1e-15)
+    assert np.allclose(O.rope_inv_freq(4, 10000.0), [1.0, 0.01], atol=1e-18)
+
+
+def test_rope_rotation_properties():
+    x = RNG.standard_normal((3, 128))
+    y = RNG.standard_normal((3, 128))
+    for p in (0, 1, 4095, 131071, 1 << 20):
+        r = O.apply_rope(x, p, 64, 10000.0)
+        assert np.allclose(np.linalg.norm(r, axis=1), np.linalg.norm(x, axis=1), rtol=1e-13)
+        assert np.allclose(O.apply_rope(r, p, 64, 10000.0, inverse=True), x, atol=1e-12)
+        assert np.array_equal(r[:, :64], x[:, :64])
+    # <R_a x, R_b y> depends only on a - b
+    a = np.einsum("ij,ij->i", O.apply_rope(x, 1000, 64, 1e4), O.apply_rope(y, 900, 64, 1e4))
+    b = np.einsum("ij,ij->i", O.apply_rope(x, 100, 64, 1e4), O.apply_rope(y, 0, 64, 1e4))
+    assert np.allclose(a, b, atol=1e-11)
+
+
+def test_rope_angles_at_one_million_match_high_precision():
+    mpmath.mp.dps = 40
+    p, r = (1 << 20) + 7, 64
+    x = np.zeros(r)
+    x[0::2] = 1.0  # every pair = (1, 0) -> (cos a, sin a)
+    y = O.apply_rope(x, p, r, 10000.0)
+    for i in range(r // 2):
+        a = mpmath.mpf(p) * mpmath.power(10000, mpmath.mpf(-2 * i) / r)
+        assert abs(y[2 * i] - float(mpmath.cos(a))) < 1e-9
+        assert abs(y[2 * i + 1] - float(mpmath.sin(a))) < 1e-9
+
+
+# ----------------------------------------------------------------- compressor
+def _cache(m, D, dtype, B=1, blocks=8, seed=0):
+    rng = np.random.default_rng(seed)
+    pp = O.PAGE_POSITIONS // m
+    num_pages = B * blocks + 2
+    bt = rng.permutation(num_pages)[: B * blocks].reshape(B, blocks).astype(np.int32)
+    pages = np.zeros((num_pages, pp, D), dtype=O.CODE_DTYPE[dtype])
+    return O.PagedCache(dtype, m, D, pages, np.ones((num_pages, pp), np.float32), bt)
+
+
+def test_compressor_streaming_is_chunking_invariant():
+    m, D, T = 4, 16, 61
+    kv = RNG.standard_normal((T, D)).astype(np.float32)
+    g = RNG.standard_normal((T, D)).astype(np.float32)
+    gamma = 1 + 0.1 * RNG.standard_normal(D)
+    outs = []
+    for cuts in ([0, T], [0, 37, T], list(range(T + 1))):
+        st = O.CompressorState(m, D, D, np.zeros((1, m, 2 * D), np.float32))
+        c = _cache(m, D, "f32")
+        for a, b in zip(cuts[:-1], cuts[1:]):
+            O.compress_tokens(st, c, 0, a, kv[a:b], g[a:b], gamma, 1e-6, 8, 1e4)
+        outs.append((c.read(0, np.arange(T // m)), st.buf.copy()))
+    for e, s in outs[1:]:
+        assert np.array_equal(e, outs[0][0]) and np.array_equal(s, outs[0][1])
+    # the ring keeps the last T % m tokens in their slots
+    tail = np.arange(T - T % m, T)
+    assert np.array_equal(outs[0][1][0, tail % m, :D], kv[tail])
+    # entry b is exactly the formula on tokens 4b..4b+3
+    b = 9
+    want = O.apply_rope(O.rms_norm(O.gated_pool(kv[4 * b:4 * b + 4], g[4 * b:4 * b + 4]), gamma, 1e-6),
+                        4 * b, 8, 1e4)
+    assert np.allclose(outs[0][0][b], O.f32(want), atol=0)
+
+
+def test_compress_block_with_m1_is_the_window_key():
+    kv = RNG.standard_normal(32)
+    gamma = RNG.standard_normal(32)
+    for t in (0, 5, 1000):
+        a = O.compress_block(kv[None], RNG.standard_normal((1, 32)), t, 1, gamma, 1e-6, 16, 1e4)
+        assert np.allclose(a, O.window_key(kv, t, gamma, 1e-6, 16, 1e4), atol=1e-14)
+
+
+# ----------------------------------------------------------------- indexer / top-k
+def test_indexer_scores_brute_force():
+    q = RNG.standard_normal((3, 5))
+    w = RNG.standard_normal(3)
+    k = RNG.standard_normal((7, 5))
+    want = []
+    for j in range(7):
+        s = 0.0
+        for h in range(3):
+            dot = sum(q[h, c] * k[j, c] for c in range(5))
+            s += w[h] * (dot if dot > 0 else 0.0)
+        want.append(s)
+    assert np.allclose(O.indexer_scores(q, w, k), want, atol=1e-14)
+    # every q.k < 0 -> every score is 0 (a full tie)
+    kneg = -np.abs(k)
+    assert np.all(O.indexer_scores(np.abs(q), w, kneg) == 0.0)
+
+
+def _check_topk_property(s, k, idx):
+    n = len(s)
+    sel = [int(j) for j in idx if j >= 0]
+    assert len(sel) == min(k, n) and len(set(sel)) == len(sel)
+    assert all(j == -1 for j in idx[len(sel):])
+    rest = set(range(n)) - set(sel)
+    for a in sel:
+        for b in rest:
+            assert s[a] > s[b] or (s[a] == s[b] and a < b)
+
+
+def test_topk_selection_property_and_ties():
+    for n, k in ((50, 7), (5, 8), (64, 64), (200, 17)):
+        s = RNG.integers(-3, 4, n).astype(np.float64)  # many exact ties
+        _check_topk_property(s, k, O.topk_select(s, k))
+        s = RNG.standard_normal(n)
+        _check_topk_property(s, k, O.topk_select(s, k))
+    # brute force over all subsets on a tiny case
+    s = np.array([0.5, 2.0, 2.0, -1.0, 0.5, 3.0])
+    best = max(itertools.combinations(range(6), 3), key=lambda c: sorted(((s[j], -j) for j in c), reverse=True))
+    assert set(O.topk_select(s, 3)) == set(best) == {5, 1, 2}
+    assert list(O.topk_select(np.zeros(5), 3)) == [0, 1, 2]
+
+
+# ----------------------------------------------------------------- attention
+def test_shared_kv_attention_matches_library_sdpa():
+    H, D, N, r = 8, 64, 37, 32
+    q = RNG.standard_normal((H, D))
+    keys = RNG.standard_normal((N, D))
+    p = 12345
+    tau = 1 / math.sqrt(D)
+    got = O.shared_kv_attention(q, p, keys, tau, r, 1e4)
+    qr = torch.from_numpy(O.apply_rope(q, p, r, 1e4))[None, :, None, :]  # [1, H, 1, D]
+    K = torch.from_numpy(keys)[None, None].expand(1, H, N, D)
+    o = torch.nn.functional.scaled_dot_product_attention(qr, K, K, scale=tau)[0, :, 0].numpy()
+    assert np.allclose(got, O.apply_rope(o, p, r, 1e4, inverse=True), atol=1e-12)
+
+
+def _tiny_layer(kind, m, W, k, D=32, H=4, B=1, ctx_blocks=8, d_I=8, H_I=2):
+    cfg = O.LayerConfig(kind=kind, m=m, H=H, D=D, W=W, k=k, H_I=H_I, d_I=d_I, rope_dims=16,
+                        idx_rope_dims=4, eps=1e-6)
+    st = O.LayerState(cfg=cfg, gamma=1 + 0.1 * RNG.standard_normal(D),
+                      main_state=O.CompressorState(m, D, D, np.zeros((B, m, 2 * D), np.float32)),
+                      main_cache=_cache(m, D, "f32", B, ctx_blocks),
+                      window=O.WindowRing("f32", W, D, np.zeros((B, W, D), np.float32), np.ones((B, W), np.float32)))
+    if kind == "c4":
+        st.gamma_idx = np.ones(d_I)
+        st.idx_state = O.CompressorState(m, d_I, d_I, np.zeros((B, m, 2 * d_I), np.float32))
+        st.idx_cache = _cache(m, d_I, "f32", B, ctx_blocks, seed=1)
+    return st
+
+
+def _run_tokens(layer, T):
+    """Decode T tokens one at a time; return inputs of the last step."""
+    c = layer.cfg
+    for t in range(T):
+        step = O.StepInputs(pos=np.array([t]), kv=RNG.standard_normal((1, c.D)),
+                            gate=RNG.standard_normal((1, c.D)), q=RNG.standard_normal((1, c.H, c.D)),
+                            q_idx=RNG.standard_normal((1, c.H_I, c.d_I)), w=RNG.standard_normal((1, c.H_I)),
+                            idx_kv=RNG.standard_normal((1, c.d_I)), idx_gate=RNG.standard_normal((1, c.d_I)))
+        O.decode_update(layer, step)
+    return step
+
+
+def test_inverse_rope_end_to_end_single_key():
+    # only the current token is visible: n_c = floor(6/128) = 0, W = 1
+    layer = _tiny_layer("c128", 128, 1, 0)
+    step = _run_tokens(layer, 6)
+    o, sel, _ = O.decode_attend(layer, step)[0]
+    want = O.rms_norm(O.f32(O.f32(step.kv[0])), layer.gamma, 1e-6)  # window stores float32
+    assert sel.shape[0] == 0
+    assert np.allclose(o, np.broadcast_to(want, o.shape), atol=2e-6)
+
+
+def test_window_covering_context_is_dense_causal_attention():
+    # C128 with p+1 < m: no compressed entry, window >= p+1 -> causal attention over all raw keys
+    layer = _tiny_layer("c128", 128, 64, 0)
+    T = 40
+    kvs = []
+    c = layer.cfg
+    for t in range(T):
+        step = O.StepInputs(pos=np.array([t]), kv=RNG.standard_normal((1, c.D)),
+                            gate=RNG.standard_normal((1, c.D)), q=RNG.standard_normal((1, c.H, c.D)))
+        O.decode_update(layer, step)
+        kvs.append(step.kv[0])
+    keys = np.stack([O.f32(O.window_key(kv, t, layer.gamma, 1e-6, 16, 1e4)) for t, kv in enumerate(kvs)])
+    o, _, _ = O.decode_attend(layer, step)[0]
+    qr = torch.from_numpy(O.apply_rope(step.q[0], T - 1, 16, 1e4))[None, :, None, :]
+    K = torch.from_numpy(keys.astype(np.float64))[None, None].expand(1, c.H, T, c.D)
+    ref = torch.nn.functional.scaled_dot_product_attention(qr, K, K, scale=c.tau)[0, :, 0].numpy()
+    assert np.allclose(o, O.apply_rope(ref, T - 1, 16, 1e4, inverse=True), atol=1e-12)
+
+
+def test_topk_covering_all_entries_is_dense_over_window_and_entries():
+    # C4 with k >= n_c and W >= p+1: attention over window U all compressed entries
+    layer = _tiny_layer("c4", 4, 64, 64)
+    step = _run_tokens(layer, 43)
+    p = 42
+    n_c = O.visible_entries(p, 4)
+    assert n_c == 10
+    o, sel, _ = O.decode_attend(layer, step)[0]
+    assert sorted(sel) == list(range(n_c))
+    keys = np.concatenate([layer.window.read(0, np.arange(0, p + 1)), layer.main_cache.read(0, np.arange(n_c))])
+    assert np.allclose(o, O.shared_kv_attention(step.q[0], p, keys, layer.cfg.tau, 16, 1e4), atol=1e-13)
+    # m = 1 compression is the identity on raw keys: entries equal window keys
+    l1 = _tiny_layer("c4", 1, 64, 64)
+    _run_tokens(l1, 20)
+    assert np.allclose(l1.main_cache.read(0, np.arange(20)), l1.window.read(0, np.arange(20)), atol=0)
+
+
+def test_visible_counts_of_the_workloads(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "layer_shapes.json")))
+    assert g["page_positions"] == O.PAGE_POSITIONS
+    # the decode token at position L sees floor((L+1)/m) complete blocks
+    assert O.visible_entries(4096, g["c4_ratio"]) == 1024
+    assert O.visible_entries(65536, g["c128_ratio"]) == 512
+    assert O.visible_entries(131072, g["c4_ratio"]) == 32768
+    assert O.visible_entries(1 << 20, g["c4_ratio"]) == 262144
+    assert O.visible_entries(1 << 20, g["c128_ratio"]) == 8192
+    assert O.visible_entries((1 << 20) + 3, 4) == 262145   # first new C4 entry at step 3
+    assert list(O.window_positions(5, g["swa_window"])) == list(range(6))
+    assert len(O.window_positions(10_000, g["swa_window"])) == 128
+
+
+# ----------------------------------------------------------------- sizing
+def test_kv_state_sizing_reproduces_the_page(golden_dir):
+    g = json.load(open(os.path.join(golden_dir, "kv_state_sizing.json")))
+    L = g["context_tokens"]
+    gib = float(1 << 30)
+    v32 = O.kv_state_bytes(L, [(1, 576 + 128, 0, 0)] * 61, g["bytes_per_value"]) / gib
+    v4 = O.kv_state_bytes(L, [(4, 512 + 128, 0, 0)] * 30 + [(128, 512, 0, 0)] * 31, g["bytes_per_value"]) / gib
+    assert round(v32, 1) == g["v32_gib"]
+    assert round(v4, 2) == g["v4_gib"]
+    assert round(v32 / v4, 1) == g["ratio"]
