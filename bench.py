@@ -1,0 +1,387 @@
+#!/usr/bin/env python
+"""Decode-step benchmark of the hybrid-attention library on B200.
+
+Workload (per GPU): one C4 layer decode step for B = 32 sequences at a 131072-token context
+(32768 fp8 C4 entries per sequence, top-512 of a 64-head x 128-dim fp8 lightning indexer,
+a 128-token fp8 sliding window, 64 query heads, KV dim 512, bf16 queries and outputs), on
+seeded synthetic inputs. Each step appends one token per sequence; positions cycle over
+131072..131583 so the context stays at 131K.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+With N > 1 (launched by torchrun) every rank runs its own 32 sequences (weak scaling, no
+data-path collective); the step time is the max over ranks. Rank 0 prints one JSON line.
+"""
+
+from __future__ import annotations
+
+import argparse
+import ctypes as C
+import json
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+B_PER_GPU = 32
+CONTEXT = 131072
+POS_CYCLE = 512
+N_INPUT_SETS = 8
+FLUSH_BYTES = 256 << 20
+METRIC = "hybrid-attn decode tokens/s (C4 layer, 131072-token context, top-512 + SWA-128)"
+UNIT = "tokens/s"
+
+SPEC_ROWS = dict(D=512, H=64, k=512, W=128, H_I=64, d_I=128)
+
+
+def algorithmic_bytes_per_seq(n_c: int) -> dict:
+    """Bytes one sequence's decode step must move (fp8 caches with a 4-byte row scale).
+
+    indexer: every visible indexer key row (128 B + scale); attention: the k selected
+    rows and the W window rows (512 B + scale), the bf16 query and output; updates:
+    the new token's kv/gate and indexer kv/gate (bf16) read, the two compressor ring
+    slots (float32) and the window row written; the indexer query, its scales and weights.
+    """
+    D, H, k, W, H_I, d_I = (SPEC_ROWS[x] for x in ("D", "H", "k", "W", "H_I", "d_I"))
+    idx = n_c * (d_I + 4)
+    attn = (k + W) * (D + 4) + 2 * H * D * 2
+    upd = 2 * D * 2 + 2 * d_I * 2 + 2 * D * 4 + 2 * d_I * 4 + (D + 4)
+    qidx = H_I * d_I + H_I * 4 + H_I * 2
+    return dict(indexer=idx + qidx, attention=attn, updates=upd, total=idx + qidx + attn + upd)
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    def __init__(self, gpu_id: str):
+        self.gpu_id = gpu_id
+        self.proc = None
+
+    def __enter__(self):
+        q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={q}", "--format=csv,noheader,nounits",
+                                          "-lms", "100", "-i", self.gpu_id], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        self.rows = []
+        if self.proc is None:
+            return
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 9:
+                self.rows.append(parts)
+
+    def summary(self, t_start: float, t_end: float) -> dict:
+        rows = getattr(self, "rows", [])
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i, v in enumerate(r[5:9]) if v.lower() == "active"})
+        load = sorted(sm)[len(sm) // 2:] if sm else []
+        return {"sm_mhz": float(np.median(load)) if load else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- distributed
+def dist_setup(n_gpus: int):
+    import torch
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(la, steps, budget_s: float, min_seqs: int = 2):
+    """Time the oracle's decode step on whole sequences until budget_s is spent."""
+    import oracle.dsv4_oracle as O
+    from oracle import adapters as OA
+
+    spec = la.spec
+    ol = OA.layer_state(la)
+    oin = OA.step_inputs(spec, steps[0])
+    done, t0 = 0, time.perf_counter()
+    O.decode_update(ol, oin)  # the update part of every sequence (cheap)
+    for s in range(la.B):
+        O.decode_attend(ol, oin, [s])
+        done += 1
+        if done >= min_seqs and time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return done, dt
+
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:  # noqa: BLE001
+        return 1
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args):
+    import torch
+
+    import compressed_sparse_kv_dsv4_b200 as dsv4
+    from compressed_sparse_kv_dsv4_b200 import _abi as A
+    import synthetic as W
+
+    rank, world, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    lib = dsv4.load()
+    la, sets = W.c4_sparse(seed=2 + 1000 * rank, B=B_PER_GPU, context=CONTEXT, steps=N_INPUT_SETS)
+    spec = la.spec
+    dl = dsv4.DeviceLayer.from_arrays(la, dev)
+    dsteps = [dsv4.DeviceStep.from_arrays(spec, st, dev) for st in sets]
+    total = args.warmup + args.steps
+    pos_table = torch.tensor([[CONTEXT + (i % POS_CYCLE)] * B_PER_GPU for i in range(total)],
+                             dtype=torch.int32, device=dev)
+    ws = dl.workspace(B_PER_GPU)
+    L = dl.struct()
+    stream = torch.cuda.current_stream(dev)
+    sh = C.c_void_p(stream.cuda_stream)
+    structs = []
+    for i in range(total):
+        ds = dsteps[i % N_INPUT_SETS]
+        S = ds.struct()
+        S.pos = pos_table[i].data_ptr()
+        structs.append(S)
+    flush = torch.empty(FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(i):
+        A.check("dsv4_hybrid_decode", lib.dsv4_hybrid_decode(C.byref(L), C.byref(structs[i]),
+                                                              C.c_void_p(ws.data_ptr()), ws.numel(), sh))
+
+    for i in range(args.warmup):
+        flush.fill_(i & 0xFF)
+        step(i)
+    torch.cuda.synchronize()
+    ev0 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ev1 = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    with ClockSampler(gpu_id) as clk:
+        barrier(world)
+        torch.cuda.synchronize()
+        t_a = time.time()
+        for j in range(args.steps):
+            flush.fill_(j & 0xFF)
+            ev0[j].record(stream)
+            step(args.warmup + j)
+            ev1[j].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        t_b = time.time()
+    times = np.array([ev0[j].elapsed_time(ev1[j]) for j in range(args.steps)])
+    ms_local = float(times.mean())
+    ms = max_over_ranks(ms_local, world)
+    status = int(dsteps[0].d_status.item())
+
+    # ---- dominant kernel alone: the lightning indexer + top-k, same launch configuration
+    st0 = dsteps[0]
+    n_c = CONTEXT // spec.m
+    n_ent = torch.full((B_PER_GPU,), n_c, dtype=torch.int32, device=dev)
+    idx_out = torch.empty((B_PER_GPU, spec.k), dtype=torch.int32, device=dev)
+    from compressed_sparse_kv_dsv4_b200.binding import indexer_args
+    ia = indexer_args(st0.q_idx, st0.w, dl.idx_cache, n_ent, spec.k, q_dtype="fp8", w_dtype="bf16",
+                      q_scale=st0.q_idx_scale, idx=idx_out, d_status=st0.d_status)
+    iws = torch.empty(lib.dsv4_indexer_workspace_size(C.byref(ia)), dtype=torch.uint8, device=dev)
+    k_iters = max(10, min(args.steps, 200))
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(k_iters)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(k_iters)]
+    for j in range(3):
+        lib.dsv4_indexer_topk(C.byref(ia), C.c_void_p(iws.data_ptr()), iws.numel(), sh)
+    for j in range(k_iters):
+        flush.fill_(j & 0xFF)
+        e0[j].record(stream)
+        A.check("dsv4_indexer_topk", lib.dsv4_indexer_topk(C.byref(ia), C.c_void_p(iws.data_ptr()), iws.numel(), sh))
+        e1[j].record(stream)
+    torch.cuda.synchronize()
+    ix_ms = float(np.mean([e0[j].elapsed_time(e1[j]) for j in range(k_iters)]))
+
+    # ---- end to end through the public API: inputs from pinned host memory, output back
+    host_in = []
+    for ds in dsteps:
+        tensors = [ds.kv, ds.gate, ds.idx_kv, ds.idx_gate, ds.q, ds.q_idx, ds.q_idx_scale, ds.w]
+        host_in.append([t.cpu().pin_memory() for t in tensors])
+    out_host = torch.empty(dsteps[0].out.shape, dtype=dsteps[0].out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host_in[0]) + B_PER_GPU * 4
+    d2h = out_host.numel() * out_host.element_size()
+    pos_host = pos_table.cpu().pin_memory()
+    pos_dev = torch.empty(B_PER_GPU, dtype=torch.int32, device=dev)
+    e2e_steps = max(10, min(args.steps, 200))
+    f0 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    f1 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
+    for j in range(e2e_steps):
+        i = args.warmup + j
+        ds = dsteps[i % N_INPUT_SETS]
+        S = structs[i]
+        S.pos = pos_dev.data_ptr()
+        flush.fill_(j & 0xFF)
+        f0[j].record(stream)
+        for dst, src in zip([ds.kv, ds.gate, ds.idx_kv, ds.idx_gate, ds.q, ds.q_idx, ds.q_idx_scale, ds.w],
+                            host_in[i % N_INPUT_SETS]):
+            dst.copy_(src, non_blocking=True)
+        pos_dev.copy_(pos_host[i], non_blocking=True)
+        step(i)
+        out_host.copy_(ds.out, non_blocking=True)
+        f1[j].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(float(np.mean([f0[j].elapsed_time(f1[j]) for j in range(e2e_steps)])), world)
+
+    if rank != 0:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+        return
+
+    byts = algorithmic_bytes_per_seq(n_c)
+    step_bytes = byts["total"] * B_PER_GPU
+    ix_bytes = byts["indexer"] * B_PER_GPU
+    peaks = {}
+    try:
+        peaks = json.load(open(os.path.join(ROOT, "MEASURED_PEAKS.json")))
+        hbm_peak, peak_src = float(peaks["hbm_gbs"]), "measured"
+    except Exception:  # noqa: BLE001
+        hbm_peak, peak_src = 6650.0, "fallback"
+    ix_gbs = ix_bytes / (ix_ms * 1e-3) / 1e9
+    step_gbs = step_bytes / (ms * 1e-3) / 1e9
+    traffic = None
+    tfile = os.path.join(ROOT, "profiles", "indexer_traffic.json")
+    if os.path.exists(tfile):
+        try:
+            traffic = json.load(open(tfile)).get("dram_bytes_per_launch")
+        except Exception:  # noqa: BLE001
+            traffic = None
+    value = world * B_PER_GPU / (ms * 1e-3)
+    line = {
+        "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8 indexer + bf16 attention (fp32 accumulate)", "data": "synthetic",
+        "config": {"workload": "c4_sparse_131k", "batch_per_gpu": B_PER_GPU, "global_batch": world * B_PER_GPU,
+                   "context": CONTEXT, "c4_entries": n_c, "topk": spec.k, "window": spec.W, "heads": spec.H,
+                   "kv_dim": spec.D, "indexer": f"{spec.H_I} heads x {spec.d_I} fp8", "cache": "fp8 e4m3 + fp32 row scale",
+                   "parallelism": f"dp{world} (independent sequences)", "l2": "flushed between steps (256 MiB write)",
+                   "positions": f"advance by one per step, cycling over {CONTEXT}..{CONTEXT + POS_CYCLE - 1}"},
+        "hbm": {"step_algorithmic_bytes": step_bytes, "achieved_gbs": round(step_gbs, 1),
+                "pct_of_8tbs": round(100 * step_gbs / 8000.0, 1),
+                "pct_of_measured_copy": round(100 * step_gbs / hbm_peak, 1)},
+        "roofline": {"kernel": "indexer_tc_kernel (+ top-k select)", "bound": "hbm", "achieved": round(ix_gbs, 1),
+                     "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s", "frac": round(ix_gbs / hbm_peak, 4),
+                     "traffic": traffic, "algorithmic_bytes_per_launch": ix_bytes, "launch_ms": round(ix_ms, 5)},
+        "e2e": {"value": round(world * B_PER_GPU / (e2e_ms * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
+        "gpu_launches": 5 * args.steps,
+        "clocks": clk.summary(t_a, t_b),
+        "device_status": status,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        seqs, dt = oracle_sample(la, sets, budget_s=args.cpu_budget)
+        line["cpu_baseline"] = {"value": round(seqs / dt, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                                "host_cores": os.cpu_count(),
+                                "sample": f"{seqs} of {B_PER_GPU} sequences of one decode step (float64 oracle)"}
+    print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import synthetic as W
+
+    la, sets = W.c4_sparse(seed=2, B=B_PER_GPU, context=CONTEXT, steps=1)
+    per_step = []
+    budget = max(1.0, 120.0 / max(1, args.steps + args.warmup))
+    for i in range(args.warmup + args.steps):
+        seqs, dt = oracle_sample(la, sets, budget_s=budget, min_seqs=1)
+        if i >= args.warmup:
+            per_step.append(seqs / dt)
+    value = float(np.mean(per_step))
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * B_PER_GPU / value, 3),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "c4_sparse_131k", "batch_per_gpu": B_PER_GPU, "context": CONTEXT},
+            "cpu_baseline": {"value": round(value, 3), "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": "each step: whole sequences of one C4 decode step until its time budget"},
+            "e2e": {"value": round(value, 3), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,152 @@
+// Host-side interface between the C ABI (api.cu) and the kernel translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+#include "../../include/dsv4.h"
+
+namespace dsv4 {
+
+// number of SMs of the current device (cached per device)
+int sm_count();
+
+// ---------------------------------------------------------------- compressor / window
+struct CompressLaunch {
+  int B;
+  int total_tokens;
+  const void *kv;
+  const void *gate;
+  dsv4_dtype kv_dt;
+  const int32_t *cu_seqlens;
+  const int32_t *start_pos;
+  const float *gamma;
+  float eps;
+  int rope_dims;
+  float rope_base;
+  float *state;
+  int m, D, G;
+  void *pages;
+  float *scales;
+  const int32_t *block_table;
+  int num_pages, max_blocks;
+  dsv4_dtype cache_dt;
+  uint32_t *d_status;
+};
+cudaError_t launch_compress(const CompressLaunch &p, cudaStream_t st);
+
+struct SwaLaunch {
+  int B;
+  int total_tokens;
+  const void *kv;
+  dsv4_dtype kv_dt;
+  const int32_t *cu_seqlens;
+  const int32_t *start_pos;
+  const float *gamma;
+  float eps;
+  int rope_dims;
+  float rope_base;
+  void *rows;
+  float *scales;
+  int W, D;
+  dsv4_dtype ring_dt;
+  uint32_t *d_status;
+};
+cudaError_t launch_swa_insert(const SwaLaunch &p, cudaStream_t st);
+
+// one decode step's state updates: window insert, compressor append(s)
+struct PrologueLaunch {
+  int B;
+  const int32_t *pos;
+  dsv4_dtype kv_dt;
+  // main
+  const void *kv, *gate;
+  const float *gamma;
+  float eps;
+  int rope_dims;
+  float rope_base;
+  float *state;
+  int m, D, G;
+  void *pages;
+  float *scales;
+  const int32_t *block_table;
+  int num_pages, max_blocks;
+  dsv4_dtype cache_dt;
+  void *ring_rows;
+  float *ring_scales;
+  int W;
+  dsv4_dtype ring_dt;
+  // indexer-key compressor (idx_D == 0: none)
+  const void *idx_kv, *idx_gate;
+  const float *gamma_idx;
+  int idx_rope_dims;
+  float *idx_state;
+  int idx_D, idx_G;
+  void *idx_pages;
+  float *idx_scales;
+  const int32_t *idx_block_table;
+  int idx_num_pages, idx_max_blocks;
+  dsv4_dtype idx_dt;
+  uint32_t *d_status;
+};
+cudaError_t launch_decode_prologue(const PrologueLaunch &p, cudaStream_t st);
+
+// ---------------------------------------------------------------- indexer + top-k
+struct IndexerLaunch {
+  int B, H, Dq, k;
+  const void *q;
+  dsv4_dtype q_dt;
+  const float *q_scale;
+  const void *w;
+  dsv4_dtype w_dt;
+  const void *k_pages;
+  const float *k_scales;
+  const int32_t *block_table;
+  int num_pages, max_blocks, m;
+  dsv4_dtype k_dt;
+  const int32_t *n_entries;  // NULL: derived from pos as floor((pos+1)/m)
+  const int32_t *pos;
+  int q_rope_dims;
+  float rope_base;
+  int32_t *idx;
+  float *scores;
+  uint32_t *d_status;
+};
+bool indexer_uses_tensor_cores(const IndexerLaunch &p);
+size_t indexer_workspace_bytes(const IndexerLaunch &p);
+cudaError_t launch_indexer_topk(const IndexerLaunch &p, void *ws, cudaStream_t st);
+
+// ---------------------------------------------------------------- sparse / dense MQA
+struct MqaLaunch {
+  int B, H, D;
+  const void *q;
+  dsv4_dtype q_dt;
+  const int32_t *pos;
+  const void *pages;
+  const float *scales;
+  const int32_t *block_table;
+  int num_pages, max_blocks, m;
+  dsv4_dtype kv_dt;
+  const int32_t *n_entries;  // NULL: derived from pos as floor((pos+1)/m)
+  const int32_t *idx;        // NULL: dense
+  int k;
+  const void *ring_rows;
+  const float *ring_scales;
+  int W;
+  float softmax_scale;
+  int rope_dims;
+  float rope_base;
+  void *out;
+  dsv4_dtype out_dt;
+  float *lse;
+  uint32_t *d_status;
+};
+bool mqa_uses_tensor_cores(const MqaLaunch &p);
+size_t mqa_workspace_bytes(const MqaLaunch &p);
+cudaError_t launch_mqa(const MqaLaunch &p, void *ws, cudaStream_t st);
+
+inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace dsv4

@@ -1,0 +1,285 @@
+"""GPU parity of each entry point of the C ABI against the oracle, on the same bytes.
+
+Sizes span several tiles with ragged tails; edge cases: unaligned prefill starts,
+truncated windows, n_c = 0, n_c <= k, full score ties, -1 padding and an
+out-of-range index in the selection.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import compressed_sparse_kv_dsv4_b200 as dsv4
+import oracle.dsv4_oracle as O
+import synthetic as W
+from oracle import adapters as OA
+from tests.parity import check_output, check_topk, decode_out, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    require_gpu()
+
+
+def _codes_close(gpu_codes, ref_codes, gpu_scales, ref_scales, dtype, ctx):
+    """Rows rounded into a cache dtype by the two sides from slightly different
+    float32 values: equal, or one rounding step apart."""
+    if dtype == "f32":
+        g = np.asarray(gpu_codes, np.float64)
+        r = np.asarray(ref_codes, np.float64)
+        assert np.max(np.abs(g - r)) <= 2e-5 * max(1.0, np.max(np.abs(r))), ctx
+        return
+    if dtype == "bf16":
+        g, r = O.bf16_decode(gpu_codes), O.bf16_decode(ref_codes)
+        assert np.all(np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 1e-30), ctx
+        return
+    gs, rs = np.asarray(gpu_scales, np.float64), np.asarray(ref_scales, np.float64)
+    assert np.all(np.abs(gs - rs) <= 1e-6 * rs), f"{ctx}: scales"
+    g = np.asarray(gpu_codes).astype(np.int32)
+    r = np.asarray(ref_codes).astype(np.int32)
+    same_sign = (g & 0x80) == (r & 0x80)
+    step = np.abs((g & 0x7F) - (r & 0x7F))
+    zero = ((g & 0x7F) == 0) & ((r & 0x7F) <= 1) | ((r & 0x7F) == 0) & ((g & 0x7F) <= 1)
+    ok = (same_sign & (step <= 1)) | zero
+    assert np.all(ok), f"{ctx}: fp8 codes more than one step apart"
+    assert np.mean(g != r) < 0.01, f"{ctx}: too many fp8 rounding differences"
+
+
+# ---------------------------------------------------------------------------- compressor
+@pytest.mark.parametrize("m,cache_dtype,D", [(4, "bf16", 512), (128, "fp8", 512), (4, "fp8", 128), (4, "f32", 32)])
+def test_compress_prefill_matches_oracle(m, cache_dtype, D):
+    rng = W.rng_for(11)
+    lens = np.array([37, 300, 129], dtype=np.int32)
+    start = np.array([0, 37, 5], dtype=np.int32)
+    if m == 128:
+        lens = np.array([300, 129, 411], dtype=np.int32)
+        start = np.array([0, 200, 5], dtype=np.int32)
+    B = len(lens)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    kv_dt = "f32" if cache_dtype == "f32" else "bf16"
+    kv = W.encode_values(W.normal_f32(rng, (T, D)), kv_dt)
+    gate = W.encode_values(W.normal_f32(rng, (T, D)), kv_dt)
+    spec = W.LayerSpec(kind="c128", m=m, H=8, D=D, cache_dtype=cache_dtype, kv_dtype=kv_dt, swa_dtype="bf16")
+    la = W.make_layer(spec, B, int((start + lens).max()) // m + 1, seed=5)
+    la.gamma = (1 + 0.2 * W.normal_f32(rng, (D,))).astype(np.float32)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    dsv4.compress(dsv4.to_device_codes(kv, kv_dt, "cuda"), dsv4.to_device_codes(gate, kv_dt, "cuda"),
+                  torch.from_numpy(cu).cuda(), torch.from_numpy(start).cuda(), dl.state, dl.cache, dl.gamma,
+                  kv_dtype=kv_dt, eps=1e-6, rope_dims=min(64, D // 2), rope_base=1e4, d_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ol = OA.layer_state(la)
+    dec = lambda a: OA.decode_input(a, kv_dt)  # noqa: E731
+    O.compress(dec(kv), dec(gate), cu, start, ol.main_state, ol.main_cache, ol.gamma, 1e-6, min(64, D // 2), 1e4)
+    # the state ring holds exact copies of the inputs
+    assert np.array_equal(dl.state.buf.cpu().numpy(), ol.main_state.buf)
+    pages = dsv4.to_numpy_codes(dl.cache.pages, cache_dtype)
+    scales = dl.cache.scales.cpu().numpy()
+    for s in range(B):
+        for b in range(start[s] // m, (start[s] + lens[s]) // m):
+            pg, sl = ol.main_cache.locate(s, b)
+            _codes_close(pages[pg, sl], ol.main_cache.pages[pg, sl], scales[pg, sl], ol.main_cache.scales[pg, sl],
+                         cache_dtype, f"seq {s} block {b}")
+    # rows that no block wrote keep their bytes
+    untouched = np.ones(pages.shape[:2], bool)
+    for s in range(B):
+        for b in range(start[s] // m, (start[s] + lens[s]) // m):
+            untouched[ol.main_cache.locate(s, b)] = False
+    assert np.array_equal(pages[untouched], la.pages[untouched])
+
+
+def test_compress_prefill_equals_token_by_token():
+    rng = W.rng_for(12)
+    D, m, T = 128, 4, 77
+    kv = W.bf16_bits(W.normal_f32(rng, (T, D)))
+    gate = W.bf16_bits(W.normal_f32(rng, (T, D)))
+    spec = W.LayerSpec(kind="c128", m=m, H=8, D=D, cache_dtype="fp8", kv_dtype="bf16")
+    la = W.make_layer(spec, 1, T // m + 1, seed=6)
+    outs = []
+    for chunks in ([T], [1] * T, [37, 40]):
+        dl = dsv4.DeviceLayer.from_arrays(la)
+        kvd = dsv4.to_device_codes(kv, "bf16", "cuda")
+        gd = dsv4.to_device_codes(gate, "bf16", "cuda")
+        p0 = 0
+        for c in chunks:
+            dsv4.compress(kvd[p0:p0 + c], gd[p0:p0 + c], torch.tensor([0, c], dtype=torch.int32, device="cuda"),
+                          torch.tensor([p0], dtype=torch.int32, device="cuda"), dl.state, dl.cache, dl.gamma,
+                          kv_dtype="bf16", rope_dims=64)
+            p0 += c
+        torch.cuda.synchronize()
+        outs.append((dl.cache.pages.cpu().numpy(), dl.cache.scales.cpu().numpy(), dl.state.buf.cpu().numpy()))
+    for o in outs[1:]:
+        for a, b in zip(o, outs[0]):
+            assert np.array_equal(a, b)
+
+
+@pytest.mark.parametrize("dtype,D", [("fp8", 512), ("bf16", 512), ("f32", 128)])
+def test_swa_insert_matches_oracle(dtype, D):
+    rng = W.rng_for(13)
+    lens = np.array([5, 200, 128], dtype=np.int32)
+    start = np.array([0, 1000, 70], dtype=np.int32)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    kv_dt = "f32" if dtype == "f32" else "bf16"
+    kv = W.encode_values(W.normal_f32(rng, (int(cu[-1]), D)), kv_dt)
+    spec = W.LayerSpec(kind="c128", m=128, H=8, D=D, swa_dtype=dtype, cache_dtype="bf16", kv_dtype=kv_dt)
+    la = W.make_layer(spec, 3, 4, seed=7)
+    la.gamma = (1 + 0.2 * W.normal_f32(rng, (D,))).astype(np.float32)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    dsv4.swa_insert(dsv4.to_device_codes(kv, kv_dt, "cuda"), torch.from_numpy(cu).cuda(),
+                    torch.from_numpy(start).cuda(), dl.ring, dl.gamma, kv_dtype=kv_dt, rope_dims=64)
+    torch.cuda.synchronize()
+    ol = OA.layer_state(la)
+    kvf = OA.decode_input(kv, kv_dt)
+    for s in range(3):
+        for i in range(lens[s]):
+            t = start[s] + i
+            if t >= start[s] + lens[s] - 128:
+                O.swa_insert(ol.window, s, t, kvf[cu[s] + i], ol.gamma, 1e-6, 64, 1e4)
+    rows = dsv4.to_numpy_codes(dl.ring.rows, dtype)
+    sc = dl.ring.scales.cpu().numpy()
+    for s in range(3):
+        for i in range(128):
+            _codes_close(rows[s, i], ol.window.rows[s, i], sc[s, i], ol.window.scales[s, i], dtype, f"seq {s} slot {i}")
+
+
+# ---------------------------------------------------------------------------- indexer
+def _indexer_case(n_list, k, H=64, seed=21, spec=W.C4_SPEC, all_negative=False):
+    B = len(n_list)
+    la = W.make_layer(spec, B, max(n_list) + 1, seed, outlier_frac=0.05)
+    st = W.make_step(spec, B, 0, seed + 1)
+    if all_negative:  # every q.k < 0: all scores are exactly zero
+        st.q_idx = st.q_idx & 0x7F
+        la.idx_pages = la.idx_pages | 0x80
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    q = dsv4.to_device_codes(st.q_idx, spec.q_idx_dtype, "cuda")
+    w = dsv4.to_device_codes(st.w, spec.w_dtype, "cuda")
+    n = torch.tensor(n_list, dtype=torch.int32, device="cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx, scores = dsv4.indexer_topk(q, w, dl.idx_cache, n, k, q_dtype=spec.q_idx_dtype, w_dtype=spec.w_dtype,
+                                    q_scale=torch.from_numpy(st.q_idx_scale).cuda(), d_status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ol = OA.layer_state(la)
+    qd = OA.decode_input(st.q_idx, spec.q_idx_dtype, st.q_idx_scale)
+    wd = OA.decode_input(st.w, spec.w_dtype)
+    return idx.cpu().numpy(), scores.cpu().numpy(), ol, qd, wd
+
+
+@pytest.mark.parametrize("k", [512, 64, 1024])
+def test_indexer_tensor_core_topk_matches_oracle(k):
+    n_list = [130, 1000, 4097, 0, 600]
+    idx, scores, ol, qd, wd = _indexer_case(n_list, k)
+    for s, n in enumerate(n_list):
+        if n == 0:
+            assert np.all(idx[s] == -1)
+            continue
+        ref = O.indexer_scores(qd[s], wd[s], ol.idx_cache.read(s, np.arange(n)))
+        check_topk(idx[s], ref, k, n, f"seq {s}")
+        v = idx[s] >= 0
+        got = scores[s][v]
+        want = ref[idx[s][v]]
+        assert np.all(np.abs(got - want) <= 1e-5 * np.abs(want).max()), f"seq {s}: scores"
+
+
+def test_indexer_full_tie_takes_lowest_indices():
+    idx, scores, ol, qd, wd = _indexer_case([3000, 700], 512, all_negative=True)
+    for s in range(2):
+        assert sorted(idx[s].tolist()) == list(range(512))
+        assert np.all(scores[s] == 0.0)
+
+
+def test_indexer_cuda_core_path_fp32_with_query_rope():
+    spec = W.TINY_SPEC
+    B, n = 2, 1024
+    la = W.make_layer(spec, B, n + 1, 31)
+    st = W.make_step(spec, B, [4096, 777], 32)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    q = torch.from_numpy(st.q_idx).cuda()
+    w = torch.from_numpy(st.w).cuda()
+    pos = torch.from_numpy(st.pos).cuda()
+    n_t = torch.tensor([n, 301], dtype=torch.int32, device="cuda")
+    idx, scores = dsv4.indexer_topk(q, w, dl.idx_cache, n_t, 64, q_dtype="f32", w_dtype="f32", pos=pos,
+                                    q_rope_dims=16)
+    torch.cuda.synchronize()
+    ol = OA.layer_state(la)
+    for s, ns in enumerate([n, 301]):
+        qr = O.apply_rope(st.q_idx[s].astype(np.float64), int(st.pos[s]), 16, 1e4)
+        ref = O.indexer_scores(qr, st.w[s].astype(np.float64), ol.idx_cache.read(s, np.arange(ns)))
+        check_topk(idx[s].cpu().numpy(), ref, 64, ns, f"seq {s}")
+
+
+# ---------------------------------------------------------------------------- attention
+def _mqa_case(spec, B, pos, n_entries, idx=None, seed=41, value_std=1.0):
+    la = W.make_layer(spec, B, max(n_entries) + 1, seed, value_std=value_std, outlier_frac=0.05)
+    st = W.make_step(spec, B, pos, seed + 1, q_std=value_std)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    q = dsv4.to_device_codes(st.q, spec.q_dtype, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    idx_t = None if idx is None else torch.from_numpy(idx.astype(np.int32)).cuda()
+    out, lse = dsv4.sparse_mqa_decode(q, torch.from_numpy(st.pos).cuda(), dl.cache, dl.ring, q_dtype=spec.q_dtype,
+                                      out_dtype=spec.out_dtype, idx=idx_t,
+                                      n_entries=torch.tensor(n_entries, dtype=torch.int32, device="cuda"),
+                                      rope_dims=spec.rope_dims, with_lse=True, d_status=status)
+    torch.cuda.synchronize()
+    ol = OA.layer_state(la)
+    qd = OA.decode_input(st.q, spec.q_dtype)
+    return decode_out(out), lse.cpu().numpy(), status.item(), ol, qd, st
+
+
+def _ref_attention(ol, qd, st, s, sel, spec):
+    p = int(st.pos[s])
+    parts = [ol.window.read(s, O.window_positions(p, spec.W))]
+    if len(sel):
+        parts.append(ol.main_cache.read(s, np.asarray(sel)))
+    keys = np.concatenate(parts)
+    o = O.shared_kv_attention(qd[s], p, keys, 1 / np.sqrt(spec.D), spec.rope_dims, spec.rope_base)
+    qr = O.apply_rope(qd[s], p, spec.rope_dims, spec.rope_base)
+    lg = qr @ keys.T / np.sqrt(spec.D)
+    lse = lg.max(1) + np.log(np.exp(lg - lg.max(1, keepdims=True)).sum(1))
+    return o, lse
+
+
+def test_mqa_tensor_core_dense_bf16():
+    spec = W.C128_SPEC
+    pos = [3, 70000, 65536]           # a truncated window, then full ones
+    n_entries = [0, 300, 513]          # n_c = 0, then ragged chunk tails
+    out, lse, status, ol, qd, st = _mqa_case(spec, 3, pos, n_entries, value_std=1 / np.sqrt(512))
+    assert status == 0
+    for s in range(3):
+        o, l = _ref_attention(ol, qd, st, s, np.arange(n_entries[s]), spec)
+        check_output(out[s], o, "bf16", f"seq {s}")
+        assert np.max(np.abs(lse[s] - l)) < 2e-2
+
+
+def test_mqa_tensor_core_sparse_fp8_with_padding_and_bad_index():
+    spec = W.C4_SPEC
+    B, n_c = 2, 5000
+    rng = np.random.default_rng(5)
+    idx = np.stack([rng.permutation(n_c)[:512] for _ in range(B)]).astype(np.int64)
+    idx[0, 500:] = -1             # padding
+    idx[1, 7] = n_c + 3           # out of range: skipped and reported
+    out, lse, status, ol, qd, st = _mqa_case(spec, B, [20000, 131072], [n_c, n_c], idx=idx)
+    assert status == dsv4._abi.DEV_BAD_INDEX
+    for s in range(B):
+        sel = [j for j in idx[s] if 0 <= j < n_c]
+        o, l = _ref_attention(ol, qd, st, s, sel, spec)
+        check_output(out[s], o, "bf16", f"seq {s}")
+
+
+def test_mqa_cuda_core_fp32():
+    spec = W.TINY_SPEC
+    B = 2
+    rng = np.random.default_rng(6)
+    idx = np.stack([rng.permutation(1024)[:64] for _ in range(B)]).astype(np.int64)
+    idx[1, 60:] = -1
+    out, lse, status, ol, qd, st = _mqa_case(spec, B, [4096, 100], [1024, 1024], idx=idx)
+    assert status == 0
+    for s in range(B):
+        sel = [j for j in idx[s] if j >= 0]
+        o, l = _ref_attention(ol, qd, st, s, sel, spec)
+        check_output(out[s], o, "f32", f"seq {s}")
+        assert np.max(np.abs(lse[s] - l)) < 1e-4
