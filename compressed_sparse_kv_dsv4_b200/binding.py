@@ -284,6 +284,11 @@ def mqa_args(q, pos, cache: DeviceCache, ring: DeviceRing, *, q_dtype: str, out,
                      out=_ptr(out), out_dtype=DT[out_dtype], lse=_ptr(lse), d_status=_ptr(d_status))
 
 
+def mqa_workspace_size(args: A.MqaArgs) -> int:
+    """dsv4_mqa_workspace_size for the marshalled arguments of a sparse_mqa_decode call."""
+    return A.load().dsv4_mqa_workspace_size(C.byref(args))
+
+
 def sparse_mqa_decode(q, pos, cache: DeviceCache, ring: DeviceRing, *, q_dtype: str, out_dtype: str, idx=None,
                       n_entries=None, softmax_scale: float = 0.0, rope_dims: int = 64, rope_base: float = 10000.0,
                       with_lse: bool = False, d_status=None, workspace=None, stream=None):

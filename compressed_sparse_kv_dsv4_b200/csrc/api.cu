@@ -52,7 +52,7 @@ bool valid_cache(const dsv4_paged_cache &c, bool need_scales_if_fp8 = true) {
   if (!c.pages || !c.block_table || c.num_pages <= 0 || c.max_blocks <= 0 || c.dim <= 0) return false;
   if (!pow2(c.m) || c.m > DSV4_PAGE_POSITIONS || !valid_dtype(c.dtype)) return false;
   if (!aligned16(c.pages) || (c.dim * dsize(c.dtype)) % 16 != 0) return false;
-  if (c.dtype == DSV4_FP8E4M3 && need_scales_if_fp8 && !c.scales) return false;
+  if (c.dtype == DSV4_FP8E4M3 && need_scales_if_fp8 && (!c.scales || !aligned16(c.scales))) return false;
   return true;
 }
 

@@ -63,13 +63,13 @@ __device__ void pool_block(const TokenSource &src, int64_t b, float *e, float *s
       float v[8], g[8];
       if (t < src.p0) {
         const float *row = src.state + static_cast<size_t>(t % m) * (D + G);
-        load_row_f<8>(row, DSV4_F32, static_cast<size_t>(cg) * 8, v);
-        if (G == D) {
+        if (G == D) {  // rows of 2D floats: 16-byte aligned
+          load_row_f<8>(row, DSV4_F32, static_cast<size_t>(cg) * 8, v);
           load_row_f<8>(row + D, DSV4_F32, static_cast<size_t>(cg) * 8, g);
-        } else {
+        } else {  // rows of D + 1 floats: scalar loads
           const float g0 = row[D];
 #pragma unroll
-          for (int i = 0; i < 8; ++i) g[i] = g0;
+          for (int i = 0; i < 8; ++i) { v[i] = row[cg * 8 + i]; g[i] = g0; }
         }
       } else {
         const size_t r = static_cast<size_t>(src.row0 + (t - src.p0));
@@ -234,10 +234,10 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressLaunch
         finish_and_store(e, p.D, p.gamma, p.eps, b * p.m, p.rope_dims, p.rope_base, p.cache_dt, row, sp, red);
     }
     if (i == 0) {
-      // tokens of the trailing incomplete block go to the state ring, after the first
-      // block (which may read ring slots) has been pooled
+      // the state ring keeps the latest m tokens (slot t % m); written after the first
+      // block, the only one that may read ring slots, has been pooled
       __syncthreads();
-      int64_t t0 = (r.p1 / p.m) * p.m;
+      int64_t t0 = r.p1 - p.m;
       if (t0 < r.p0) t0 = r.p0;
       const int width = p.D + p.G;
       for (int64_t t = t0; t < r.p1; ++t) {

@@ -90,6 +90,41 @@ __device__ __forceinline__ const uint8_t *key_row(const MqaLaunch &p, int b, con
   return static_cast<const uint8_t *>(p.pages) + row * p.D * esz;
 }
 
+// prefix[b] = number of 64-key chunks of sequences 0..b-1, prefix[B] = total; computed by
+// every thread of the CTA (contiguous slices of sequences, then a scan of the slices).
+// red: blockDim.x scratch values.
+__device__ void chunk_prefix(const MqaLaunch &p, long long *prefix, long long *red, bool report_it) {
+  const int nt = blockDim.x, t = threadIdx.x;
+  const int lo = static_cast<int>((static_cast<long long>(p.B) * t) / nt);
+  const int hi = static_cast<int>((static_cast<long long>(p.B) * (t + 1)) / nt);
+  long long mine = 0;
+  for (int b = lo; b < hi; ++b) {
+    const KeyList L = key_list(p, b, report_it);
+    const long long c = (L.nw + L.nsel + 63) / 64;
+    prefix[b] = c;
+    mine += c;
+  }
+  red[t] = mine;
+  __syncthreads();
+  if (t == 0) {
+    long long acc = 0;
+    for (int i = 0; i < nt; ++i) {
+      const long long v = red[i];
+      red[i] = acc;
+      acc += v;
+    }
+    prefix[p.B] = acc;
+  }
+  __syncthreads();
+  long long acc = red[t];
+  for (int b = lo; b < hi; ++b) {
+    const long long c = prefix[b];
+    prefix[b] = acc;
+    acc += c;
+  }
+  __syncthreads();
+}
+
 __device__ __forceinline__ int find_seq(const long long *prefix, int B, long long g) {
   int lo = 0, hi = B - 1;
   while (lo < hi) {
@@ -104,14 +139,28 @@ __device__ __forceinline__ int find_seq(const long long *prefix, int B, long lon
 
 constexpr int kH = 64, kD = 512, kCh = 64, kThreads = 256;
 constexpr int kAtom = kCh * 128;  // one 64-dim column block of a 64-row tile: 8 KB
+constexpr int kMetaChunks = 8;
 
 struct alignas(1024) MqaSmem {
   uint8_t q[kD / 64][kH * 128];      // 64 KB, K-major SW128, 8 atoms of 64 dims
   uint8_t k[2][kD / 64][kCh * 128];  // 2 x 64 KB
-  uint8_t p[kH * 128];               // 8 KB: P'[64 heads][64 keys] bf16, K-major SW128
+  uint8_t p[kH * 128];               // 8 KB: P[64 heads][64 keys], K-major SW128
   const uint8_t *rowp[2][kCh];
-  float rscale[2][kCh];
+  float rscale[2][kCh];              // row scale of each key (0: no key)
+  // key metadata of up to kMetaChunks consecutive chunks, resolved together so the
+  // idx -> block table -> scale load chain is paid once per batch, not once per chunk
+  const uint8_t *mrow[kMetaChunks * kCh];
+  float mscale[kMetaChunks * kCh];
+  KeyList mkl[kMetaChunks];
+  int mb[kMetaChunks];
+  long long mlc[kMetaChunks];
+  long long meta_first;
+  int meta_n;
   float cs[kD / 2], sn[kD / 2];
+  float qinv[kH];                    // 2^-e of the per-head query scale (fp16 operands)
+  float smax[2][2];                  // per-warp max row scale of a chunk being gathered
+  int ec[2];                         // chunk exponent: K rows hold code * scale * 2^-ec
+  unsigned qmax[kH];
   uint64_t bar_s, bar_o;
   uint32_t tmem_base;
   int abort_flag;
@@ -124,19 +173,68 @@ struct MqaTcParams {
   float *part_ml;  // [B + G][H][2]
 };
 
-__device__ void gather_chunk(const MqaTcParams &P, MqaSmem &S, int b, const KeyList &L, long long lc, int kb) {
+// Operands of the two MMAs. fp8 caches: fp16 (e4m3 -> fp16 is exact, and fp16 keeps 11
+// significand bits of the rotated query and of P); bf16 caches: bf16.
+__device__ __forceinline__ bool fp16_operands(const MqaLaunch &p) { return p.kv_dt == DSV4_FP8E4M3; }
+
+__device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t *>(&h);
+}
+
+// Resolve the row address and scale of every key of chunks [g0, g0 + n) (n <= kMetaChunks).
+__device__ void resolve_meta(const MqaTcParams &P, MqaSmem &S, const long long *prefix, long long g0, long long c1) {
   const MqaLaunch &p = P.a;
   const int tid = threadIdx.x;
-  if (tid < kCh) {
+  const int n = static_cast<int>(c1 - g0 < kMetaChunks ? c1 - g0 : kMetaChunks);
+  if (tid < n) {
+    const int b = find_seq(prefix, p.B, g0 + tid);
+    S.mb[tid] = b;
+    S.mlc[tid] = g0 + tid - prefix[b];
+    S.mkl[tid] = key_list(p, b, false);
+  }
+  __syncthreads();
+  // the cached range changes only after every thread has passed the barrier above, that
+  // is, after every thread has taken its decision to resolve from the old range
+  if (tid == 0) {
+    S.meta_first = g0;
+    S.meta_n = n;
+  }
+  for (int i = tid; i < n * kCh; i += kThreads) {
+    const int c = i / kCh;
+    const KeyList &L = S.mkl[c];
+    const long long t = S.mlc[c] * kCh + (i % kCh);
     float sc = 0.f;
-    const uint8_t *rp = key_row(p, b, L, lc * kCh + tid, &sc);
-    if (lc * kCh + tid >= L.nw + L.nsel) rp = nullptr;
+    const uint8_t *rp = t < L.nw + L.nsel ? key_row(p, S.mb[c], L, t, &sc) : nullptr;
+    S.mrow[i] = rp;
+    S.mscale[i] = rp ? sc : 0.f;
+  }
+  __syncthreads();
+}
+
+// Gather one 64-key chunk into a swizzled K-major tile. For fp8 rows the row scale is
+// folded in: tile row j = code_j * (scale_j * 2^-ec) in fp16, with ec the exponent of the
+// chunk's largest row scale, so every tile value stays within +-448.
+__device__ void gather_chunk(const MqaTcParams &P, MqaSmem &S, const long long *prefix, long long g, long long c1,
+                             int kb) {
+  const MqaLaunch &p = P.a;
+  const int tid = threadIdx.x;
+  if (g < S.meta_first || g >= S.meta_first + S.meta_n) resolve_meta(P, S, prefix, g, c1);
+  if (tid < kCh) {
+    const int i = static_cast<int>(g - S.meta_first) * kCh + tid;
+    const uint8_t *rp = S.mrow[i];
+    const float sc = S.mscale[i];
     S.rowp[kb][tid] = rp;
-    S.rscale[kb][tid] = rp ? sc : 0.f;
+    S.rscale[kb][tid] = sc;
+    const float wm = warp_max(sc);
+    if ((tid & 31) == 0) S.smax[kb][tid >> 5] = wm;
   }
   __syncthreads();
   uint8_t *kt = &S.k[kb][0][0];
   if (p.kv_dt == DSV4_FP8E4M3) {
+    int ec = 0;
+    frexpf(fmaxf(S.smax[kb][0], S.smax[kb][1]), &ec);  // max scale = f * 2^ec, f in [0.5, 1)
+    if (tid == 0) S.ec[kb] = ec;
     uint4 v[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
@@ -147,14 +245,17 @@ __device__ void gather_chunk(const MqaTcParams &P, MqaSmem &S, int b, const KeyL
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int sid = i * kThreads + tid, row = sid >> 5, seg = sid & 31;
+      const __half2 sc2 = __float2half2_rn(ldexpf(S.rscale[kb][row], -ec));
       const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
       uint32_t o[8];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const float2 a = e4m3x2_to_float2(static_cast<uint16_t>(w[u] & 0xFFFF));
-        const float2 c = e4m3x2_to_float2(static_cast<uint16_t>(w[u] >> 16));
-        o[2 * u] = pack_bf16x2(a.x, a.y);
-        o[2 * u + 1] = pack_bf16x2(c.x, c.y);
+        __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[u] & 0xFFFF), __NV_E4M3);
+        __half2_raw c = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[u] >> 16), __NV_E4M3);
+        __half2 ha = __hmul2(*reinterpret_cast<__half2 *>(&a), sc2);
+        __half2 hc = __hmul2(*reinterpret_cast<__half2 *>(&c), sc2);
+        o[2 * u] = *reinterpret_cast<uint32_t *>(&ha);
+        o[2 * u + 1] = *reinterpret_cast<uint32_t *>(&hc);
       }
       const int atom = seg >> 2, c0 = (seg & 3) * 2;
       uint8_t *base = kt + atom * kAtom;
@@ -162,6 +263,7 @@ __device__ void gather_chunk(const MqaTcParams &P, MqaSmem &S, int b, const KeyL
       *reinterpret_cast<uint4 *>(base + sw128_offset(row, c0 + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
     }
   } else {  // bf16 rows: straight 16-byte copies into the swizzled tile
+    if (tid == 0) S.ec[kb] = 0;
     uint4 v[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
@@ -177,34 +279,82 @@ __device__ void gather_chunk(const MqaTcParams &P, MqaSmem &S, int b, const KeyL
   }
 }
 
-// rotated query of sequence b -> bf16, K-major swizzled
+// rotated query of sequence b, K-major swizzled: bf16, or fp16 scaled per head by a power
+// of two (qinv[h] undoes it in the logits) so that |q| < 2^14 whatever the input range.
+// A bf16 query is loaded once, all 16 segments of a thread up front.
 __device__ void load_query(const MqaTcParams &P, MqaSmem &S, int b, int64_t pos) {
   const MqaLaunch &p = P.a;
   const int tid = threadIdx.x;
   const int half = p.rope_dims / 2;
+  const bool f16 = fp16_operands(p);
+  const bool raw_bf16 = p.q_dt == DSV4_BF16;
+  uint4 raw[16];
+  if (raw_bf16) {
+    const uint16_t *q = static_cast<const uint16_t *>(p.q) + static_cast<size_t>(b) * kH * kD;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) raw[i] = __ldg(reinterpret_cast<const uint4 *>(q) + i * kThreads + tid);
+  }
   for (int i = tid; i < half; i += kThreads) rope_cos_sin(pos, i, p.rope_dims, p.rope_base, &S.cs[i], &S.sn[i]);
+  if (tid < kH) S.qmax[tid] = 0u;
   __syncthreads();
   const int rope0 = kD - p.rope_dims;
-#pragma unroll 4
-  for (int i = 0; i < 16; ++i) {
-    const int sid = i * kThreads + tid, h = sid >> 6, seg = sid & 63;
-    float x[8];
-    load_row_f<8>(p.q, p.q_dt, (static_cast<size_t>(b) * kH + h) * kD + seg * 8, x);
-    const int d0 = seg * 8;
-    if (d0 >= rope0) {
+  for (int pass = f16 ? 0 : 1; pass < 2; ++pass) {
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int pi = (d0 + 2 * u - rope0) >> 1;
-        const float c = S.cs[pi], s = S.sn[pi];
-        const float x0 = x[2 * u], x1 = x[2 * u + 1];
-        x[2 * u] = x0 * c - x1 * s;
-        x[2 * u + 1] = x0 * s + x1 * c;
+    for (int i = 0; i < 16; ++i) {
+      const int sid = i * kThreads + tid, h = sid >> 6, seg = sid & 63;
+      float x[8];
+      if (raw_bf16) {
+        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          x[2 * k] = __uint_as_float(w[k] << 16);
+          x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+        }
+      } else {
+        load_row_f<8>(p.q, p.q_dt, (static_cast<size_t>(b) * kH + h) * kD + seg * 8, x);
       }
+      const int d0 = seg * 8;
+      if (d0 >= rope0) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int pi = (d0 + 2 * u - rope0) >> 1;
+          const float c = S.cs[pi], s = S.sn[pi];
+          const float x0 = x[2 * u], x1 = x[2 * u + 1];
+          x[2 * u] = x0 * c - x1 * s;
+          x[2 * u + 1] = x0 * s + x1 * c;
+        }
+      }
+      if (pass == 0) {  // per-head max |q| (32 lanes of a warp cover half a head)
+        float am = 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) am = fmaxf(am, fabsf(x[u]));
+        am = warp_max(am);
+        if ((tid & 31) == 0) atomicMax(&S.qmax[h], __float_as_uint(am));
+        continue;
+      }
+      uint4 o;
+      if (f16) {
+        const float qs = 1.0f / S.qinv[h];
+        o = make_uint4(pack_f16x2(x[0] * qs, x[1] * qs), pack_f16x2(x[2] * qs, x[3] * qs),
+                       pack_f16x2(x[4] * qs, x[5] * qs), pack_f16x2(x[6] * qs, x[7] * qs));
+      } else {
+        o = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                       pack_bf16x2(x[6], x[7]));
+      }
+      *reinterpret_cast<uint4 *>(&S.q[seg >> 3][0] + sw128_offset(h, seg & 7)) = o;
     }
-    const uint4 o = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                               pack_bf16x2(x[6], x[7]));
-    *reinterpret_cast<uint4 *>(&S.q[seg >> 3][0] + sw128_offset(h, seg & 7)) = o;
+    if (pass == 0) {
+      __syncthreads();
+      if (tid < kH) {
+        int e = 0;
+        const float am = __uint_as_float(S.qmax[tid]);
+        if (am > 0.f) frexpf(am, &e);                         // am < 2^e
+        S.qinv[tid] = am > 0.f ? ldexpf(1.0f, e - 14) : 1.0f;  // scaled |q| < 2^14
+      }
+      __syncthreads();
+    }
   }
+  if (!f16 && tid < kH) S.qinv[tid] = 1.0f;
 }
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaTcParams P) {
@@ -224,15 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     tmem_alloc(&S.tmem_base, 512);
     tmem_relinquish();
   }
-  if (tid == 0) {
-    long long acc = 0;
-    for (int b = 0; b < p.B; ++b) {
-      prefix[b] = acc;
-      const KeyList L = key_list(p, b, blockIdx.x == 0);
-      acc += (L.nw + L.nsel + kCh - 1) / kCh;
-    }
-    prefix[p.B] = acc;
-  }
+  chunk_prefix(p, prefix, prefix + p.B + 1, blockIdx.x == 0);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -240,22 +382,28 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
   const long long T = prefix[p.B], G = gridDim.x;
   const long long c0 = (T * blockIdx.x) / G, c1 = (T * (blockIdx.x + 1)) / G;
 
+  const bool f16 = fp16_operands(p);
   const bool smax_thread = warp < 4 && lane >= 16;  // owns S/O row (head) 16*warp + lane - 16
   const int quad = warp & 3;
   const int head = quad * 16 + (lane & 15);
-  float m_ref = -INFINITY, l_run = 0.f;
+  // Online softmax in log2 units. With z_j = x_j + ec (x_j the logit of key j), the
+  // accumulators hold O = sum_j 2^(z_j - R) * Krow_j and l = sum_j 2^(z_j - R) * 2^-ec, both
+  // from the same rounded P, in units of 2^R; R is raised lazily (only when a chunk's max z
+  // exceeds it by more than 8), so P stays <= 2^8 and O is rescaled rarely.
+  float R = -INFINITY, l_run = 0.f;
   int cur_b = -1;
   bool first_in_seg = true;
   KeyList L{};
-  constexpr uint32_t idesc1 = idesc_bf16(kH, kCh, 0, 0);
-  constexpr uint32_t idesc2 = idesc_bf16(kH, 256, 0, 1);
+  const uint32_t idesc1 = f16 ? idesc_f16(kH, kCh, 0, 0) : idesc_bf16(kH, kCh, 0, 0);
+  const uint32_t idesc2 = f16 ? idesc_f16(kH, 256, 0, 1) : idesc_bf16(kH, 256, 0, 1);
   const uint32_t s_tmem = tmem + (16u << 16);  // S accumulator: lanes 16..31 of each quadrant
 
-  if (c0 < c1) {
-    const int b0 = find_seq(prefix, p.B, c0);
-    L = key_list(p, b0, false);
-    gather_chunk(P, S, b0, L, c0 - prefix[b0], 0);
+  if (tid == 0) {
+    S.meta_first = 0;
+    S.meta_n = 0;
   }
+  __syncthreads();
+  if (c0 < c1) gather_chunk(P, S, prefix, c0, c1, 0);
   for (long long g = c0; g < c1; ++g) {
     const long long it = g - c0;
     const int kb = static_cast<int>(it & 1);
@@ -263,13 +411,14 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     if (b != cur_b) {
       cur_b = b;
       first_in_seg = true;
-      m_ref = -INFINITY;
+      R = -INFINITY;
       l_run = 0.f;
       L = key_list(p, b, false);
       load_query(P, S, b, L.pos);
     }
     fence_proxy_async_smem();
     __syncthreads();
+    const int ec = S.ec[kb];
     if (tid == 0) {
       tc_fence_after();
       const uint32_t qa = smem_u32(&S.q[0][0]), ka = smem_u32(&S.k[kb][0][0]);
@@ -282,11 +431,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
       mma_commit(&S.bar_s);
     }
     // prefetch the next chunk while MMA1 runs (its buffer was released by MMA2 of it-1)
-    if (g + 1 < c1) {
-      const int bn = find_seq(prefix, p.B, g + 1);
-      const KeyList Ln = bn == b ? L : key_list(p, bn, false);
-      gather_chunk(P, S, bn, Ln, g + 1 - prefix[bn], kb ^ 1);
-    }
+    if (g + 1 < c1) gather_chunk(P, S, prefix, g + 1, c1, kb ^ 1);
     bool ok = mbar_wait(&S.bar_s, static_cast<uint32_t>(it & 1), &S.abort_flag);
     ok = __all_sync(0xFFFFFFFFu, ok);
     tc_fence_after();
@@ -299,34 +444,47 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
       tmem_ld_wait();
       if (smax_thread) {
         const float *rs = S.rscale[kb];
-        float x[kCh];
-        float mc = -INFINITY;
+        // logit in log2 units of key j: acc * tau*log2(e) * qinv[h] * (fp8: 2^ec; bf16: 1)
+        const float coef = P.scale_log2 * S.qinv[head] * ldexpf(1.0f, ec);
+        const float fec = static_cast<float>(ec);
+        float z[kCh];
+        float mz = -INFINITY;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
-          const float s0 = rs[j], s1 = rs[j + 32];
-          x[j] = s0 != 0.f ? __uint_as_float(r0[j]) * (P.scale_log2 * s0) : -INFINITY;
-          x[j + 32] = s1 != 0.f ? __uint_as_float(r1[j]) * (P.scale_log2 * s1) : -INFINITY;
-          mc = fmaxf(mc, fmaxf(x[j], x[j + 32]));
+          z[j] = rs[j] != 0.f ? fmaf(__uint_as_float(r0[j]), coef, fec) : -INFINITY;
+          z[j + 32] = rs[j + 32] != 0.f ? fmaf(__uint_as_float(r1[j]), coef, fec) : -INFINITY;
+          mz = fmaxf(mz, fmaxf(z[j], z[j + 32]));
         }
-        float ref = m_ref;
-        if (mc > m_ref + 8.f) ref = mc;
-        alpha = (ref == m_ref) ? 1.f : exp2f(m_ref - ref);  // m_ref = -inf -> 0
-        need_rescale = (ref != m_ref) && !first_in_seg;
+        float Rn = R;
+        if (mz > R + 8.f) Rn = mz;
+        alpha = (Rn == R) ? 1.f : exp2f(R - Rn);  // R = -inf -> 0
+        need_rescale = (Rn != R) && !first_in_seg;
+        const float lsc = ldexpf(1.0f, -ec);
         float lsum = 0.f;
         uint32_t pk[kCh / 2];
 #pragma unroll
         for (int j = 0; j < kCh; j += 2) {
-          const float e0 = x[j] == -INFINITY ? 0.f : exp2f(x[j] - ref);
-          const float e1 = x[j + 1] == -INFINITY ? 0.f : exp2f(x[j + 1] - ref);
-          lsum += e0 + e1;
-          pk[j / 2] = pack_bf16x2(e0 * rs[j], e1 * rs[j + 1]);
+          const float e0 = z[j] == -INFINITY ? 0.f : exp2f(z[j] - Rn);
+          const float e1 = z[j + 1] == -INFINITY ? 0.f : exp2f(z[j + 1] - Rn);
+          float r0f, r1f;
+          if (f16) {
+            __half2 h = __floats2half2_rn(e0, e1);
+            pk[j / 2] = *reinterpret_cast<uint32_t *>(&h);
+            const float2 back = __half22float2(h);
+            r0f = back.x;
+            r1f = back.y;
+          } else {
+            pk[j / 2] = pack_bf16x2(e0, e1);
+            r0f = __uint_as_float(pk[j / 2] << 16);
+            r1f = __uint_as_float(pk[j / 2] & 0xFFFF0000u);
+          }
+          lsum += r0f + r1f;  // the denominator uses the rounded P, like the numerator
         }
-        l_run = l_run * alpha + lsum;
-        m_ref = ref;
-        const int prow = head;
+        l_run = l_run * alpha + lsum * lsc;
+        R = Rn;
 #pragma unroll
         for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(S.p + sw128_offset(prow, c)) =
+          *reinterpret_cast<uint4 *>(S.p + sw128_offset(head, c)) =
               make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
       }
       // O rows (lanes 0..15) take their head's rescale factor from lane + 16
@@ -373,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
       const size_t slot = static_cast<size_t>(b) + blockIdx.x;
       if (smax_thread) {
         float *ml = P.part_ml + (slot * kH + head) * 2;
-        ml[0] = m_ref;
+        ml[0] = R;
         ml[1] = l_run;
       }
       // all 8 warps read O: warps 0-3 columns 0..255, warps 4-7 columns 256..511
@@ -409,48 +567,42 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
 // Merge the partials of every sequence, inverse RoPE, store. grid (B, H / 8), 256 threads.
 __global__ void __launch_bounds__(256) mqa_merge_kernel(const MqaTcParams P, int grid_ctas) {
   const MqaLaunch &p = P.a;
-  __shared__ long long prefix[2];
-  __shared__ int cfirst, clast;  // CTAs of the main kernel whose chunk range meets this sequence
+  __shared__ int np_s;  // partials of this sequence
   __shared__ float cs[kD / 2], sn[kD / 2];
-  extern __shared__ float wgt[];  // [grid_ctas][8]: weight of each partial, per head
+  extern __shared__ __align__(16) uint8_t dyn[];
+  float *wgt = reinterpret_cast<float *>(dyn);  // [grid_ctas][8]: weight of each partial, per head
+  int *cta = reinterpret_cast<int *>(wgt + static_cast<size_t>(grid_ctas) * 8);  // [grid_ctas]
+  long long *prefix = reinterpret_cast<long long *>(cta + ((grid_ctas + 1) & ~1));  // [B + 1]
+  long long *red = prefix + p.B + 1;                                             // [blockDim]
   __shared__ float inv_l[8], lse_s[8];
   const int b = blockIdx.x, h0 = blockIdx.y * 8, tid = threadIdx.x;
+  chunk_prefix(p, prefix, red, false);
   if (tid == 0) {
-    long long acc = 0, mine = 0, cnt = 0;
-    for (int bb = 0; bb < p.B; ++bb) {
-      const KeyList L = key_list(p, bb, false);
-      const long long c = (L.nw + L.nsel + kCh - 1) / kCh;
-      if (bb == b) { mine = acc; cnt = c; }
-      acc += c;
-    }
-    prefix[0] = mine;
-    prefix[1] = cnt;
-    int f = -1, l = -2;
+    // the CTAs of the main kernel whose (non-empty) chunk range meets this sequence; with
+    // fewer chunks than CTAs some ranges are empty and those CTAs wrote no partial
+    const long long acc = prefix[p.B], mine = prefix[b], cnt = prefix[b + 1] - prefix[b];
+    int n = 0;
     for (int c = 0; c < grid_ctas && cnt > 0; ++c) {
       const long long a0 = (acc * c) / grid_ctas, a1 = (acc * (c + 1)) / grid_ctas;
-      if (a0 < mine + cnt && a1 > mine && a1 > a0) {
-        if (f < 0) f = c;
-        l = c;
-      }
+      if (a0 < mine + cnt && a1 > mine && a1 > a0) cta[n++] = c;
     }
-    cfirst = f;
-    clast = l;
+    np_s = n;
   }
   const KeyList L = key_list(p, b, false);
   const int half = p.rope_dims / 2;
   for (int i = tid; i < half; i += 256) rope_cos_sin(L.pos, i, p.rope_dims, p.rope_base, &cs[i], &sn[i]);
   __syncthreads();
-  const int np = clast - cfirst + 1;  // partials of this sequence (<= grid_ctas)
+  const int np = np_s;
   if (tid < 8) {
     const int h = h0 + tid;
     float M = -INFINITY;
     for (int i = 0; i < np; ++i) {
-      const size_t slot = static_cast<size_t>(b) + cfirst + i;
+      const size_t slot = static_cast<size_t>(b) + cta[i];
       M = fmaxf(M, P.part_ml[(slot * kH + h) * 2]);
     }
     float Ls = 0.f;
     for (int i = 0; i < np; ++i) {
-      const size_t slot = static_cast<size_t>(b) + cfirst + i;
+      const size_t slot = static_cast<size_t>(b) + cta[i];
       const float mi = P.part_ml[(slot * kH + h) * 2], li = P.part_ml[(slot * kH + h) * 2 + 1];
       const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
       wgt[i * 8 + tid] = w;
@@ -465,7 +617,7 @@ __global__ void __launch_bounds__(256) mqa_merge_kernel(const MqaTcParams P, int
     const int hh = t / (kD / 2), pr = t % (kD / 2), h = h0 + hh;
     float o0 = 0.f, o1 = 0.f;
     for (int i = 0; i < np; ++i) {
-      const size_t slot = static_cast<size_t>(b) + cfirst + i;
+      const size_t slot = static_cast<size_t>(b) + cta[i];
       const float2 v = *reinterpret_cast<const float2 *>(P.part_o + (slot * kH + h) * kD + 2 * pr);
       o0 = fmaf(wgt[i * 8 + hh], v.x, o0);
       o1 = fmaf(wgt[i * 8 + hh], v.y, o1);
@@ -605,7 +757,7 @@ float softmax_scale_log2(const MqaLaunch &p) {
 
 bool mqa_uses_tensor_cores(const MqaLaunch &p) {
   return (p.kv_dt == DSV4_BF16 || p.kv_dt == DSV4_FP8E4M3) && p.D == kD && p.H == kH &&
-         (p.q_dt == DSV4_BF16 || p.q_dt == DSV4_F32) && p.rope_dims % 8 == 0 && p.B <= 8192;
+         (p.q_dt == DSV4_BF16 || p.q_dt == DSV4_F32) && p.rope_dims % 8 == 0 && p.B <= 1024;
 }
 
 size_t mqa_workspace_bytes(const MqaLaunch &p) {
@@ -622,13 +774,18 @@ cudaError_t launch_mqa(const MqaLaunch &p, void *ws, cudaStream_t st) {
     const size_t slots = static_cast<size_t>(p.B) + tc_grid();
     P.part_o = static_cast<float *>(ws);
     P.part_ml = reinterpret_cast<float *>(static_cast<char *>(ws) + align_up(slots * kH * kD * sizeof(float), 256));
-    const size_t smem = sizeof(MqaSmem) + 1024 + (static_cast<size_t>(p.B) + 1) * sizeof(long long);
+    const size_t smem = sizeof(MqaSmem) + 1024 + (static_cast<size_t>(p.B) + 1 + kThreads) * sizeof(long long);
     cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     mqa_tc_kernel<<<tc_grid(), kThreads, smem, st>>>(P);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    mqa_merge_kernel<<<dim3(p.B, kH / 8), 256, static_cast<size_t>(tc_grid()) * 8 * sizeof(float), st>>>(P, tc_grid());
+    const size_t msmem = static_cast<size_t>(tc_grid()) * 8 * sizeof(float) +
+                         static_cast<size_t>((tc_grid() + 1) & ~1) * sizeof(int) +
+                         (static_cast<size_t>(p.B) + 1 + 256) * sizeof(long long);
+    e = cudaFuncSetAttribute(mqa_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    if (e != cudaSuccess) return e;
+    mqa_merge_kernel<<<dim3(p.B, kH / 8), 256, msmem, st>>>(P, tc_grid());
     return cudaGetLastError();
   }
   const size_t smem = (2 * static_cast<size_t>(p.D) + 2 * kSimtChunk + 32) * sizeof(float) +

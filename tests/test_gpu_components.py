@@ -13,7 +13,7 @@ import compressed_sparse_kv_dsv4_b200 as dsv4
 import oracle.dsv4_oracle as O
 import synthetic as W
 from oracle import adapters as OA
-from tests.parity import check_output, check_topk, decode_out, require_gpu
+from tests.parity import check_output, check_topk, decode_out, input_class, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -213,17 +213,24 @@ def test_indexer_cuda_core_path_fp32_with_query_rope():
 
 
 # ---------------------------------------------------------------------------- attention
-def _mqa_case(spec, B, pos, n_entries, idx=None, seed=41, value_std=1.0):
+def _mqa_case(spec, B, pos, n_entries, idx=None, seed=41, value_std=1.0, out_dtype=None, garbage_ws=True):
     la = W.make_layer(spec, B, max(n_entries) + 1, seed, value_std=value_std, outlier_frac=0.05)
     st = W.make_step(spec, B, pos, seed + 1, q_std=value_std)
     dl = dsv4.DeviceLayer.from_arrays(la)
     q = dsv4.to_device_codes(st.q, spec.q_dtype, "cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
     idx_t = None if idx is None else torch.from_numpy(idx.astype(np.int32)).cuda()
-    out, lse = dsv4.sparse_mqa_decode(q, torch.from_numpy(st.pos).cuda(), dl.cache, dl.ring, q_dtype=spec.q_dtype,
-                                      out_dtype=spec.out_dtype, idx=idx_t,
-                                      n_entries=torch.tensor(n_entries, dtype=torch.int32, device="cuda"),
-                                      rope_dims=spec.rope_dims, with_lse=True, d_status=status)
+    args = dict(q_dtype=spec.q_dtype, out_dtype=out_dtype or spec.out_dtype, idx=idx_t,
+                n_entries=torch.tensor(n_entries, dtype=torch.int32, device="cuda"), rope_dims=spec.rope_dims)
+    ws = None
+    if garbage_ws:
+        # the workspace holds no state between calls: whatever it contains (NaN bytes here)
+        # must not reach the output
+        need = dsv4.mqa_workspace_size(dsv4.mqa_args(q, torch.from_numpy(st.pos).cuda(), dl.cache, dl.ring,
+                                                             out=torch.empty(1, device="cuda"), **args))
+        ws = torch.full((max(need, 256),), 0xFF, dtype=torch.uint8, device="cuda")
+    out, lse = dsv4.sparse_mqa_decode(q, torch.from_numpy(st.pos).cuda(), dl.cache, dl.ring, with_lse=True,
+                                      d_status=status, workspace=ws, **args)
     torch.cuda.synchronize()
     ol = OA.layer_state(la)
     qd = OA.decode_input(st.q, spec.q_dtype)
@@ -251,7 +258,7 @@ def test_mqa_tensor_core_dense_bf16():
     assert status == 0
     for s in range(3):
         o, l = _ref_attention(ol, qd, st, s, np.arange(n_entries[s]), spec)
-        check_output(out[s], o, "bf16", f"seq {s}")
+        check_output(out[s], o, "lowp", f"seq {s}", stored_bf16=True)
         assert np.max(np.abs(lse[s] - l)) < 2e-2
 
 
@@ -262,12 +269,14 @@ def test_mqa_tensor_core_sparse_fp8_with_padding_and_bad_index():
     idx = np.stack([rng.permutation(n_c)[:512] for _ in range(B)]).astype(np.int64)
     idx[0, 500:] = -1             # padding
     idx[1, 7] = n_c + 3           # out of range: skipped and reported
-    out, lse, status, ol, qd, st = _mqa_case(spec, B, [20000, 131072], [n_c, n_c], idx=idx)
-    assert status == dsv4._abi.DEV_BAD_INDEX
-    for s in range(B):
-        sel = [j for j in idx[s] if 0 <= j < n_c]
-        o, l = _ref_attention(ol, qd, st, s, sel, spec)
-        check_output(out[s], o, "bf16", f"seq {s}")
+    for out_dtype in ("f32", "bf16"):
+        out, lse, status, ol, qd, st = _mqa_case(spec, B, [20000, 131072], [n_c, n_c], idx=idx, out_dtype=out_dtype)
+        assert status == dsv4._abi.DEV_BAD_INDEX
+        for s in range(B):
+            sel = [j for j in idx[s] if 0 <= j < n_c]
+            o, l = _ref_attention(ol, qd, st, s, sel, spec)
+            check_output(out[s], o, "lowp", f"seq {s} out {out_dtype}", stored_bf16=out_dtype == "bf16")
+            assert np.max(np.abs(lse[s] - l)) < 2e-2
 
 
 def test_mqa_cuda_core_fp32():

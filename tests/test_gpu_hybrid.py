@@ -17,7 +17,7 @@ import compressed_sparse_kv_dsv4_b200 as dsv4
 import oracle.dsv4_oracle as O
 import synthetic as W
 from oracle import adapters as OA
-from tests.parity import check_output, check_topk, decode_out, require_gpu
+from tests.parity import check_output, check_topk, decode_out, input_class, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -50,7 +50,7 @@ def _step_and_check(dl, ol, spec, st, seqs=None, attend=True, extra_entries=None
         if spec.kind == "c4":
             n_c = O.visible_entries(int(st.pos[s]), spec.m)
             swaps += check_topk(idx[s], scores, spec.k, n_c, f"seq {s}", allow_extra=extra_entries)
-        check_output(out[s], o, spec.out_dtype, f"seq {s}")
+        check_output(out[s], o, input_class(spec), f"seq {s}", stored_bf16=spec.out_dtype == "bf16")
     return swaps
 
 
