@@ -192,8 +192,9 @@ dsv4_status dsv4_swa_insert(const dsv4_swa_insert_args *args, dsv4_stream stream
  *   keys: paged cache with keys.dim == dim, dtype F32 or FP8E4M3;
  *   n_entries [batch] device int32 (<= keys.max_blocks * 256/keys.m);
  *   pos [batch] device int32 (used only when q_rope_dims > 0).
- * fp8 keys with dim 128, heads in {16,32,64,128}, m <= 8 and k <= 1024 run on the tensor
- * cores (tcgen05, fed by TMA); other shapes run on a CUDA-core kernel.
+ * fp8 queries and keys with dim 128, heads 32 or 64, m == 4, k <= 512, no query RoPE and
+ * batch <= 512 run on the tensor cores (tcgen05, fed by TMA); other shapes run on a
+ * CUDA-core kernel. Both give the same entries.
  */
 typedef struct {
   int32_t batch;
