@@ -64,14 +64,16 @@ def input_class(spec) -> str:
 
 def check_output(got, want, inputs: str, ctx: str = "", stored_bf16: bool = False):
     """inputs: "f32" or "lowp" (bf16 / fp8 inputs). stored_bf16: the output was stored as
-    bf16, whose rounding alone moves a value by up to half an ulp (2^-9 relative); that
-    allowance is added to the max-abs bound, nothing else."""
+    bf16 (8 significant bits), whose round-to-nearest moves a value x by up to half an ulp,
+    2^(floor(log2|x|) - 8) <= 2^-8 |x|; that allowance, taken at |want| + the max-abs bound
+    (x is the unrounded result, within that bound of want), is added, nothing else."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     assert got.shape == want.shape, f"{ctx}: shape {got.shape} vs {want.shape}"
     assert np.all(np.isfinite(got)), f"{ctx}: non-finite output"
     err = np.abs(got - want)
-    store = 2.0 ** -9 * np.abs(want) if stored_bf16 else 0.0
+    bound = F32_MAX_ABS if inputs == "f32" else LOWP_MAX_ABS
+    store = 2.0 ** -8 * (np.abs(want) + bound) if stored_bf16 else 0.0
     if inputs == "f32":
         assert np.all(err <= F32_MAX_ABS + store), f"{ctx}: max-abs {err.max():.3e} > {F32_MAX_ABS}"
         return err.max(), None
