@@ -39,17 +39,18 @@ UNIT = "tokens/s"
 SPEC_ROWS = dict(D=512, H=64, k=512, W=128, H_I=64, d_I=128)
 
 
-def algorithmic_bytes_per_seq(n_c: int) -> dict:
+def algorithmic_bytes_per_seq(n_c: int, out_bytes: int = 2) -> dict:
     """Bytes one sequence's decode step must move (fp8 caches with a 4-byte row scale).
 
     indexer: every visible indexer key row (128 B + scale); attention: the k selected
-    rows and the W window rows (512 B + scale), the bf16 query and the f32 output; updates:
+    rows and the W window rows (512 B + scale), the bf16 query and the output (out_bytes
+    per value); updates:
     the new token's kv/gate and indexer kv/gate (bf16) read, the two compressor ring
     slots (float32) and the window row written; the indexer query, its scales and weights.
     """
     D, H, k, W, H_I, d_I = (SPEC_ROWS[x] for x in ("D", "H", "k", "W", "H_I", "d_I"))
     idx = n_c * (d_I + 4)
-    attn = (k + W) * (D + 4) + H * D * 2 + H * D * 4
+    attn = (k + W) * (D + 4) + H * D * 2 + H * D * out_bytes
     upd = 2 * D * 2 + 2 * d_I * 2 + 2 * D * 4 + 2 * d_I * 4 + (D + 4)
     qidx = H_I * d_I + H_I * 4 + H_I * 2
     return dict(indexer=idx + qidx, attention=attn, updates=upd, total=idx + qidx + attn + upd)
@@ -104,7 +105,9 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- distributed
-def dist_setup(n_gpus: int):
+def dist_setup(n_gpus: int, backend: str | None = None):
+    """Rank, world size and local rank from the torchrun environment; joins the process
+    group when world > 1 (nccl on GPUs; gloo where there is no GPU, as in the CPU tests)."""
     import torch
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -115,9 +118,13 @@ def dist_setup(n_gpus: int):
 
         import torch.distributed as dist
 
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
-                                device_id=torch.device("cuda", local))
+        backend = backend or ("nccl" if torch.cuda.is_available() else "gloo")
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=60))
     elif torch.cuda.is_available():
         torch.cuda.set_device(0)
     return rank, world, local
@@ -131,14 +138,26 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest x over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def shard_seed(rank: int) -> int:
+    """Seed of a rank's own sequences: ranks decode disjoint, independent batches."""
+    return 2 + 1000 * rank
+
+
+def job_tokens_per_s(world: int, ms_max: float) -> float:
+    """Whole-job decode tokens/s: every rank's sequences over the slowest rank's step."""
+    return world * B_PER_GPU / (ms_max * 1e-3)
 
 
 # ----------------------------------------------------------------------------- CPU oracle
@@ -171,6 +190,29 @@ def blas_threads() -> int:
         return 1
 
 
+def kernel_sources_sha256() -> str:
+    """Hash of the sources the indexer kernel is compiled from."""
+    import hashlib
+
+    h = hashlib.sha256()
+    for f in ("indexer.cu", "common.cuh", "internal.h"):
+        with open(os.path.join(ROOT, "compressed_sparse_kv_dsv4_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
+def indexer_traffic():
+    """DRAM bytes (read + write) per indexer launch at this workload, from the committed ncu
+    summary; None when there is none or the kernel's sources changed since it was taken."""
+    try:
+        rec = json.load(open(os.path.join(ROOT, "profiles", "indexer_traffic.json")))
+    except (OSError, ValueError):
+        return None
+    if rec.get("sources_sha256") != kernel_sources_sha256():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_ours(args):
     import torch
@@ -182,7 +224,7 @@ def run_ours(args):
     rank, world, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     lib = dsv4.load()
-    la, sets = W.c4_sparse(seed=2 + 1000 * rank, B=B_PER_GPU, context=CONTEXT, steps=N_INPUT_SETS)
+    la, sets = W.c4_sparse(seed=shard_seed(rank), B=B_PER_GPU, context=CONTEXT, steps=N_INPUT_SETS)
     spec = la.spec
     dl = dsv4.DeviceLayer.from_arrays(la, dev)
     dsteps = [dsv4.DeviceStep.from_arrays(spec, st, dev) for st in sets]
@@ -288,7 +330,7 @@ def run_ours(args):
             dist.destroy_process_group()
         return
 
-    byts = algorithmic_bytes_per_seq(n_c)
+    byts = algorithmic_bytes_per_seq(n_c, out_bytes=4 if spec.out_dtype == "f32" else 2)
     step_bytes = byts["total"] * B_PER_GPU
     ix_bytes = byts["indexer"] * B_PER_GPU
     peaks = {}
@@ -299,23 +341,17 @@ def run_ours(args):
         hbm_peak, peak_src = 6650.0, "fallback"
     ix_gbs = ix_bytes / (ix_ms * 1e-3) / 1e9
     step_gbs = step_bytes / (ms * 1e-3) / 1e9
-    traffic = None
-    tfile = os.path.join(ROOT, "profiles", "indexer_traffic.json")
-    if os.path.exists(tfile):
-        try:
-            traffic = json.load(open(tfile)).get("dram_bytes_per_launch")
-        except Exception:  # noqa: BLE001
-            traffic = None
-    value = world * B_PER_GPU / (ms * 1e-3)
+    traffic = indexer_traffic()
+    value = job_tokens_per_s(world, ms)
     line = {
         "metric": METRIC, "value": round(value, 1), "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8 indexer; fp16-operand attention over fp8 rows (fp32 accumulate)",
-        "data": "synthetic",
+        "vs_baseline": None, "dtype": "fp8", "data": "synthetic",
         "config": {"workload": "c4_sparse_131k", "batch_per_gpu": B_PER_GPU, "global_batch": world * B_PER_GPU,
                    "context": CONTEXT, "c4_entries": n_c, "topk": spec.k, "window": spec.W, "heads": spec.H,
                    "kv_dim": spec.D, "indexer": f"{spec.H_I} heads x {spec.d_I} fp8", "cache": "fp8 e4m3 + fp32 row scale",
                    "query": "bf16", "output": spec.out_dtype,
+                   "arithmetic": "e4m3 x e4m3 indexer MMA, fp16-operand attention MMAs over e4m3 rows, f32 accumulate",
                    "parallelism": f"dp{world} (independent sequences)", "l2": "flushed between steps (256 MiB write)",
                    "positions": f"advance by one per step, cycling over {CONTEXT}..{CONTEXT + POS_CYCLE - 1}"},
         "hbm": {"step_algorithmic_bytes": step_bytes, "achieved_gbs": round(step_gbs, 1),
@@ -324,7 +360,7 @@ def run_ours(args):
         "roofline": {"kernel": "indexer_tc_kernel (+ top-k select)", "bound": "hbm", "achieved": round(ix_gbs, 1),
                      "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s", "frac": round(ix_gbs / hbm_peak, 4),
                      "traffic": traffic, "algorithmic_bytes_per_launch": ix_bytes, "launch_ms": round(ix_ms, 5)},
-        "e2e": {"value": round(world * B_PER_GPU / (e2e_ms * 1e-3), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
+        "e2e": {"value": round(job_tokens_per_s(world, e2e_ms), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
         "gpu_launches": 5 * args.steps,
         "clocks": clk.summary(t_a, t_b),

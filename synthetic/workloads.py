@@ -301,7 +301,7 @@ C128_SPEC = LayerSpec(kind="c128", m=128, H=64, D=512, W=128, k=0, cache_dtype="
 C4_SPEC = LayerSpec(kind="c4", m=4, H=64, D=512, W=128, k=512, H_I=64, d_I=128,
                     idx_rope_dims=64, cache_dtype="fp8", swa_dtype="fp8", idx_dtype="fp8",
                     kv_dtype="bf16", q_dtype="bf16", q_idx_dtype="fp8", w_dtype="bf16",
-                    out_dtype="f32")
+                    out_dtype="bf16")
 
 
 def c128_dense_bf16(seed: int = 1, B: int = 8, context: int = 65536, steps: int = 1):
