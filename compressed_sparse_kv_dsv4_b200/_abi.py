@@ -9,7 +9,8 @@ from .build import LIB
 
 F32, BF16, FP8 = 0, 1, 2
 LAYER_C4, LAYER_C128 = 0, 1
-OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA = 0, 1, 2, 3
+OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SCRATCH_LIMIT = 0, 1, 2, 3, 4
+NOALLOC_SCRATCH_BYTES = 16 << 20
 DEV_BAD_INDEX, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
 PAGE_POSITIONS = 256
 
@@ -82,6 +83,7 @@ EXPORTS = {
     "dsv4_swa_insert": (C.c_int, [C.POINTER(SwaInsertArgs), p]),
     "dsv4_indexer_workspace_size": (C.c_size_t, [C.POINTER(IndexerArgs)]),
     "dsv4_indexer_topk": (C.c_int, [C.POINTER(IndexerArgs), p, C.c_size_t, p]),
+    "dsv4_indexer_topk_noalloc": (C.c_int, [C.POINTER(IndexerArgs), p]),
     "dsv4_mqa_workspace_size": (C.c_size_t, [C.POINTER(MqaArgs)]),
     "dsv4_sparse_mqa_decode": (C.c_int, [C.POINTER(MqaArgs), p, C.c_size_t, p]),
     "dsv4_hybrid_decode_workspace_size": (C.c_size_t, [C.POINTER(Layer), i32]),

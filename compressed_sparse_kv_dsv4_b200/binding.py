@@ -274,6 +274,17 @@ def indexer_topk(q_idx, w, keys: DeviceCache, n_entries, k: int, *, q_dtype: str
     return idx, scores
 
 
+def indexer_topk_noalloc(q_idx, w, keys: DeviceCache, n_entries, k: int, *, idx, q_dtype: str, w_dtype: str,
+                         scores=None, q_scale=None, pos=None, q_rope_dims: int = 0, rope_base: float = 10000.0,
+                         d_status=None, stream=None):
+    """indexer_topk on the library's static scratch: the caller passes the outputs (idx [B, k]
+    int32, optionally scores [B, k] float32) and nothing is allocated by this call."""
+    a = indexer_args(q_idx, w, keys, n_entries, k, q_dtype=q_dtype, w_dtype=w_dtype, q_scale=q_scale, pos=pos,
+                     q_rope_dims=q_rope_dims, rope_base=rope_base, idx=idx, scores=scores, d_status=d_status)
+    A.check("dsv4_indexer_topk_noalloc", A.load().dsv4_indexer_topk_noalloc(C.byref(a), _stream(stream)))
+    return idx, scores
+
+
 def mqa_args(q, pos, cache: DeviceCache, ring: DeviceRing, *, q_dtype: str, out, out_dtype: str, idx=None,
              n_entries=None, softmax_scale: float = 0.0, rope_dims: int = 64, rope_base: float = 10000.0, lse=None,
              d_status=None) -> A.MqaArgs:

@@ -80,6 +80,7 @@ const char *dsv4_status_string(dsv4_status s) {
     case DSV4_ERR_INVALID_ARG: return "invalid argument";
     case DSV4_ERR_UNSUPPORTED: return "unsupported combination";
     case DSV4_ERR_CUDA: return "CUDA launch error";
+    case DSV4_ERR_SCRATCH_LIMIT: return "request exceeds the library's static scratch";
   }
   return "unknown status";
 }
@@ -470,3 +471,50 @@ dsv4_status dsv4_hybrid_decode(const dsv4_layer *layer, const dsv4_step *step, v
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------
+// Indexer top-k on library-owned scratch. For callers that cannot allocate: a host
+// program without a device allocator of its own, or a decode loop that must not stall on
+// cudaMalloc/cudaFree. The scratch is a file-scope device array; its address is resolved
+// once per device and handed to the same launcher dsv4_indexer_topk uses.
+namespace {
+
+static __device__ __align__(256) unsigned char noalloc_scratch[DSV4_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+
+// Device address of noalloc_scratch on the current device. The first call on a device
+// resolves it (cudaGetSymbolAddress may load the module, which must not happen inside a
+// stream capture) and caches the SM count, so later calls do no set-up work at all.
+dsv4_status noalloc_scratch_address(void **out) {
+  static std::mutex mu;
+  static void *addr[kMaxDevices] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return to_status(cudaErrorInvalidDevice);
+  if (dev < 0 || dev >= kMaxDevices) return DSV4_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void *p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, noalloc_scratch);
+    if (e != cudaSuccess) return to_status(e);
+    if (!p || (reinterpret_cast<uintptr_t>(p) & 255u)) return DSV4_ERR_CUDA;
+    sm_count();
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return DSV4_OK;
+}
+
+}  // namespace
+
+extern "C" dsv4_status dsv4_indexer_topk_noalloc(const dsv4_indexer_args *a, dsv4_stream stream) {
+  IndexerLaunch p;
+  const dsv4_status s = indexer_launch_args(a, &p);
+  if (s != DSV4_OK) return s;
+  if (indexer_workspace_bytes(p) > DSV4_NOALLOC_SCRATCH_BYTES) return DSV4_ERR_SCRATCH_LIMIT;
+  void *ws = nullptr;
+  const dsv4_status r = noalloc_scratch_address(&ws);
+  if (r != DSV4_OK) return r;
+  // the launcher zeroes the candidate counts at the head of ws on `stream` itself
+  return to_status(launch_indexer_topk(p, ws, static_cast<cudaStream_t>(stream)));
+}

@@ -63,7 +63,8 @@ typedef enum {
   DSV4_OK = 0,
   DSV4_ERR_INVALID_ARG = 1,
   DSV4_ERR_UNSUPPORTED = 2,
-  DSV4_ERR_CUDA = 3
+  DSV4_ERR_CUDA = 3,
+  DSV4_ERR_SCRATCH_LIMIT = 4 /* the request needs more than the library's static scratch */
 } dsv4_status;
 
 typedef enum { DSV4_F32 = 0, DSV4_BF16 = 1, DSV4_FP8E4M3 = 2 } dsv4_dtype;
@@ -219,6 +220,34 @@ typedef struct {
 size_t dsv4_indexer_workspace_size(const dsv4_indexer_args *args);
 dsv4_status dsv4_indexer_topk(const dsv4_indexer_args *args, void *workspace,
                               size_t workspace_bytes, dsv4_stream stream);
+
+/* ------------------------------------------------------------------------------------
+ * dsv4_indexer_topk_noalloc: dsv4_indexer_topk on scratch the library owns. The pages have
+ * no counterpart to this call: it is a convenience of the library, not a step of the method.
+ * Same arguments, kernels and results as dsv4_indexer_topk; no workspace argument.
+ *
+ * Who it is for: a caller that has no device allocator of its own (a plain C host program
+ * driving the library) or that must not call cudaMalloc/cudaFree on its decode loop, where
+ * each such call stalls the device and the host. The call itself allocates and frees
+ * nothing, on the device or the host.
+ *
+ * Scratch: one file-scope device array of DSV4_NOALLOC_SCRATCH_BYTES (16 MiB) per device,
+ * created with the library's device code when the module loads.
+ * Set-up: the first call on a device (with that device current) resolves the array's
+ * address once (cudaGetSymbolAddress, which may load the module) and caches the SM count;
+ * make that first call before any stream capture begins.
+ * Limit: if dsv4_indexer_workspace_size(args) > DSV4_NOALLOC_SCRATCH_BYTES the call returns
+ * DSV4_ERR_SCRATCH_LIMIT and launches nothing (use dsv4_indexer_topk with a caller
+ * workspace instead). With fp8 keys of 128 dims, k = 512 and 32768 visible entries per
+ * sequence that admits about 13 sequences.
+ * Zero state: nothing has to start at zero; the per-sequence candidate counts at the head
+ * of the scratch are zeroed by the call itself, on `stream`, before its kernels run.
+ * Concurrency: the scratch is shared by every call on a device. Calls ordered on one
+ * stream are safe; calls that can overlap (different streams, or several host threads
+ * without ordering) race on the scratch and give wrong results: serialize them.
+ */
+#define DSV4_NOALLOC_SCRATCH_BYTES (16u << 20)
+dsv4_status dsv4_indexer_topk_noalloc(const dsv4_indexer_args *args, dsv4_stream stream);
 
 /* ------------------------------------------------------------------------------------
  * dsv4_sparse_mqa_decode: shared-K/V multi-query attention of one decode query per
