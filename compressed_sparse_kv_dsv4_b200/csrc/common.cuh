@@ -77,14 +77,23 @@ __device__ __forceinline__ uint32_t topk_key_index(unsigned long long key) {
 // The angle is formed and reduced in double precision, so positions up to 2^20 and
 // beyond keep ~1e-10 rad accuracy; the rotation itself is done in float.
 
-__device__ __forceinline__ void rope_cos_sin(int64_t pos, int pair, int rope_dims, float base,
-                                             float *c, float *s) {
-  double theta = pow(static_cast<double>(base), -2.0 * pair / static_cast<double>(rope_dims));
-  double a = static_cast<double>(pos) * theta;
-  double sd, cd;
-  sincos(a, &sd, &cd);
-  *c = static_cast<float>(cd);
-  *s = static_cast<float>(sd);
+// cos and sin of RoPE pair `pair` at position pos: angle = pos * theta1^pair with
+// theta1 = base^(-2/rope_dims). The angle is formed in float64 (theta1^pair by binary
+// powering, relative error ~1e-15) and reduced to [-pi, pi] by a two-constant Cody-Waite
+// step with fused multiply-adds; sin and cos of the reduced angle are taken in float32.
+__device__ __forceinline__ void rope_cos_sin(int64_t pos, int pair, double theta1, float *c, float *s) {
+  constexpr double kTwoPiHi = 6.283185307179586;       // 2*pi rounded to float64
+  constexpr double kTwoPiLo = 2.4492935982947064e-16;  // 2*pi - kTwoPiHi
+  constexpr double kInvTwoPi = 0.15915494309189535;
+  double th = 1.0, b = theta1;
+  for (int e = pair; e; e >>= 1) {
+    if (e & 1) th *= b;
+    b *= b;
+  }
+  const double a = static_cast<double>(pos) * th;
+  const double k = rint(a * kInvTwoPi);
+  const double r = fma(-k, kTwoPiLo, fma(-k, kTwoPiHi, a));
+  sincosf(static_cast<float>(r), s, c);
 }
 
 // --------------------------------------------------------------------------------------
@@ -235,6 +244,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 16-byte global -> shared copy (both addresses 16-byte aligned), L2 only
+__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+// one arrival on bar once every earlier cp.async of this thread has landed
+__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
 __device__ __forceinline__ void named_bar_sync(int id, int count) {

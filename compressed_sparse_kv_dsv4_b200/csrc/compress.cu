@@ -128,7 +128,7 @@ __device__ void pool_block(const TokenSource &src, int64_t b, float *e, float *s
 // RMSNorm(e) * gamma, RoPE at `rope_pos`, round into `dt`, store to `row` (+ *scale_out).
 // e: shared float[D]; red: shared float[32]. Every thread of the CTA calls this.
 __device__ void finish_and_store(float *e, int D, const float *gamma, float eps, int64_t rope_pos, int rope_dims,
-                                 float rope_base, dsv4_dtype dt, void *row, float *scale_out, float *red) {
+                                 double rope_theta1, dsv4_dtype dt, void *row, float *scale_out, float *red) {
   const int tid = threadIdx.x;
   float ss = 0.f;
   for (int c = tid; c < D; c += kThreads) ss += e[c] * e[c];
@@ -140,7 +140,7 @@ __device__ void finish_and_store(float *e, int D, const float *gamma, float eps,
   const int half = rope_dims / 2;
   for (int i = tid; i < half; i += kThreads) {
     float cs, sn;
-    rope_cos_sin(rope_pos, i, rope_dims, rope_base, &cs, &sn);
+    rope_cos_sin(rope_pos, i, rope_theta1, &cs, &sn);
     const int c0 = D - rope_dims + 2 * i;
     const float x0 = e[c0], x1 = e[c0 + 1];
     e[c0] = x0 * cs - x1 * sn;
@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressLaunch
       void *row = cache_row(p.pages, p.scales, p.block_table, p.num_pages, p.max_blocks, p.m, p.D, p.cache_dt, s, b,
                             &sp, p.d_status);
       if (row != nullptr)  // uniform over the CTA
-        finish_and_store(e, p.D, p.gamma, p.eps, b * p.m, p.rope_dims, p.rope_base, p.cache_dt, row, sp, red);
+        finish_and_store(e, p.D, p.gamma, p.eps, b * p.m, p.rope_dims, p.rope_theta1, p.cache_dt, row, sp, red);
     }
     if (i == 0) {
       // the state ring keeps the latest m tokens (slot t % m); written after the first
@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(kThreads) swa_insert_kernel(const SwaLaunch p)
   __syncthreads();
   const size_t slot = static_cast<size_t>(s) * p.W + static_cast<size_t>(t % p.W);
   void *row = static_cast<char *>(p.rows) + slot * p.D * dtype_size(p.ring_dt);
-  finish_and_store(e, p.D, p.gamma, p.eps, t, p.rope_dims, p.rope_base, p.ring_dt, row,
+  finish_and_store(e, p.D, p.gamma, p.eps, t, p.rope_dims, p.rope_theta1, p.ring_dt, row,
                    p.scales ? p.scales + slot : nullptr, red);
 }
 
@@ -288,7 +288,7 @@ __global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const Prologu
     __syncthreads();
     const size_t slot = static_cast<size_t>(s) * p.W + static_cast<size_t>(pos % p.W);
     void *row = static_cast<char *>(p.ring_rows) + slot * p.D * dtype_size(p.ring_dt);
-    finish_and_store(e, p.D, p.gamma, p.eps, pos, p.rope_dims, p.rope_base, p.ring_dt, row,
+    finish_and_store(e, p.D, p.gamma, p.eps, pos, p.rope_dims, p.rope_theta1, p.ring_dt, row,
                      p.ring_scales ? p.ring_scales + slot : nullptr, red);
     return;
   }
@@ -312,14 +312,16 @@ __global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const Prologu
                               p.d_status);
   if (row != nullptr)
     finish_and_store(e, D, idx ? p.gamma_idx : p.gamma, p.eps, b * m, idx ? p.idx_rope_dims : p.rope_dims,
-                     p.rope_base, idx ? p.idx_dt : p.cache_dt, row, sp, red);
+                     idx ? p.idx_rope_theta1 : p.rope_theta1, idx ? p.idx_dt : p.cache_dt, row, sp, red);
 }
 
 constexpr size_t kPoolSmem = (4 * kMaxD + 32) * sizeof(float);
 
 }  // namespace
 
-cudaError_t launch_compress(const CompressLaunch &p, cudaStream_t st) {
+cudaError_t launch_compress(const CompressLaunch &p0, cudaStream_t st) {
+  CompressLaunch p = p0;
+  p.rope_theta1 = rope_theta1(p.rope_base, p.rope_dims);
   const size_t smem = kPoolSmem + (p.B + 1) * sizeof(long long);
   cudaError_t e = cudaFuncSetAttribute(compress_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -330,13 +332,18 @@ cudaError_t launch_compress(const CompressLaunch &p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_swa_insert(const SwaLaunch &p, cudaStream_t st) {
+cudaError_t launch_swa_insert(const SwaLaunch &p0, cudaStream_t st) {
+  SwaLaunch p = p0;
+  p.rope_theta1 = rope_theta1(p.rope_base, p.rope_dims);
   dim3 grid(p.W, p.B);
   swa_insert_kernel<<<grid, kThreads, 0, st>>>(p);
   return cudaGetLastError();
 }
 
-cudaError_t launch_decode_prologue(const PrologueLaunch &p, cudaStream_t st) {
+cudaError_t launch_decode_prologue(const PrologueLaunch &p0, cudaStream_t st) {
+  PrologueLaunch p = p0;
+  p.rope_theta1 = rope_theta1(p.rope_base, p.rope_dims);
+  p.idx_rope_theta1 = rope_theta1(p.rope_base, p.idx_rope_dims);
   cudaError_t e =
       cudaFuncSetAttribute(decode_prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPoolSmem);
   if (e != cudaSuccess) return e;

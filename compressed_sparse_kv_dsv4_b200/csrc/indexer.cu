@@ -5,13 +5,15 @@
 //   keep the k largest s_j (ties to the lower j)
 //
 // Tensor-core path (fp8 keys, 128-dim, the C4 layers): a persistent kernel, one CTA per
-// SM, over the flattened (sequence, 128-entry tile) space. Warp 0 streams key tiles with
-// TMA (two 8 KB page boxes per tile, 128B swizzle) into an 8-stage ring; warp 1 issues
-// tcgen05.mma kind::f8f6f4 (M = 128 entries, N = H heads, K = 128) into a double-buffered
-// TMEM accumulator; warps 2-5 read the accumulator back (tcgen05.ld), apply ReLU, the
-// per-head weights w_h * scale_q[h] and the per-entry key scale, and keep a running
-// top-k in shared memory (threshold filter + radix-select compaction). Each CTA writes at
-// most k candidates per sequence segment; a small select kernel merges them.
+// SM, over the flattened (sequence, 128-entry tile) space, in stages of up to two tiles of
+// one sequence. Warp 0 streams key pages with TMA (8 KB boxes, 128B swizzle) into a
+// 5-stage ring, with the block-table entries fetched a batch of 8 stages ahead and the key
+// scales copied by cp.async; warp 1 issues tcgen05.mma kind::f8f6f4 (M = 128 entries,
+// N = H heads, K = 128) into two TMEM accumulator sets; two groups of four warps take
+// alternate stages, read their accumulators back (tcgen05.ld), apply ReLU, the per-head
+// weights w_h * scale_q[h] and the per-entry key scale, and store every score (4 bytes per
+// entry, coalesced). A second kernel selects the top k of each sequence from the scores
+// in shared memory (radix select), writing them in ascending entry order.
 //
 // The scale handling relies on ReLU(a * x) = a * ReLU(x) for a > 0:
 //   s_j = scale_k[j] * sum_h (w_h * scale_q[h]) * ReLU(q8_h . k8_j).
@@ -88,7 +90,7 @@ __global__ void __launch_bounds__(256) indexer_simt_kernel(const IndexerLaunch p
     for (int t = threadIdx.x; t < H * half; t += blockDim.x) {
       const int h = t / half, i = t % half;
       float c, s;
-      rope_cos_sin(p.pos[b], i, p.q_rope_dims, p.rope_base, &c, &s);
+      rope_cos_sin(p.pos[b], i, p.rope_theta1, &c, &s);
       float *x = sq + h * Dq + Dq - p.q_rope_dims + 2 * i;
       const float x0 = x[0], x1 = x[1];
       x[0] = x0 * c - x1 * s;
@@ -118,7 +120,7 @@ __global__ void __launch_bounds__(256) indexer_simt_kernel(const IndexerLaunch p
 }
 
 // ------------------------------------------------------------------------------------
-// Tensor-core scoring with a fused per-CTA top-k.
+// Tensor-core scoring: every visible entry's score streamed to a [B][ld] float buffer.
 
 struct TcParams {
   CUtensorMap tmap_k;  // keys as [num_pages * 64 rows][128 bytes], 128B swizzle
@@ -129,12 +131,11 @@ struct TcParams {
   const float *q_scale;
   const void *w;
   dsv4_dtype w_dt;
-  int B, k, m;
+  int B, m;
   const int32_t *n_entries;
   const int32_t *pos;
-  unsigned long long *cand;
-  int64_t stride;
-  int *cand_count;
+  float *scores;  // [B][ld]; -inf where the entry has no valid page
+  int64_t ld;
   uint32_t *d_status;
 };
 
@@ -142,31 +143,22 @@ struct TcParams {
 // a pipeline stage = up to 2 tiles of one sequence (32 KB of keys).
 constexpr int kPerPage = 64;
 constexpr int kStageTiles = 2;
+constexpr int kStagePages = kStageTiles * kTile / kPerPage;  // 4
 constexpr int kStages = 5;       // key stages in flight (160 KB)
 constexpr int kSlots = 8;        // key-scale ring, one slot per stage
+constexpr int kBatchStages = 32 / kStagePages;  // stages whose page ids one warp load covers (8)
 constexpr int kGroups = 2;       // epilogue warp groups, alternating stages
-constexpr int kCapG = 1024;      // candidate buffer of a group
-constexpr int kMaxKTc = 512;     // largest k of the tensor-core path
 constexpr int kGroupThreads = 128;
 constexpr int kIxThreads = 64 + kGroups * kGroupThreads;
-
-struct GroupState {
-  unsigned long long thr, sel_prefix, sel_mask;
-  int cnt, cnt2, out_base, sel_digit, sel_above, sel_count, stop;
-};
 
 template <int H>  // H in {32, 64}
 struct alignas(1024) TcSmem {
   uint8_t stage[kStages][kStageTiles][kTile * kRowBytes];  // key tiles (rows = entries)
   uint8_t q[2][H * kRowBytes];
-  float sig[kSlots][kStageTiles * kTile];                   // key scales of each stage (0: no key)
-  unsigned long long cand[kGroups][kCapG];
-  unsigned long long cand2[kGroups][kMaxKTc];
-  float coef[kGroups][H];
-  int hist[kGroups][256];
+  float sig[kSlots][kStageTiles * kTile];  // key scales of each stage (0: no key)
+  float coef[kGroups * 4][H];              // per epilogue warp: w_h * scale_q[h] of its sequence
   uint64_t full[kStages], empty[kStages], sfull[kSlots], sempty[kSlots];
   uint64_t tfull[kGroups], tempty[kGroups], qfull[2], qempty[2];
-  GroupState gs[kGroups];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -209,106 +201,30 @@ struct StageIter {
   }
 };
 
-__device__ __forceinline__ void cp_async16(void *smem_dst, const void *gsrc) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem_dst)), "l"(gsrc) : "memory");
-}
-// one arrival on bar once every earlier cp.async of this thread has landed
-__device__ __forceinline__ void cp_async_arrive(uint64_t *bar) {
-  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// Top-k of one epilogue group: MSB-first radix select over the bytes of the (distinct)
-// 64-bit keys of cand[gi][0..cnt). Leaves (prefix, mask) such that
-// {key : (key & mask) >= prefix} has exactly k elements. 128 threads of the group.
-template <int H>
-__device__ void group_select(TcSmem<H> &S, int gi, int cnt, int k, int gt) {
-  GroupState &G = S.gs[gi];
-  int *hist = S.hist[gi];
-  const int bar = 1 + gi;
-  unsigned long long prefix = 0, mask = 0;
-  int need = k;
-  for (int shift = 56; shift >= 0; shift -= 8) {
-    for (int i = gt; i < 256; i += kGroupThreads) hist[i] = 0;
-    named_bar_sync(bar, kGroupThreads);
-    hist_add_warp(hist, S.cand[gi], cnt, gt >> 5, kGroupThreads >> 5, prefix, mask, shift);
-    named_bar_sync(bar, kGroupThreads);
-    if (gt < 32) {
-      int c[8], tot = 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) { c[u] = hist[255 - gt * 8 - u]; tot += c[u]; }
-      int incl = tot;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (gt >= o) incl += v;
-      }
-      int run = incl - tot;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (run < need && run + c[u] >= need) {
-          G.sel_digit = 255 - gt * 8 - u;
-          G.sel_above = run;
-          G.sel_count = c[u];
-        }
-        run += c[u];
-      }
-    }
-    named_bar_sync(bar, kGroupThreads);
-    const int digit = G.sel_digit, above = G.sel_above, cntd = G.sel_count;
-    prefix |= static_cast<unsigned long long>(digit) << shift;
-    mask |= 0xFFull << shift;
-    need -= above;
-    named_bar_sync(bar, kGroupThreads);
-    if (cntd == need) break;
-  }
-  if (gt == 0) { G.sel_prefix = prefix; G.sel_mask = mask; }
-  named_bar_sync(bar, kGroupThreads);
-}
-
-// keep exactly the k best candidates of group gi and raise its insertion threshold
-template <int H>
-__device__ void group_compact(TcSmem<H> &S, int gi, int k, int gt) {
-  GroupState &G = S.gs[gi];
-  const int bar = 1 + gi;
-  const int cnt = G.cnt;
-  group_select(S, gi, cnt, k, gt);
-  const unsigned long long prefix = G.sel_prefix, mask = G.sel_mask;
-  if (gt == 0) G.cnt2 = 0;
-  named_bar_sync(bar, kGroupThreads);
-  for (int i = gt; i < cnt; i += kGroupThreads) {
-    const unsigned long long key = S.cand[gi][i];
-    if ((key & mask) >= prefix) {
-      const int at = atomicAdd(&G.cnt2, 1);
-      if (at < kMaxKTc) S.cand2[gi][at] = key;
+// Page ids of the next kBatchStages stages, one per lane (lane = 4 * stage + page): the
+// block-table loads of a whole batch are in flight together, a batch ahead of their use.
+__device__ __forceinline__ int load_page_batch(const TcParams &p, const long long *prefix, const int64_t *nvis,
+                                               StageIter &ahead, int lane) {
+  int sb_l = -1;
+  int64_t first_l = 0;
+#pragma unroll 1
+  for (int i = 0; i < kBatchStages; ++i) {
+    int sb, nt;
+    long long lt0;
+    bool ns, se;
+    if (!ahead.next(prefix, sb, lt0, nt, ns, se)) break;
+    if ((lane >> 2) == i && (lane & 3) < nt * 2) {
+      sb_l = sb;
+      first_l = lt0 * kTile + static_cast<int64_t>(lane & 3) * kPerPage;
     }
   }
-  named_bar_sync(bar, kGroupThreads);
-  const int kept = G.cnt2 < k ? G.cnt2 : k;
-  for (int i = gt; i < kept; i += kGroupThreads) S.cand[gi][i] = S.cand2[gi][i];
-  named_bar_sync(bar, kGroupThreads);
-  if (gt == 0) {
-    G.cnt = kept;
-    if (prefix > G.thr) G.thr = prefix;
+  int pid = -1;
+  if (sb_l >= 0 && first_l < nvis[sb_l]) {
+    const int pg = p.block_table[static_cast<size_t>(sb_l) * p.max_blocks + first_l / kPerPage];
+    if (pg >= 0 && pg < p.num_pages) pid = pg;
+    else report(p.d_status, DSV4_DEV_BAD_PAGE);
   }
-  named_bar_sync(bar, kGroupThreads);
-}
-
-template <int H>
-__device__ void group_flush(TcSmem<H> &S, const TcParams &p, int gi, int b, int gt) {
-  GroupState &G = S.gs[gi];
-  const int bar = 1 + gi;
-  named_bar_sync(bar, kGroupThreads);
-  if (G.cnt > p.k) group_compact(S, gi, p.k, gt);
-  const int nout = G.cnt;
-  if (gt == 0) G.out_base = atomicAdd(&p.cand_count[b], nout);
-  named_bar_sync(bar, kGroupThreads);
-  const int base = G.out_base;
-  if (base + nout > p.stride) {
-    if (gt == 0) report(p.d_status, DSV4_DEV_BAD_LENGTH);
-  } else {
-    for (int i = gt; i < nout; i += kGroupThreads) p.cand[static_cast<size_t>(b) * p.stride + base + i] = S.cand[gi][i];
-  }
-  named_bar_sync(bar, kGroupThreads);
+  return pid;
 }
 
 template <int H>
@@ -338,13 +254,21 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   for (int b = tid; b < p.B; b += kIxThreads)
     nvis[b] = visible_entries(p.n_entries, p.pos, p.m, b, capacity, p.d_status, blockIdx.x == 0);
   __syncthreads();
-  if (tid == 0) {
-    long long acc = 0;
-    for (int b = 0; b < p.B; ++b) {
-      prefix[b] = acc;
-      acc += (nvis[b] + kTile - 1) / kTile;
+  if (warp == 0) {  // tiles per sequence, scanned by one warp
+    long long carry = 0;
+    for (int b0 = 0; b0 < p.B; b0 += 32) {
+      const int b = b0 + lane;
+      const long long c = b < p.B ? (nvis[b] + kTile - 1) / kTile : 0;
+      long long v = c;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long u = __shfl_up_sync(0xFFFFFFFFu, v, o);
+        if (lane >= o) v += u;
+      }
+      if (b < p.B) prefix[b] = carry + v - c;
+      carry += __shfl_sync(0xFFFFFFFFu, v, 31);
     }
-    prefix[p.B] = acc;
+    if (lane == 0) prefix[p.B] = carry;
   }
   tc_fence_before();
   __syncthreads();
@@ -355,44 +279,27 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   const long long t0 = (T * blockIdx.x) / G, t1 = (T * (blockIdx.x + 1)) / G;
 
   if (warp == 0) {
-    // ---------------- producer. Lane 0 issues the key TMA of stage k; the 32 lanes copy
-    // the key scales of stage k into scale slot k % kSlots with cp.async (two 16-byte copies
-    // per lane), each lane's copies arriving on the slot's barrier when they land, so
-    // neither the block-table nor the scale latency stalls the key stream.
-    // Page ids of stage k+1 are fetched while stage k is issued. A page that is invalid
-    // or starts past the visible entries gets scale 0 and a zero-filled key box.
+    // ---------------- producer. Lane 0 issues the key TMA of stage k (one box per 64-row
+    // page; an invalid page, or one past the visible entries, takes a zero-filled
+    // out-of-range box). All 32 lanes copy the stage's key scales with cp.async, each
+    // arriving on the slot's barrier when its copies land.
     const int oob_row = p.num_pages * kPerPage;
     StageIter it, ahead;
     it.init(prefix, p.B, t0, t1);
     ahead = it;
-    int ab, ant;
-    long long alt0;
-    bool anew, aend;
-    // page id of this lane's page in the next stage (lanes 0..3)
-    auto fetch_pid = [&](int sb, long long lt0, int nt) -> int {
-      int pid = -1;
-      if (lane < nt * kStageTiles) {
-        const int64_t first = lt0 * kTile + static_cast<int64_t>(lane) * kPerPage;
-        if (first < nvis[sb]) {
-          const int pg = p.block_table[static_cast<size_t>(sb) * p.max_blocks + first / kPerPage];
-          if (pg >= 0 && pg < p.num_pages) pid = pg;
-          else report(p.d_status, DSV4_DEV_BAD_PAGE);
-        }
-      }
-      return pid;
-    };
-    int pid_next = -1;
-    if (ahead.next(prefix, ab, alt0, ant, anew, aend)) pid_next = fetch_pid(ab, alt0, ant);
+    int batch_cur = load_page_batch(p, prefix, nvis, ahead, lane);
+    int batch_next = load_page_batch(p, prefix, nvis, ahead, lane);
     int seg = -1;
     long long k = 0;
-    bool stop = false;
     int sb, nt;
     long long lt0;
     bool new_seg, seg_end;
-    while (!stop && it.next(prefix, sb, lt0, nt, new_seg, seg_end)) {
-      const int pid = pid_next;
-      pid_next = -1;
-      if (ahead.next(prefix, ab, alt0, ant, anew, aend)) pid_next = fetch_pid(ab, alt0, ant);
+    while (it.next(prefix, sb, lt0, nt, new_seg, seg_end)) {
+      const int bs = static_cast<int>(k % kBatchStages);
+      if (bs == 0 && k > 0) {
+        batch_cur = batch_next;
+        batch_next = load_page_batch(p, prefix, nvis, ahead, lane);
+      }
       const int slot = static_cast<int>(k % kSlots);
       int ok = 1;
       if (lane == 0 && k >= kSlots &&
@@ -401,8 +308,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
       if (!ok) break;
       {  // scales of stage k: lane l copies 2 x 16 bytes of page l / 8
-        const int pg_slot = lane >> 3;  // 0..3 = tile * 2 + half
-        const int my_pid = __shfl_sync(0xFFFFFFFFu, pid, pg_slot);
+        const int pg_slot = lane >> 3;
+        const int my_pid = __shfl_sync(0xFFFFFFFFu, batch_cur, bs * kStagePages + pg_slot);
         float *dst = &S.sig[slot][pg_slot * kPerPage + (lane & 7) * 8];
         if (my_pid >= 0) {
           const float *src = p.k_scales + static_cast<size_t>(my_pid) * kPerPage + (lane & 7) * 8;
@@ -415,10 +322,10 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
           mbar_arrive(&S.sfull[slot]);
         }
       }
-      int rows[kStageTiles * 2];
+      int rows[kStagePages];
 #pragma unroll
-      for (int i = 0; i < kStageTiles * 2; ++i) {
-        const int v = __shfl_sync(0xFFFFFFFFu, pid, i);
+      for (int i = 0; i < kStagePages; ++i) {
+        const int v = __shfl_sync(0xFFFFFFFFu, batch_cur, bs * kStagePages + i);
         rows[i] = v >= 0 ? v * kPerPage : oob_row;
       }
       if (lane == 0) {
@@ -443,10 +350,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
         }
       }
       ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok) {
-        stop = true;
-        break;
-      }
+      if (!ok) break;
       ++k;
     }
     asm volatile("cp.async.wait_all;" ::: "memory");
@@ -477,13 +381,12 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
         const int a = static_cast<int>(k % kGroups);
         if (k >= kGroups && !mbar_wait(&S.tempty[a], static_cast<uint32_t>((k / kGroups - 1) & 1), &S.abort_flag)) break;
         tc_fence_after();
-        const uint32_t b0 = smem_u32(S.q[seg & 1]);
+        const uint64_t bq = sw128_desc(smem_u32(S.q[seg & 1]), 16, 1024);
         for (int t = 0; t < nt; ++t) {
-          const uint32_t a0 = smem_u32(S.stage[s][t]);
+          const uint64_t ak = sw128_desc(smem_u32(S.stage[s][t]), 16, 1024);
 #pragma unroll
-          for (int kk = 0; kk < kRowBytes / 32; ++kk)
-            mma_e4m3(tmem + (a * kStageTiles + t) * H, sw128_desc(a0 + kk * 32, 16, 1024),
-                     sw128_desc(b0 + kk * 32, 16, 1024), idesc, kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kRowBytes / 32; ++kk)  // K step of 32 bytes = +2 in the descriptor
+            mma_e4m3(tmem + (a * kStageTiles + t) * H, ak + 2 * kk, bq + 2 * kk, idesc, kk > 0 ? 1u : 0u);
         }
         mma_commit(&S.empty[s]);
         mma_commit(&S.tfull[a]);
@@ -493,94 +396,75 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
     }
   } else {
     // ---------------- epilogue groups (warps 2..5: group 0, warps 6..9: group 1). Group gi
-    // scores the stages k with k % 2 == gi and keeps its own running top-k per sequence.
+    // scores the stages k with k % 2 == gi: each thread one entry row, the H accumulators
+    // of its row weighted by c_h = w_h * scale_q[h] after ReLU, times the key's scale.
     const int gi = (warp - 2) / 4;
-    const int gt = tid - 64 - gi * kGroupThreads;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
-    const int bar = 1 + gi;
-    GroupState &GS = S.gs[gi];
+    float *coef = S.coef[warp - 2];
     StageIter it;
     it.init(prefix, p.B, t0, t1);
     int sb, nt, cur_b = -1;
     long long lt0, k = 0;
     bool new_seg, seg_end;
-    unsigned long long thr = 1;
     while (it.next(prefix, sb, lt0, nt, new_seg, seg_end)) {
       const long long kk = k++;
       if (kk % kGroups != gi) continue;
-      if (sb != cur_b) {
-        if (cur_b >= 0) group_flush(S, p, gi, cur_b, gt);
+      if (sb != cur_b) {  // this warp's own copy of the sequence's head coefficients
         cur_b = sb;
-        for (int h = gt; h < H; h += kGroupThreads) {
+        __syncwarp();
+        for (int h = lane; h < H; h += 32) {
           const float qs = p.q_scale ? p.q_scale[static_cast<size_t>(sb) * H + h] : 1.0f;
-          S.coef[gi][h] = load_one_f(p.w, p.w_dt, static_cast<size_t>(sb) * H + h) * qs;
+          coef[h] = load_one_f(p.w, p.w_dt, static_cast<size_t>(sb) * H + h) * qs;
         }
-        if (gt == 0) { GS.cnt = 0; GS.thr = 1; }
-        thr = 1;
-        named_bar_sync(bar, kGroupThreads);
+        __syncwarp();
       }
       const int slot = static_cast<int>(kk % kSlots);
       bool ok = mbar_wait(&S.sfull[slot], static_cast<uint32_t>((kk / kSlots) & 1), &S.abort_flag);
       ok = mbar_wait(&S.tfull[gi], static_cast<uint32_t>((kk / kGroups) & 1), &S.abort_flag) && ok;
-      ok = __all_sync(0xFFFFFFFFu, ok);
-      unsigned long long key[kStageTiles] = {0ull, 0ull};
-      if (ok) {
-        tc_fence_after();
-        const float4 *cf4 = reinterpret_cast<const float4 *>(S.coef[gi]);
-        // one tile at a time keeps 64 accumulator registers live, not 128
-#pragma unroll
-        for (int t = 0; t < kStageTiles; ++t) {
-          if (t < nt) {
-            uint32_t r[H];
-            const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + (gi * kStageTiles + t) * H;
-            tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-            if (H > 32) tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32 % H]));
-            const float sc = S.sig[slot][t * kTile + row];
-            tmem_ld_wait();
-            float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 short chains, not one of H
-#pragma unroll
-            for (int i = 0; i < H; i += 4) {
-              const float4 c = cf4[i / 4];
-              part[0] = fmaf(c.x, fmaxf(__uint_as_float(r[i]), 0.f), part[0]);
-              part[1] = fmaf(c.y, fmaxf(__uint_as_float(r[i + 1]), 0.f), part[1]);
-              part[2] = fmaf(c.z, fmaxf(__uint_as_float(r[i + 2]), 0.f), part[2]);
-              part[3] = fmaf(c.w, fmaxf(__uint_as_float(r[i + 3]), 0.f), part[3]);
-            }
-            const float score = ((part[0] + part[1]) + (part[2] + part[3])) * sc;
-            const int64_t j = (lt0 + t) * kTile + row;
-            if (j < nvis[sb] && sc > 0.f) key[t] = topk_key(score, static_cast<uint32_t>(j));
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) {
-          mbar_arrive(&S.tempty[gi]);
-          mbar_arrive(&S.sempty[slot]);
-        }
-      } else if (lane == 0) {
-        S.abort_flag = 1;
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        if (lane == 0) S.abort_flag = 1;
+        break;
       }
-      // insert the keys that beat the group's threshold
+      tc_fence_after();
+      float score[kStageTiles];
+      const float4 *cf4 = reinterpret_cast<const float4 *>(coef);
 #pragma unroll
       for (int t = 0; t < kStageTiles; ++t) {
-        const bool pass = key[t] != 0ull && key[t] >= thr;
-        const unsigned bal = __ballot_sync(0xFFFFFFFFu, pass);
-        int base = 0;
-        if (lane == 0 && bal) base = atomicAdd(&GS.cnt, __popc(bal));
-        base = __shfl_sync(0xFFFFFFFFu, base, 0);
-        if (pass) S.cand[gi][base + __popc(bal & ((1u << lane) - 1u))] = key[t];
+        score[t] = -INFINITY;
+        if (t < nt) {
+          uint32_t r[H];
+          const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + (gi * kStageTiles + t) * H;
+          tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+          if (H > 32) tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32 % H]));
+          const float sc = S.sig[slot][t * kTile + row];
+          tmem_ld_wait();
+          float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 short chains, not one of H
+#pragma unroll
+          for (int i = 0; i < H; i += 4) {
+            const float4 c = cf4[i / 4];
+            part[0] = fmaf(c.x, fmaxf(__uint_as_float(r[i]), 0.f), part[0]);
+            part[1] = fmaf(c.y, fmaxf(__uint_as_float(r[i + 1]), 0.f), part[1]);
+            part[2] = fmaf(c.z, fmaxf(__uint_as_float(r[i + 2]), 0.f), part[2]);
+            part[3] = fmaf(c.w, fmaxf(__uint_as_float(r[i + 3]), 0.f), part[3]);
+          }
+          if (sc > 0.f) score[t] = ((part[0] + part[1]) + (part[2] + part[3])) * sc;
+        }
       }
-      // one group barrier per stage: abort check, and compaction when the buffer could
-      // not take another stage (abort_flag is read after the barrier by every warp)
-      named_bar_sync(bar, kGroupThreads);
-      if (gt == 0) GS.stop = S.abort_flag;
-      named_bar_sync(bar, kGroupThreads);
-      if (GS.stop) break;
-      if (GS.cnt > kCapG - kStageTiles * kTile) group_compact(S, gi, p.k, gt);
-      thr = GS.thr;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        mbar_arrive(&S.tempty[gi]);
+        mbar_arrive(&S.sempty[slot]);
+      }
+      const int64_t nv = nvis[sb];
+      float *out = p.scores + static_cast<size_t>(sb) * p.ld;
+#pragma unroll
+      for (int t = 0; t < kStageTiles; ++t) {
+        const int64_t j = (lt0 + t) * kTile + row;
+        if (t < nt && j < nv) out[j] = score[t];
+      }
     }
-    if (cur_b >= 0 && !GS.stop) group_flush(S, p, gi, cur_b, gt);
   }
 
   if (tid == 0 && S.abort_flag) report(p.d_status, DSV4_DEV_TIMEOUT);
@@ -590,6 +474,230 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
     tc_fence_after();
     tmem_dealloc(tmem, kGroups * kStageTiles * H);
   }
+}
+
+// ------------------------------------------------------------------------------------
+// Top-k over the score buffer: one thread-block cluster of cs CTAs per sequence, CTA r
+// holding entries [r * slice, (r + 1) * slice) in shared memory as order-preserving keys
+// (0 = not a candidate). An MSB-first byte radix select finds the k-th largest key with
+// the cluster's histograms summed through distributed shared memory; kept are the keys
+// above its class and, of the class, the lowest indices. Each warp walks a contiguous
+// segment of the slice 32 keys at a time, so ballots give every kept key its rank in index
+// order, and per-CTA counts exchanged in the cluster give each slice its offset: the
+// output is in ascending entry order and does not depend on thread timing.
+
+constexpr int kTkThreads = 1024;
+constexpr int kTkWarps = kTkThreads / 32;
+constexpr int kTkSlice = 49152;  // largest slice per CTA (192 KB of keys)
+constexpr int kTkMaxCluster = 16;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// every thread of every CTA of the cluster; orders shared-memory writes before it with reads after it
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// a shared int of CTA `rank` of this cluster
+__device__ __forceinline__ int ld_cluster(const int *p, uint32_t rank) {
+  uint32_t ra;
+  int v;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+  return v;
+}
+__device__ __forceinline__ int warp_sum_int(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+__global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float *scores, int64_t ld,
+                                                                   const int32_t *n_entries, const int32_t *pos,
+                                                                   int m, int64_t capacity, int k, int slice,
+                                                                   int32_t *idx, float *out_scores, uint32_t *d_status) {
+  extern __shared__ uint32_t keys[];  // [slice]
+  __shared__ int hist[2][256];        // this CTA's histogram of the current pass (double buffered)
+  __shared__ int ghist[256];          // the cluster's
+  __shared__ int xch[2];              // read by the other CTAs: class members, kept keys
+  __shared__ int warp_cnt[kTkWarps], warp_base[kTkWarps];
+  __shared__ int sel_digit, sel_above, sel_count, bcast;
+  const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const uint32_t rank = cluster_rank(), cs = cluster_size();
+  const int64_t n = visible_entries(n_entries, pos, m, b, capacity, d_status, rank == 0 && tid == 0);
+  const int64_t lo = static_cast<int64_t>(rank) * slice;
+  const int cnt = static_cast<int>(n > lo ? (n - lo < slice ? n - lo : slice) : 0);
+  const float *src = scores + static_cast<size_t>(b) * ld + lo;
+  for (int i = tid * 4; i < cnt; i += kTkThreads * 4) {
+    float v[4];
+    if (i + 4 <= cnt) {
+      const float4 f = __ldcs(reinterpret_cast<const float4 *>(src + i));
+      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
+    } else {
+#pragma unroll
+      for (int u = 0; u < 4; ++u) v[u] = i + u < cnt ? src[i + u] : -INFINITY;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) keys[i + u] = isfinite(v[u]) ? float_order_key(v[u]) : 0u;
+  }
+  const int seg = (cnt + kTkWarps * 32 - 1) / (kTkWarps * 32) * 32;  // keys per warp, a multiple of 32
+  const int w0 = warp * seg, w1 = min(cnt, w0 + seg);
+  // one radix pass: the cluster histogram of digit `shift` over keys matching prefix/mask;
+  // returns (in sel_*) the digit holding the need-th largest key
+  uint32_t prefix = 0, mask = 0;
+  int need = 0, total_valid = 0, kk = 0;
+  auto pass = [&](int shift, int par) {
+    for (int i = tid; i < 256; i += kTkThreads) hist[par][i] = 0;
+    __syncthreads();
+    for (int i0 = 0; i0 < cnt; i0 += kTkThreads) {
+      const int i = i0 + tid;
+      int bin = 256;
+      if (i < cnt) {
+        const uint32_t key = keys[i];
+        if (key != 0u && (key & mask) == prefix) bin = static_cast<int>((key >> shift) & 0xFF);
+      }
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, bin);
+      if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[par][bin], __popc(peers));
+    }
+    cluster_sync_all();
+    if (tid < 256) {
+      int s = 0;
+      for (uint32_t r = 0; r < cs; ++r) s += ld_cluster(&hist[par][tid], r);
+      ghist[tid] = s;
+    }
+    __syncthreads();
+  };
+  auto pick = [&](int want) {  // warp 0: the digit holding the want-th largest key
+    if (tid < 32) {
+      int c[8], tot = 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) { c[u] = ghist[255 - tid * 8 - u]; tot += c[u]; }
+      int incl = tot;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (tid >= o) incl += v;
+      }
+      int run = incl - tot;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (run < want && run + c[u] >= want) {
+          sel_digit = 255 - tid * 8 - u;
+          sel_above = run;
+          sel_count = c[u];
+        }
+        run += c[u];
+      }
+      const int all = __shfl_sync(0xFFFFFFFFu, incl, 31);
+      if (tid == 0) bcast = all;
+    }
+    __syncthreads();
+  };
+  // first pass: also counts the valid keys of the whole sequence
+  pass(24, 0);
+  if (tid == 0) sel_count = -1;
+  __syncthreads();
+  pick(1 << 30);  // total in bcast; the digit choice is redone below once k is known
+  total_valid = bcast;
+  kk = total_valid < k ? total_valid : k;
+  need = kk;
+  const bool partial = kk < total_valid;
+  if (partial) {
+    pick(need);
+    int par = 0;
+    for (int shift = 24;; shift -= 8) {
+      prefix |= static_cast<uint32_t>(sel_digit) << shift;
+      mask |= 0xFFu << shift;
+      need -= sel_above;
+      const int cntd = sel_count;
+      __syncthreads();
+      if (cntd == need || shift == 0) break;  // the whole class is taken, or the key is exact
+      par ^= 1;
+      pass(shift - 8, par);
+      pick(need);
+    }
+  }
+  auto above = [&](uint32_t key) { return key != 0u && (!partial || (key & mask) > prefix); };
+  auto in_class = [&](uint32_t key) { return partial && key != 0u && (key & mask) == prefix; };
+  // class members before this CTA and before each warp
+  {
+    int e = 0;
+    for (int i = w0 + lane; i < w1; i += 32) e += in_class(keys[i]);
+    e = warp_sum_int(e);
+    if (lane == 0) warp_cnt[warp] = e;
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int w = 0; w < kTkWarps; ++w) { warp_base[w] = run; run += warp_cnt[w]; }
+      xch[0] = run;
+    }
+    cluster_sync_all();
+    if (tid == 0) {
+      int before = 0;
+      for (uint32_t r = 0; r < rank; ++r) before += ld_cluster(&xch[0], r);
+      bcast = before;
+    }
+    __syncthreads();
+  }
+  const int eq_before = bcast + warp_base[warp];
+  __syncthreads();
+  // kept keys of each warp, then of the CTA, then the CTA's offset in the cluster
+  auto walk = [&](bool write, int out0) {
+    int e = eq_before, kept = 0;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+      const int i = i0 + lane;
+      const uint32_t key = i < w1 ? keys[i] : 0u;
+      const bool cl = in_class(key);
+      const unsigned clb = __ballot_sync(0xFFFFFFFFu, cl);
+      const bool keep = above(key) || (cl && e + __popc(clb & ((1u << lane) - 1u)) < need);
+      e += __popc(clb);
+      const unsigned kb = __ballot_sync(0xFFFFFFFFu, keep);
+      if (write && keep) {
+        const int at = out0 + kept + __popc(kb & ((1u << lane) - 1u));
+        if (at < k) {
+          idx[static_cast<size_t>(b) * k + at] = static_cast<int32_t>(lo + i);
+          if (out_scores) out_scores[static_cast<size_t>(b) * k + at] = order_key_to_float(key);
+        }
+      }
+      kept += __popc(kb);
+    }
+    return kept;
+  };
+  const int my_kept = walk(false, 0);
+  if (lane == 0) warp_cnt[warp] = my_kept;
+  __syncthreads();
+  if (tid == 0) {
+    int run = 0;
+    for (int w = 0; w < kTkWarps; ++w) { warp_base[w] = run; run += warp_cnt[w]; }
+    xch[1] = run;
+  }
+  cluster_sync_all();
+  if (tid == 0) {
+    int before = 0, all = 0;
+    for (uint32_t r = 0; r < cs; ++r) {
+      const int v = ld_cluster(&xch[1], r);
+      if (r < rank) before += v;
+      all += v;
+    }
+    sel_above = before;
+    sel_count = all;
+  }
+  __syncthreads();
+  walk(true, sel_above + warp_base[warp]);
+  if (rank == 0) {
+    for (int i = sel_count + tid; i < k; i += kTkThreads) {
+      idx[static_cast<size_t>(b) * k + i] = -1;
+      if (out_scores) out_scores[static_cast<size_t>(b) * k + i] = -INFINITY;
+    }
+  }
+  cluster_sync_all();  // no CTA leaves while another may still read its shared memory
 }
 
 // ------------------------------------------------------------------------------------
@@ -715,20 +823,34 @@ bool make_rows_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t b
 
 int tc_grid() { return sm_count(); }
 
+int64_t capacity_of(const IndexerLaunch &p) {
+  return static_cast<int64_t>(p.max_blocks) * (DSV4_PAGE_POSITIONS / p.m);
+}
+int64_t score_ld(const IndexerLaunch &p) { return (capacity_of(p) + 3) / 4 * 4; }
+
+// CTAs per sequence of the top-k cluster: enough for a slice to fit in shared memory, and
+// as many as keep the batch within one wave of SMs (a power of two, at most 16)
+int tk_cluster(const IndexerLaunch &p) {
+  int need = 1;
+  while (static_cast<int64_t>(need) * kTkSlice < capacity_of(p)) need <<= 1;
+  int par = 1;
+  while (par < 8 && static_cast<int64_t>(par) * 2 * p.B <= sm_count()) par <<= 1;
+  return need > par ? need : par;
+}
+int tk_slice(const IndexerLaunch &p) {
+  const int cs = tk_cluster(p);
+  return static_cast<int>((capacity_of(p) + cs - 1) / cs + 3) / 4 * 4;
+}
+
+// candidate list length per sequence (CUDA-core path: every entry)
 int64_t cand_stride(const IndexerLaunch &p) {
-  const int64_t capacity = static_cast<int64_t>(p.max_blocks) * (DSV4_PAGE_POSITIONS / p.m);
-  if (indexer_uses_tensor_cores(p)) {
-    // one list of at most k keys per (CTA, epilogue group) that touches the sequence
-    const int64_t tiles = (capacity + kTile - 1) / kTile;
-    const int64_t ctas = tiles < tc_grid() ? tiles : tc_grid();
-    return (ctas > 0 ? ctas : 1) * kGroups * p.k;
-  }
+  if (indexer_uses_tensor_cores(p)) return 0;
+  const int64_t capacity = capacity_of(p);
   return capacity > 0 ? capacity : 1;
 }
 
 template <int H>
-cudaError_t launch_tc(const IndexerLaunch &p, unsigned long long *cand, int64_t stride, int *cand_count,
-                      cudaStream_t st) {
+cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st) {
   TcParams tp;
   if (!make_rows_map(&tp.tmap_k, p.k_pages, static_cast<uint64_t>(p.num_pages) * kPerPage, kPerPage))
     return cudaErrorInvalidValue;
@@ -741,13 +863,11 @@ cudaError_t launch_tc(const IndexerLaunch &p, unsigned long long *cand, int64_t 
   tp.w = p.w;
   tp.w_dt = p.w_dt;
   tp.B = p.B;
-  tp.k = p.k;
   tp.m = p.m;
   tp.n_entries = p.n_entries;
   tp.pos = p.pos;
-  tp.cand = cand;
-  tp.stride = stride;
-  tp.cand_count = cand_count;
+  tp.scores = scores;
+  tp.ld = score_ld(p);
   tp.d_status = p.d_status;
   const size_t smem = sizeof(TcSmem<H>) + 1024 + (2 * static_cast<size_t>(p.B) + 1) * 8;
   cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -760,36 +880,66 @@ cudaError_t launch_tc(const IndexerLaunch &p, unsigned long long *cand, int64_t 
 
 bool indexer_uses_tensor_cores(const IndexerLaunch &p) {
   return p.k_dt == DSV4_FP8E4M3 && p.q_dt == DSV4_FP8E4M3 && p.Dq == kRowBytes &&
-         (p.H == 32 || p.H == 64) && p.m == 4 && p.k >= 1 && p.k <= kMaxKTc && p.q_rope_dims == 0 &&
-         p.B <= 512;
+         (p.H == 32 || p.H == 64) && p.m == 4 && p.k >= 1 && p.k <= 2048 && p.q_rope_dims == 0 &&
+         p.B <= 512 && static_cast<int64_t>(p.max_blocks) * (DSV4_PAGE_POSITIONS / p.m) <= kTkMaxCluster * kTkSlice;
 }
 
 size_t indexer_workspace_bytes(const IndexerLaunch &p) {
-  return align_up(static_cast<size_t>(p.B) * sizeof(int), 256) +
-         align_up(static_cast<size_t>(p.B) * cand_stride(p) * sizeof(unsigned long long), 256);
+  size_t bytes = align_up(static_cast<size_t>(p.B) * sizeof(int), 256) +
+                 align_up(static_cast<size_t>(p.B) * cand_stride(p) * sizeof(unsigned long long), 256);
+  if (indexer_uses_tensor_cores(p)) bytes += align_up(static_cast<size_t>(p.B) * score_ld(p) * sizeof(float), 256);
+  return bytes;
 }
 
-cudaError_t launch_indexer_topk(const IndexerLaunch &p, void *ws, cudaStream_t st) {
-  int *cand_count = static_cast<int *>(ws);
-  unsigned long long *cand = reinterpret_cast<unsigned long long *>(
-      static_cast<char *>(ws) + align_up(static_cast<size_t>(p.B) * sizeof(int), 256));
+cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t st) {
+  IndexerLaunch p = p0;
+  p.rope_theta1 = rope_theta1(p.rope_base, p.q_rope_dims);
+  char *w = static_cast<char *>(ws);
+  int *cand_count = reinterpret_cast<int *>(w);
+  w += align_up(static_cast<size_t>(p.B) * sizeof(int), 256);
+  unsigned long long *cand = reinterpret_cast<unsigned long long *>(w);
   const int64_t stride = cand_stride(p);
-  cudaError_t e = cudaMemsetAsync(cand_count, 0, static_cast<size_t>(p.B) * sizeof(int), st);
-  if (e != cudaSuccess) return e;
+  w += align_up(static_cast<size_t>(p.B) * stride * sizeof(unsigned long long), 256);
+  cudaError_t e = cudaSuccess;
   if (indexer_uses_tensor_cores(p)) {
-    if (p.H == 32) e = launch_tc<32>(p, cand, stride, cand_count, st);
-    else e = launch_tc<64>(p, cand, stride, cand_count, st);
+    float *scores = reinterpret_cast<float *>(w);
+    e = p.H == 32 ? launch_tc<32>(p, scores, st) : launch_tc<64>(p, scores, st);
+    if (e != cudaSuccess) return e;
+    const int cs = tk_cluster(p), slice = tk_slice(p);
+    const size_t tsmem = static_cast<size_t>(slice) * sizeof(uint32_t);
+    e = cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem);
+    if (e != cudaSuccess) return e;
+    if (cs > 8) {
+      e = cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B));
+    cfg.blockDim = dim3(kTkThreads);
+    cfg.dynamicSmemBytes = tsmem;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, topk_scores_kernel, static_cast<const float *>(scores), score_ld(p),
+                              p.n_entries, p.pos, p.m, capacity_of(p), p.k, slice, p.idx, p.scores, p.d_status);
   } else {
-    const int64_t capacity = static_cast<int64_t>(p.max_blocks) * (DSV4_PAGE_POSITIONS / p.m);
+    e = cudaMemsetAsync(cand_count, 0, static_cast<size_t>(p.B) * sizeof(int), st);
+    if (e != cudaSuccess) return e;
+    const int64_t capacity = capacity_of(p);
     dim3 grid(static_cast<unsigned>((capacity + 255) / 256), p.B);
     const size_t smem = (static_cast<size_t>(p.H) * p.Dq + p.H) * sizeof(float);
     e = cudaFuncSetAttribute(indexer_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     indexer_simt_kernel<<<grid, 256, smem, st>>>(p, cand, stride, cand_count);
     e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
   }
-  if (e != cudaSuccess) return e;
-  // stage up to ~200 KB of candidates in shared memory (the rest of the kernel's smem is small)
+  // merge candidate lists: stage up to ~200 KB of candidates in shared memory
   const int smem_keys = static_cast<int>(std::min<int64_t>(stride + kMaxSortK, 25600));
   const size_t ssmem = static_cast<size_t>(smem_keys) * sizeof(unsigned long long);
   e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);

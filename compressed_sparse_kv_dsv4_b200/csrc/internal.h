@@ -6,12 +6,20 @@
 #include <stddef.h>
 #include <stdint.h>
 
+#include <cmath>
+
 #include "../../include/dsv4.h"
 
 namespace dsv4 {
 
 // number of SMs of the current device (cached per device)
 int sm_count();
+
+// RoPE's angle step of pair 1, base^(-2/rope_dims), in float64 on the host; pair i turns by
+// pos * theta1^i. The launchers fill the rope_theta1 fields below from it.
+inline double rope_theta1(float base, int rope_dims) {
+  return rope_dims > 0 ? std::pow(static_cast<double>(base), -2.0 / rope_dims) : 1.0;
+}
 
 // ---------------------------------------------------------------- compressor / window
 struct CompressLaunch {
@@ -26,6 +34,7 @@ struct CompressLaunch {
   float eps;
   int rope_dims;
   float rope_base;
+  double rope_theta1 = 1.0;  // filled by the launcher
   float *state;
   int m, D, G;
   void *pages;
@@ -48,6 +57,7 @@ struct SwaLaunch {
   float eps;
   int rope_dims;
   float rope_base;
+  double rope_theta1 = 1.0;  // filled by the launcher
   void *rows;
   float *scales;
   int W, D;
@@ -67,6 +77,7 @@ struct PrologueLaunch {
   float eps;
   int rope_dims;
   float rope_base;
+  double rope_theta1 = 1.0, idx_rope_theta1 = 1.0;  // filled by the launcher
   float *state;
   int m, D, G;
   void *pages;
@@ -110,6 +121,7 @@ struct IndexerLaunch {
   const int32_t *pos;
   int q_rope_dims;
   float rope_base;
+  double rope_theta1 = 1.0;  // of q_rope_dims; filled by the launcher
   int32_t *idx;
   float *scores;
   uint32_t *d_status;
@@ -138,6 +150,7 @@ struct MqaLaunch {
   float softmax_scale;
   int rope_dims;
   float rope_base;
+  double rope_theta1 = 1.0;  // filled by the launcher
   void *out;
   dsv4_dtype out_dt;
   float *lse;

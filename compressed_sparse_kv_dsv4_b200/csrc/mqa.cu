@@ -91,10 +91,10 @@ __device__ __forceinline__ const uint8_t *key_row(const MqaLaunch &p, int b, con
 }
 
 // prefix[b] = number of 64-key chunks of sequences 0..b-1, prefix[B] = total; computed by
-// every thread of the CTA (contiguous slices of sequences, then a scan of the slices).
-// red: blockDim.x scratch values.
+// every thread of the CTA (contiguous slices of sequences, then a two-level shuffle scan of
+// the slice sums). red: 32 scratch values. blockDim.x is a multiple of 32.
 __device__ void chunk_prefix(const MqaLaunch &p, long long *prefix, long long *red, bool report_it) {
-  const int nt = blockDim.x, t = threadIdx.x;
+  const int nt = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int lo = static_cast<int>((static_cast<long long>(p.B) * t) / nt);
   const int hi = static_cast<int>((static_cast<long long>(p.B) * (t + 1)) / nt);
   long long mine = 0;
@@ -104,19 +104,26 @@ __device__ void chunk_prefix(const MqaLaunch &p, long long *prefix, long long *r
     prefix[b] = c;
     mine += c;
   }
-  red[t] = mine;
+  long long v = mine;  // inclusive scan within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const long long u = __shfl_up_sync(0xFFFFFFFFu, v, o);
+    if (lane >= o) v += u;
+  }
+  if (lane == 31) red[warp] = v;
   __syncthreads();
-  if (t == 0) {
-    long long acc = 0;
-    for (int i = 0; i < nt; ++i) {
-      const long long v = red[i];
-      red[i] = acc;
-      acc += v;
+  if (warp == 0) {
+    long long w = lane < (nt >> 5) ? red[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const long long u = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += u;
     }
-    prefix[p.B] = acc;
+    red[lane] = w;
   }
   __syncthreads();
-  long long acc = red[t];
+  long long acc = v - mine + (warp > 0 ? red[warp - 1] : 0);
+  if (t == nt - 1) prefix[p.B] = acc + mine;
   for (int b = lo; b < hi; ++b) {
     const long long c = prefix[b];
     prefix[b] = acc;
@@ -137,31 +144,25 @@ __device__ __forceinline__ int find_seq(const long long *prefix, int B, long lon
 // ------------------------------------------------------------------------------------
 // tensor-core kernel
 
-constexpr int kH = 64, kD = 512, kCh = 64, kThreads = 256;
+constexpr int kH = 64, kD = 512, kCh = 64;
 constexpr int kAtom = kCh * 128;  // one 64-dim column block of a 64-row tile: 8 KB
-constexpr int kMetaChunks = 8;
+constexpr int kMetaSlots = 4;     // chunks whose key metadata is resolved ahead
+// roles: warps 0-3 softmax + output (TMEM lane quadrant = warp), warps 4-7 gather, warp 8
+// MMA issue (and TMEM allocation), warp 9 key metadata
+constexpr int kSoftWarp0 = 0, kGatherWarp0 = 4, kMmaWarp = 8, kMetaWarp = 9;
+constexpr int kThreads = 320;
 
 struct alignas(1024) MqaSmem {
   uint8_t q[kD / 64][kH * 128];      // 64 KB, K-major SW128, 8 atoms of 64 dims
-  uint8_t k[2][kD / 64][kCh * 128];  // 2 x 64 KB
+  uint8_t k[2][kD / 64][kCh * 128];  // 2 x 64 KB key tiles (stage = chunk parity)
   uint8_t p[kH * 128];               // 8 KB: P[64 heads][64 keys], K-major SW128
-  const uint8_t *rowp[2][kCh];
-  float rscale[2][kCh];              // row scale of each key (0: no key)
-  // key metadata of up to kMetaChunks consecutive chunks, resolved together so the
-  // idx -> block table -> scale load chain is paid once per batch, not once per chunk
-  const uint8_t *mrow[kMetaChunks * kCh];
-  float mscale[kMetaChunks * kCh];
-  KeyList mkl[kMetaChunks];
-  int mb[kMetaChunks];
-  long long mlc[kMetaChunks];
-  long long meta_first;
-  int meta_n;
-  float cs[kD / 2], sn[kD / 2];
-  float qinv[kH];                    // 2^-e of the per-head query scale (fp16 operands)
-  float smax[2][2];                  // per-warp max row scale of a chunk being gathered
-  int ec[2];                         // chunk exponent: K rows hold code * scale * 2^-ec
-  unsigned qmax[kH];
-  uint64_t bar_s, bar_o;
+  const uint8_t *mrow[kMetaSlots][kCh];  // row address of each key of a chunk (nullptr: none)
+  float mscale[kMetaSlots][kCh];         // its row scale
+  float rscale[2][kCh];                  // row scale per key of a staged tile (0: no key)
+  int ec[2];                             // tile exponent: K rows hold code * scale * 2^-ec
+  float qinv[2][kH];                     // 2^-e of the per-head query scale, by segment parity
+  uint64_t meta_full[kMetaSlots], meta_empty[kMetaSlots];
+  uint64_t k_full[2], k_empty[2], q_full, q_empty, s_full, s_empty, p_full, o_full, o_empty;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -182,179 +183,494 @@ __device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// Resolve the row address and scale of every key of chunks [g0, g0 + n) (n <= kMetaChunks).
-__device__ void resolve_meta(const MqaTcParams &P, MqaSmem &S, const long long *prefix, long long g0, long long c1) {
-  const MqaLaunch &p = P.a;
-  const int tid = threadIdx.x;
-  const int n = static_cast<int>(c1 - g0 < kMetaChunks ? c1 - g0 : kMetaChunks);
-  if (tid < n) {
-    const int b = find_seq(prefix, p.B, g0 + tid);
-    S.mb[tid] = b;
-    S.mlc[tid] = g0 + tid - prefix[b];
-    S.mkl[tid] = key_list(p, b, false);
-  }
-  __syncthreads();
-  // the cached range changes only after every thread has passed the barrier above, that
-  // is, after every thread has taken its decision to resolve from the old range
-  if (tid == 0) {
-    S.meta_first = g0;
-    S.meta_n = n;
-  }
-  for (int i = tid; i < n * kCh; i += kThreads) {
-    const int c = i / kCh;
-    const KeyList &L = S.mkl[c];
-    const long long t = S.mlc[c] * kCh + (i % kCh);
-    float sc = 0.f;
-    const uint8_t *rp = t < L.nw + L.nsel ? key_row(p, S.mb[c], L, t, &sc) : nullptr;
-    S.mrow[i] = rp;
-    S.mscale[i] = rp ? sc : 0.f;
-  }
-  __syncthreads();
+// where chunk g sits: its sequence, and whether it opens / closes this CTA's run of it
+struct ChunkPos {
+  int b;
+  bool first, last;
+};
+__device__ __forceinline__ ChunkPos chunk_pos(const long long *prefix, int B, long long g, long long c0,
+                                              long long c1) {
+  ChunkPos c;
+  c.b = find_seq(prefix, B, g);
+  c.first = g == c0 || prefix[c.b] == g;
+  c.last = g + 1 == c1 || prefix[c.b + 1] == g + 1;
+  return c;
 }
 
-// Gather one 64-key chunk into a swizzled K-major tile. For fp8 rows the row scale is
-// folded in: tile row j = code_j * (scale_j * 2^-ec) in fp16, with ec the exponent of the
-// chunk's largest row scale, so every tile value stays within +-448.
-__device__ void gather_chunk(const MqaTcParams &P, MqaSmem &S, const long long *prefix, long long g, long long c1,
-                             int kb) {
-  const MqaLaunch &p = P.a;
-  const int tid = threadIdx.x;
-  if (g < S.meta_first || g >= S.meta_first + S.meta_n) resolve_meta(P, S, prefix, g, c1);
-  if (tid < kCh) {
-    const int i = static_cast<int>(g - S.meta_first) * kCh + tid;
-    const uint8_t *rp = S.mrow[i];
-    const float sc = S.mscale[i];
-    S.rowp[kb][tid] = rp;
-    S.rscale[kb][tid] = sc;
-    const float wm = warp_max(sc);
-    if ((tid & 31) == 0) S.smax[kb][tid >> 5] = wm;
-  }
-  __syncthreads();
-  uint8_t *kt = &S.k[kb][0][0];
-  if (p.kv_dt == DSV4_FP8E4M3) {
-    int ec = 0;
-    frexpf(fmaxf(S.smax[kb][0], S.smax[kb][1]), &ec);  // max scale = f * 2^ec, f in [0.5, 1)
-    if (tid == 0) S.ec[kb] = ec;
-    uint4 v[8];
+// ---- warp 9: row address and scale of every key of up to kMetaSlots chunks at a time.
+// The idx -> block table -> scale chain is staged over all keys of the batch, so its three
+// memory latencies are paid once per batch.
+__device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const long long *prefix, long long c0, long long c1) {
+  const int lane = threadIdx.x & 31;
+  const int per_page = DSV4_PAGE_POSITIONS / p.m;
+  const size_t esz = dtype_size(p.kv_dt);
+  constexpr int kKeys = kMetaSlots * 2;  // keys per lane per batch
+  for (long long g0 = c0; g0 < c1; g0 += kMetaSlots) {
+    const int nb = static_cast<int>(c1 - g0 < kMetaSlots ? c1 - g0 : kMetaSlots);
+    bool ok = true;
+    for (int i = 0; i < nb; ++i) {
+      const long long n = g0 + i - c0;
+      if (n >= kMetaSlots && lane == 0 &&
+          !mbar_wait(&S.meta_empty[n % kMetaSlots], static_cast<uint32_t>((n / kMetaSlots - 1) & 1), &S.abort_flag))
+        ok = false;
+    }
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) S.abort_flag = 1;
+      return;
+    }
+    int bc[kMetaSlots];
+    KeyList Lc[kMetaSlots];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int sid = i * kThreads + tid, row = sid >> 5, seg = sid & 31;
-      const uint8_t *rp = S.rowp[kb][row];
-      v[i] = rp ? __ldg(reinterpret_cast<const uint4 *>(rp + seg * 16)) : make_uint4(0, 0, 0, 0);
+    for (int i = 0; i < kMetaSlots; ++i) {
+      bc[i] = i < nb ? find_seq(prefix, p.B, g0 + i) : 0;
+      if (i < nb) Lc[i] = key_list(p, bc[i], false);
+    }
+    int bseq[kKeys];
+    int64_t j[kKeys];  // >= 0: entry index; -1: none; -2 - slot: window ring slot
+    int32_t page[kKeys];
+#pragma unroll
+    for (int u = 0; u < kKeys; ++u) {  // stage 1: key list position -> entry index (idx load)
+      const int i = u >> 1;
+      j[u] = -1;
+      bseq[u] = 0;
+      if (i < nb) {
+        const int b = bc[i];
+        const KeyList &L = Lc[i];
+        const int64_t t = (g0 + i - prefix[b]) * kCh + lane + 32 * (u & 1);
+        bseq[u] = b;
+        if (t < L.nw) {
+          const int64_t pw = L.pos - L.nw + 1 + t;
+          j[u] = -2 - (static_cast<int64_t>(b) * p.W + pw % p.W);
+        } else if (t - L.nw < L.nsel) {
+          const int64_t uu = t - L.nw;
+          int64_t e = uu;
+          if (p.idx) {
+            e = p.idx[static_cast<size_t>(b) * p.k + uu];
+            if (e >= L.n_entries) {
+              report(p.d_status, DSV4_DEV_BAD_INDEX);
+              e = -1;
+            }
+          }
+          j[u] = e < 0 ? -1 : e;
+        }
+      }
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int sid = i * kThreads + tid, row = sid >> 5, seg = sid & 31;
-      const __half2 sc2 = __float2half2_rn(ldexpf(S.rscale[kb][row], -ec));
-      const uint32_t w[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      uint32_t o[8];
+    for (int u = 0; u < kKeys; ++u) {  // stage 2: entry -> physical page (block table load)
+      page[u] = -1;
+      if (j[u] >= 0) {
+        page[u] = p.block_table[static_cast<size_t>(bseq[u]) * p.max_blocks + j[u] / per_page];
+        if (page[u] < 0 || page[u] >= p.num_pages) {
+          report(p.d_status, DSV4_DEV_BAD_PAGE);
+          page[u] = -1;
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kKeys; ++u) {  // stage 3: row address and scale
+      const int i = u >> 1;
+      if (i >= nb) continue;
+      const uint8_t *rp = nullptr;
+      float sc = 0.f;
+      if (j[u] <= -2) {
+        const size_t slot = static_cast<size_t>(-2 - j[u]);
+        rp = static_cast<const uint8_t *>(p.ring_rows) + slot * p.D * esz;
+        sc = p.kv_dt == DSV4_FP8E4M3 ? p.ring_scales[slot] : 1.0f;
+      } else if (page[u] >= 0) {
+        const size_t row = static_cast<size_t>(page[u]) * per_page + static_cast<size_t>(j[u] % per_page);
+        rp = static_cast<const uint8_t *>(p.pages) + row * p.D * esz;
+        sc = p.kv_dt == DSV4_FP8E4M3 ? p.scales[row] : 1.0f;
+      }
+      const int slot = static_cast<int>((g0 + i - c0) % kMetaSlots);
+      S.mrow[slot][lane + 32 * (u & 1)] = rp;
+      S.mscale[slot][lane + 32 * (u & 1)] = rp ? sc : 0.f;
+    }
+    __syncwarp();
+    if (lane == 0)
+      for (int i = 0; i < nb; ++i) mbar_arrive(&S.meta_full[(g0 + i - c0) % kMetaSlots]);
+  }
+}
+
+// ---- warps 4-7 (gw = 0..3): query of a new segment and the key tiles.
+// Query: warp gw owns heads 16gw .. 16gw+15; lane l owns 16-byte runs (8 dims) l and l + 32
+// of each. The raw bf16 runs are copied into their swizzled homes, then rotated by RoPE_pos
+// and stored as bf16, or as fp16 scaled per head by a power of two (qinv undoes it in the
+// logits) so that |q| < 2^14 whatever the input range. RoPE pairs never straddle a run.
+__device__ __forceinline__ void query_issue(const MqaLaunch &p, MqaSmem &S, int b, int gw, int lane) {
+  const uint16_t *q = static_cast<const uint16_t *>(p.q) + static_cast<size_t>(b) * kH * kD;
+#pragma unroll 4
+  for (int hh = 0; hh < 16; ++hh) {
+    const int h = gw * 16 + hh;
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int seg = lane + 32 * r;
+      cp_async16(&S.q[seg >> 3][0] + sw128_offset(h, seg & 7), q + (static_cast<size_t>(h) * kD + seg * 8));
+    }
+  }
+  cp_async_commit();
+}
+
+__device__ __forceinline__ void query_finish(const MqaLaunch &p, MqaSmem &S, int64_t pos, int par, int gw, int lane) {
+  const bool f16 = fp16_operands(p);
+  const int rope0 = kD - p.rope_dims;
+  float c[2][4], sn[2][4];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int d0 = (lane + 32 * r) * 8;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      c[r][u] = 1.f;
+      sn[r][u] = 0.f;
+      if (d0 >= rope0) rope_cos_sin(pos, (d0 + 2 * u - rope0) >> 1, p.rope_theta1, &c[r][u], &sn[r][u]);
+    }
+  }
+  cp_async_wait_all();
+  __syncwarp();
+#pragma unroll 1
+  for (int hh = 0; hh < 16; ++hh) {
+    const int h = gw * 16 + hh;
+    float x[2][8];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int seg = lane + 32 * r;
+      const uint4 w = *reinterpret_cast<const uint4 *>(&S.q[seg >> 3][0] + sw128_offset(h, seg & 7));
+      const uint32_t v[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[u] & 0xFFFF), __NV_E4M3);
-        __half2_raw c = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[u] >> 16), __NV_E4M3);
-        __half2 ha = __hmul2(*reinterpret_cast<__half2 *>(&a), sc2);
-        __half2 hc = __hmul2(*reinterpret_cast<__half2 *>(&c), sc2);
-        o[2 * u] = *reinterpret_cast<uint32_t *>(&ha);
-        o[2 * u + 1] = *reinterpret_cast<uint32_t *>(&hc);
+        const float x0 = __uint_as_float(v[u] << 16), x1 = __uint_as_float(v[u] & 0xFFFF0000u);
+        x[r][2 * u] = x0 * c[r][u] - x1 * sn[r][u];
+        x[r][2 * u + 1] = x0 * sn[r][u] + x1 * c[r][u];
       }
-      const int atom = seg >> 2, c0 = (seg & 3) * 2;
-      uint8_t *base = kt + atom * kAtom;
-      *reinterpret_cast<uint4 *>(base + sw128_offset(row, c0)) = make_uint4(o[0], o[1], o[2], o[3]);
-      *reinterpret_cast<uint4 *>(base + sw128_offset(row, c0 + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
     }
-  } else {  // bf16 rows: straight 16-byte copies into the swizzled tile
-    if (tid == 0) S.ec[kb] = 0;
-    uint4 v[16];
+    float qs = 1.0f, qi = 1.0f;
+    if (f16) {
+      float am = 0.f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int sid = i * kThreads + tid, row = sid >> 6, seg = sid & 63;
-      const uint8_t *rp = S.rowp[kb][row];
-      v[i] = rp ? __ldg(reinterpret_cast<const uint4 *>(rp + seg * 16)) : make_uint4(0, 0, 0, 0);
+      for (int u = 0; u < 8; ++u) am = fmaxf(am, fmaxf(fabsf(x[0][u]), fabsf(x[1][u])));
+      am = warp_max(am);
+      int e = 0;
+      if (am > 0.f) frexpf(am, &e);  // am < 2^e
+      qi = am > 0.f ? ldexpf(1.0f, e - 14) : 1.0f;
+      qs = am > 0.f ? ldexpf(1.0f, 14 - e) : 1.0f;
     }
+    if (lane == 0) S.qinv[par][h] = qi;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int sid = i * kThreads + tid, row = sid >> 6, seg = sid & 63;
-      *reinterpret_cast<uint4 *>(kt + (seg >> 3) * kAtom + sw128_offset(row, seg & 7)) = v[i];
-    }
-  }
-}
-
-// rotated query of sequence b, K-major swizzled: bf16, or fp16 scaled per head by a power
-// of two (qinv[h] undoes it in the logits) so that |q| < 2^14 whatever the input range.
-// A bf16 query is loaded once, all 16 segments of a thread up front.
-__device__ void load_query(const MqaTcParams &P, MqaSmem &S, int b, int64_t pos) {
-  const MqaLaunch &p = P.a;
-  const int tid = threadIdx.x;
-  const int half = p.rope_dims / 2;
-  const bool f16 = fp16_operands(p);
-  const bool raw_bf16 = p.q_dt == DSV4_BF16;
-  uint4 raw[16];
-  if (raw_bf16) {
-    const uint16_t *q = static_cast<const uint16_t *>(p.q) + static_cast<size_t>(b) * kH * kD;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) raw[i] = __ldg(reinterpret_cast<const uint4 *>(q) + i * kThreads + tid);
-  }
-  for (int i = tid; i < half; i += kThreads) rope_cos_sin(pos, i, p.rope_dims, p.rope_base, &S.cs[i], &S.sn[i]);
-  if (tid < kH) S.qmax[tid] = 0u;
-  __syncthreads();
-  const int rope0 = kD - p.rope_dims;
-  for (int pass = f16 ? 0 : 1; pass < 2; ++pass) {
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int sid = i * kThreads + tid, h = sid >> 6, seg = sid & 63;
-      float x[8];
-      if (raw_bf16) {
-        const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          x[2 * k] = __uint_as_float(w[k] << 16);
-          x[2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
-        }
-      } else {
-        load_row_f<8>(p.q, p.q_dt, (static_cast<size_t>(b) * kH + h) * kD + seg * 8, x);
-      }
-      const int d0 = seg * 8;
-      if (d0 >= rope0) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int pi = (d0 + 2 * u - rope0) >> 1;
-          const float c = S.cs[pi], s = S.sn[pi];
-          const float x0 = x[2 * u], x1 = x[2 * u + 1];
-          x[2 * u] = x0 * c - x1 * s;
-          x[2 * u + 1] = x0 * s + x1 * c;
-        }
-      }
-      if (pass == 0) {  // per-head max |q| (32 lanes of a warp cover half a head)
-        float am = 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) am = fmaxf(am, fabsf(x[u]));
-        am = warp_max(am);
-        if ((tid & 31) == 0) atomicMax(&S.qmax[h], __float_as_uint(am));
-        continue;
-      }
+    for (int r = 0; r < 2; ++r) {
+      const int seg = lane + 32 * r;
       uint4 o;
       if (f16) {
-        const float qs = 1.0f / S.qinv[h];
-        o = make_uint4(pack_f16x2(x[0] * qs, x[1] * qs), pack_f16x2(x[2] * qs, x[3] * qs),
-                       pack_f16x2(x[4] * qs, x[5] * qs), pack_f16x2(x[6] * qs, x[7] * qs));
+        o = make_uint4(pack_f16x2(x[r][0] * qs, x[r][1] * qs), pack_f16x2(x[r][2] * qs, x[r][3] * qs),
+                       pack_f16x2(x[r][4] * qs, x[r][5] * qs), pack_f16x2(x[r][6] * qs, x[r][7] * qs));
       } else {
-        o = make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                       pack_bf16x2(x[6], x[7]));
+        o = make_uint4(pack_bf16x2(x[r][0], x[r][1]), pack_bf16x2(x[r][2], x[r][3]), pack_bf16x2(x[r][4], x[r][5]),
+                       pack_bf16x2(x[r][6], x[r][7]));
       }
       *reinterpret_cast<uint4 *>(&S.q[seg >> 3][0] + sw128_offset(h, seg & 7)) = o;
     }
-    if (pass == 0) {
-      __syncthreads();
-      if (tid < kH) {
-        int e = 0;
-        const float am = __uint_as_float(S.qmax[tid]);
-        if (am > 0.f) frexpf(am, &e);                         // am < 2^e
-        S.qinv[tid] = am > 0.f ? ldexpf(1.0f, e - 14) : 1.0f;  // scaled |q| < 2^14
-      }
-      __syncthreads();
+  }
+}
+
+// Key tile of one chunk: warp gw fills rows 16gw .. 16gw+15. fp8 rows (32 runs of 16
+// codes): lane l loads run l of each row and stores it as fp16 code * (scale * 2^-ec), ec
+// the exponent of the chunk's largest row scale, so every tile value stays within +-448.
+// bf16 rows (64 runs of 8 values) are copied as they are.
+__device__ __forceinline__ void gather_issue_bf16(const MqaSmem &S, uint8_t *kt, int ms, int gw, int lane) {
+#pragma unroll 4
+  for (int rr = 0; rr < 16; ++rr) {
+    const int row = gw * 16 + rr;
+    const uint8_t *rp = S.mrow[ms][row];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int seg = lane + 32 * r;
+      uint8_t *dst = kt + (seg >> 3) * kAtom + sw128_offset(row, seg & 7);
+      if (rp) cp_async16(dst, rp + seg * 16);
+      else *reinterpret_cast<uint4 *>(dst) = make_uint4(0, 0, 0, 0);
     }
   }
-  if (!f16 && tid < kH) S.qinv[tid] = 1.0f;
+  cp_async_commit();
+}
+
+__device__ __forceinline__ void gather_load_fp8(const MqaSmem &S, int ms, int gw, int lane, uint4 (&v)[16]) {
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) {
+    const uint8_t *rp = S.mrow[ms][gw * 16 + rr];
+    v[rr] = rp ? __ldg(reinterpret_cast<const uint4 *>(rp + lane * 16)) : make_uint4(0, 0, 0, 0);
+  }
+}
+
+__device__ __forceinline__ void gather_store_fp8(MqaSmem &S, uint8_t *kt, int ms, int ec, int gw, int lane, const uint4 (&v)[16]) {
+  const int atom = lane >> 2, c0 = (lane & 3) * 2;
+#pragma unroll
+  for (int rr = 0; rr < 16; ++rr) {
+    const int row = gw * 16 + rr;
+    const __half2 sc2 = __float2half2_rn(ldexpf(S.mscale[ms][row], -ec));
+    const uint32_t w[4] = {v[rr].x, v[rr].y, v[rr].z, v[rr].w};
+    uint32_t o[8];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      __half2_raw a = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[u] & 0xFFFF), __NV_E4M3);
+      __half2_raw cc = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(w[u] >> 16), __NV_E4M3);
+      __half2 ha = __hmul2(*reinterpret_cast<__half2 *>(&a), sc2);
+      __half2 hc = __hmul2(*reinterpret_cast<__half2 *>(&cc), sc2);
+      o[2 * u] = *reinterpret_cast<uint32_t *>(&ha);
+      o[2 * u + 1] = *reinterpret_cast<uint32_t *>(&hc);
+    }
+    uint8_t *base = kt + atom * kAtom;
+    *reinterpret_cast<uint4 *>(base + sw128_offset(row, c0)) = make_uint4(o[0], o[1], o[2], o[3]);
+    *reinterpret_cast<uint4 *>(base + sw128_offset(row, c0 + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+  }
+}
+
+__device__ void gather_role(const MqaLaunch &p, MqaSmem &S, const long long *prefix, long long c0, long long c1) {
+  const int lane = threadIdx.x & 31, gw = (threadIdx.x >> 5) - kGatherWarp0;
+  const bool fp8 = p.kv_dt == DSV4_FP8E4M3;
+  int seg = -1;
+  for (long long g = c0; g < c1; ++g) {
+    const long long n = g - c0;
+    const int s = static_cast<int>(n & 1), ms = static_cast<int>(n % kMetaSlots);
+    const ChunkPos cp = chunk_pos(prefix, p.B, g, c0, c1);
+    bool ok = mbar_wait(&S.meta_full[ms], static_cast<uint32_t>((n / kMetaSlots) & 1), &S.abort_flag);
+    if (ok && cp.first) {
+      ++seg;
+      if (seg >= 1) ok = mbar_wait(&S.q_empty, static_cast<uint32_t>((seg - 1) & 1), &S.abort_flag);
+      if (ok) query_issue(p, S, cp.b, gw, lane);
+    }
+    if (ok && n >= 2) ok = mbar_wait(&S.k_empty[s], static_cast<uint32_t>((n / 2 - 1) & 1), &S.abort_flag);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) S.abort_flag = 1;
+      break;
+    }
+    // the query copy (if any) and the key rows are in flight together; the tile is finished
+    // first, then the query
+    uint8_t *kt = &S.k[s][0][0];
+    // chunk exponent (every warp derives the same one) and the scales softmax reads
+    const float smax = warp_max(fmaxf(S.mscale[ms][lane], S.mscale[ms][lane + 32]));
+    int ec = 0;
+    if (fp8) frexpf(smax, &ec);  // largest scale = f * 2^ec, f in [0.5, 1)
+    if (lane < 16) S.rscale[s][gw * 16 + lane] = S.mscale[ms][gw * 16 + lane];
+    if (gw == 0 && lane == 0) S.ec[s] = ec;
+    if (fp8) {
+      uint4 v[16];
+      gather_load_fp8(S, ms, gw, lane, v);
+      gather_store_fp8(S, kt, ms, ec, gw, lane, v);
+    } else {
+      gather_issue_bf16(S, kt, ms, gw, lane);
+      cp_async_wait_all();
+    }
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&S.k_full[s]);
+      mbar_arrive(&S.meta_empty[ms]);
+    }
+    if (cp.first) {
+      query_finish(p, S, key_list(p, cp.b, false).pos, seg & 1, gw, lane);
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.q_full);
+    }
+  }
+  cp_async_wait_all();
+}
+
+// ---- warp 8, one thread: MMA1 S = Q K^T into TMEM lanes 16..31, MMA2 O += P K into lanes
+// 0..15 (all 512 columns; the same swizzled key tile read MN-major serves as V = K).
+__device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const long long *prefix, long long c0, long long c1,
+                         uint32_t tmem) {
+  const bool f16 = fp16_operands(p);
+  const uint32_t idesc1 = f16 ? idesc_f16(kH, kCh, 0, 0) : idesc_bf16(kH, kCh, 0, 0);
+  const uint32_t idesc2 = f16 ? idesc_f16(kH, 256, 0, 1) : idesc_bf16(kH, 256, 0, 1);
+  const uint32_t s_tmem = tmem + (16u << 16);
+  int seg = -1;
+  long long n = 0;
+  for (long long g = c0; g < c1; ++g, ++n) {
+    const int s = static_cast<int>(n & 1);
+    const ChunkPos cp = chunk_pos(prefix, p.B, g, c0, c1);
+    if (cp.first) {
+      ++seg;
+      if (!mbar_wait(&S.q_full, static_cast<uint32_t>(seg & 1), &S.abort_flag)) break;
+    }
+    if (!mbar_wait(&S.k_full[s], static_cast<uint32_t>((n / 2) & 1), &S.abort_flag)) break;
+    if (n >= 1 && !mbar_wait(&S.s_empty, static_cast<uint32_t>((n - 1) & 1), &S.abort_flag)) break;
+    tc_fence_after();
+    const uint32_t qa = smem_u32(&S.q[0][0]), ka = smem_u32(&S.k[s][0][0]);
+#pragma unroll 4
+    for (int kk = 0; kk < kD / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * (kH * 128) + (kk & 3) * 32;
+      const uint32_t offk = (kk >> 2) * kAtom + (kk & 3) * 32;
+      mma_bf16(s_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + offk, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
+    }
+    mma_commit(&S.s_full);
+    if (cp.last) mma_commit(&S.q_empty);
+    if (!mbar_wait(&S.p_full, static_cast<uint32_t>(n & 1), &S.abort_flag)) break;
+    if (cp.first && seg >= 1 && !mbar_wait(&S.o_empty, static_cast<uint32_t>((seg - 1) & 1), &S.abort_flag)) break;
+    tc_fence_after();
+    const uint32_t pa = smem_u32(S.p);
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh)
+#pragma unroll
+      for (int ks = 0; ks < kCh / 16; ++ks)
+        mma_bf16(tmem + nh * 256, sw128_desc(pa + ks * 32, 16, 1024),
+                 sw128_desc(ka + nh * 4 * kAtom + ks * 2048, kAtom, 1024), idesc2,
+                 (!cp.first || ks > 0) ? 1u : 0u);
+    mma_commit(&S.k_empty[s]);
+    mma_commit(&S.o_full);
+  }
+  // let the last MMAs finish before the CTA frees its TMEM
+  if (n > 0) {
+    volatile int dummy = 0;
+    mbar_wait(&S.o_full, static_cast<uint32_t>((n - 1) & 1), &dummy);
+  }
+}
+
+// ---- warps 0-3 (quad = warp): online softmax and the partial output. Head h = 16 quad +
+// (lane & 15): its S row is TMEM lane 32 quad + 16 + (lane & 15); lanes 16..31 take keys
+// 0..31 of it, lanes 0..15 keys 32..63 (by shuffle), and both keep the head's running state.
+// Lanes 0..15 also own the head's O row (TMEM lane 32 quad + lane) for rescaling and output.
+// Online softmax in log2 units: with z_j = x_j + ec (x_j the logit of key j), the
+// accumulators hold O = sum_j 2^(z_j - R) * Krow_j and l = sum_j 2^(z_j - R) * 2^-ec, both
+// from the same rounded P, in units of 2^R; R is raised lazily (only when a chunk's max z
+// exceeds it by more than 8), so P stays <= 2^8 and O is rescaled rarely.
+__device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const long long *prefix, long long c0, long long c1,
+                             uint32_t tmem) {
+  const MqaLaunch &p = P.a;
+  const int lane = threadIdx.x & 31, quad = (threadIdx.x >> 5) - kSoftWarp0;
+  const int head = quad * 16 + (lane & 15);
+  const bool hi = lane >= 16;            // keys 0..31 (S row owner) vs keys 32..63
+  const int key0 = hi ? 0 : 32;
+  const bool f16 = fp16_operands(p);
+  const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
+  float R = -INFINITY, l_half = 0.f;
+  int seg = -1;
+  long long n = 0;
+  for (long long g = c0; g < c1; ++g, ++n) {
+    const int s = static_cast<int>(n & 1);
+    const ChunkPos cp = chunk_pos(prefix, p.B, g, c0, c1);
+    if (cp.first) {
+      ++seg;
+      R = -INFINITY;
+      l_half = 0.f;
+    }
+    bool ok = mbar_wait(&S.k_full[s], static_cast<uint32_t>((n / 2) & 1), &S.abort_flag);
+    ok = ok && mbar_wait(&S.s_full, static_cast<uint32_t>(n & 1), &S.abort_flag);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) S.abort_flag = 1;
+      break;
+    }
+    // read the query scale before releasing S: once S is free the query of a later segment
+    // (same parity) may be written
+    const int ec = S.ec[s];
+    // logit in log2 units of key j: acc * tau*log2(e) * qinv[h] * (fp8: 2^ec; bf16: 1)
+    const float coef = P.scale_log2 * S.qinv[seg & 1][head] * ldexpf(1.0f, ec);
+    const float fec = static_cast<float>(ec);
+    tc_fence_after();
+    uint32_t r0[32], r1[32];
+    tmem_ld32(lane_base + 0, r0);
+    tmem_ld32(lane_base + 32, r1);
+    tmem_ld_wait();
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.s_empty);
+    const float *rs = S.rscale[s] + key0;
+    float z[32];
+    float mz = -INFINITY;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const uint32_t other = __shfl_sync(0xFFFFFFFFu, r1[j], (lane & 15) | 16);
+      const float x = __uint_as_float(hi ? r0[j] : other);
+      z[j] = rs[j] != 0.f ? fmaf(x, coef, fec) : -INFINITY;
+      mz = fmaxf(mz, z[j]);
+    }
+    mz = fmaxf(mz, __shfl_xor_sync(0xFFFFFFFFu, mz, 16));
+    float Rn = R;
+    if (mz > R + 8.f) Rn = mz;
+    const float alpha = (Rn == R) ? 1.f : exp2f(R - Rn);  // R = -inf -> 0
+    const bool need_rescale = (Rn != R) && !cp.first;
+    const float lsc = ldexpf(1.0f, -ec);
+    float lsum = 0.f;
+    uint32_t pk[16];
+#pragma unroll
+    for (int j = 0; j < 32; j += 2) {
+      const float e0 = z[j] == -INFINITY ? 0.f : exp2f(z[j] - Rn);
+      const float e1 = z[j + 1] == -INFINITY ? 0.f : exp2f(z[j + 1] - Rn);
+      float a0, a1;
+      if (f16) {
+        __half2 h2 = __floats2half2_rn(e0, e1);
+        pk[j / 2] = *reinterpret_cast<uint32_t *>(&h2);
+        const float2 back = __half22float2(h2);
+        a0 = back.x;
+        a1 = back.y;
+      } else {
+        pk[j / 2] = pack_bf16x2(e0, e1);
+        a0 = __uint_as_float(pk[j / 2] << 16);
+        a1 = __uint_as_float(pk[j / 2] & 0xFFFF0000u);
+      }
+      lsum += a0 + a1;  // the denominator uses the rounded P, like the numerator
+    }
+    l_half = l_half * alpha + lsum * lsc;
+    R = Rn;
+    // P and O are free once MMA2 of the previous chunk completed
+    ok = n == 0 || mbar_wait(&S.o_full, static_cast<uint32_t>((n - 1) & 1), &S.abort_flag);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) S.abort_flag = 1;
+      break;
+    }
+    tc_fence_after();
+    if (__any_sync(0xFFFFFFFFu, need_rescale)) {
+#pragma unroll 1
+      for (int col = 0; col < kD; col += 32) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + col, o);
+        tmem_ld_wait();
+        if (!hi) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        }
+        tmem_st32(lane_base + col, o);
+      }
+      tmem_st_wait();
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+      *reinterpret_cast<uint4 *>(S.p + sw128_offset(head, (key0 >> 3) + c)) =
+          make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+    tc_fence_before();
+    fence_proxy_async_smem();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&S.p_full);
+    if (cp.last) {
+      const float l = l_half + __shfl_xor_sync(0xFFFFFFFFu, l_half, 16);
+      ok = mbar_wait(&S.o_full, static_cast<uint32_t>(n & 1), &S.abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        if (lane == 0) S.abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const size_t slot = static_cast<size_t>(cp.b) + blockIdx.x;
+      if (hi) {
+        float *ml = P.part_ml + (slot * kH + head) * 2;
+        ml[0] = R;
+        ml[1] = l;
+      }
+      float *po = P.part_o + (slot * kH + head) * kD;
+#pragma unroll 1
+      for (int col = 0; col < kD; col += 32) {
+        uint32_t o[32];
+        tmem_ld32(lane_base + col, o);
+        tmem_ld_wait();
+        if (!hi) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 4)
+            __stcg(reinterpret_cast<float4 *>(po + col + i),
+                   make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]), __uint_as_float(o[i + 2]),
+                               __uint_as_float(o[i + 3])));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.o_empty);
+    }
+  }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaTcParams P) {
@@ -362,15 +678,28 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
   MqaSmem &S = *reinterpret_cast<MqaSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const MqaLaunch &p = P.a;
   long long *prefix = reinterpret_cast<long long *>(&S + 1);  // [B + 1] chunks before sequence b
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, warp = tid >> 5;
 
   if (tid == 0) {
-    mbar_init(&S.bar_s, 1);
-    mbar_init(&S.bar_o, 1);
+    for (int i = 0; i < kMetaSlots; ++i) {
+      mbar_init(&S.meta_full[i], 1);
+      mbar_init(&S.meta_empty[i], 4);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.k_full[i], 4);
+      mbar_init(&S.k_empty[i], 1);
+    }
+    mbar_init(&S.q_full, 4);
+    mbar_init(&S.q_empty, 1);
+    mbar_init(&S.s_full, 1);
+    mbar_init(&S.s_empty, 4);
+    mbar_init(&S.p_full, 4);
+    mbar_init(&S.o_full, 1);
+    mbar_init(&S.o_empty, 4);
     S.abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tmem_alloc(&S.tmem_base, 512);
     tmem_relinquish();
   }
@@ -382,261 +711,126 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
   const long long T = prefix[p.B], G = gridDim.x;
   const long long c0 = (T * blockIdx.x) / G, c1 = (T * (blockIdx.x + 1)) / G;
 
-  const bool f16 = fp16_operands(p);
-  const bool smax_thread = warp < 4 && lane >= 16;  // owns S/O row (head) 16*warp + lane - 16
-  const int quad = warp & 3;
-  const int head = quad * 16 + (lane & 15);
-  // Online softmax in log2 units. With z_j = x_j + ec (x_j the logit of key j), the
-  // accumulators hold O = sum_j 2^(z_j - R) * Krow_j and l = sum_j 2^(z_j - R) * 2^-ec, both
-  // from the same rounded P, in units of 2^R; R is raised lazily (only when a chunk's max z
-  // exceeds it by more than 8), so P stays <= 2^8 and O is rescaled rarely.
-  float R = -INFINITY, l_run = 0.f;
-  int cur_b = -1;
-  bool first_in_seg = true;
-  KeyList L{};
-  const uint32_t idesc1 = f16 ? idesc_f16(kH, kCh, 0, 0) : idesc_bf16(kH, kCh, 0, 0);
-  const uint32_t idesc2 = f16 ? idesc_f16(kH, 256, 0, 1) : idesc_bf16(kH, 256, 0, 1);
-  const uint32_t s_tmem = tmem + (16u << 16);  // S accumulator: lanes 16..31 of each quadrant
-
-  if (tid == 0) {
-    S.meta_first = 0;
-    S.meta_n = 0;
-  }
-  __syncthreads();
-  if (c0 < c1) gather_chunk(P, S, prefix, c0, c1, 0);
-  for (long long g = c0; g < c1; ++g) {
-    const long long it = g - c0;
-    const int kb = static_cast<int>(it & 1);
-    const int b = find_seq(prefix, p.B, g);
-    if (b != cur_b) {
-      cur_b = b;
-      first_in_seg = true;
-      R = -INFINITY;
-      l_run = 0.f;
-      L = key_list(p, b, false);
-      load_query(P, S, b, L.pos);
-    }
-    fence_proxy_async_smem();
-    __syncthreads();
-    const int ec = S.ec[kb];
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t qa = smem_u32(&S.q[0][0]), ka = smem_u32(&S.k[kb][0][0]);
-#pragma unroll
-      for (int kk = 0; kk < kD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * (kH * 128) + (kk & 3) * 32;
-        const uint32_t offk = (kk >> 2) * kAtom + (kk & 3) * 32;
-        mma_bf16(s_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + offk, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
-      }
-      mma_commit(&S.bar_s);
-    }
-    // prefetch the next chunk while MMA1 runs (its buffer was released by MMA2 of it-1)
-    if (g + 1 < c1) gather_chunk(P, S, prefix, g + 1, c1, kb ^ 1);
-    bool ok = mbar_wait(&S.bar_s, static_cast<uint32_t>(it & 1), &S.abort_flag);
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    tc_fence_after();
-    float alpha = 1.f;
-    bool need_rescale = false;
-    if (warp < 4 && ok) {
-      uint32_t r0[32], r1[32];
-      tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16), r0);
-      tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + 32, r1);
-      tmem_ld_wait();
-      if (smax_thread) {
-        const float *rs = S.rscale[kb];
-        // logit in log2 units of key j: acc * tau*log2(e) * qinv[h] * (fp8: 2^ec; bf16: 1)
-        const float coef = P.scale_log2 * S.qinv[head] * ldexpf(1.0f, ec);
-        const float fec = static_cast<float>(ec);
-        float z[kCh];
-        float mz = -INFINITY;
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          z[j] = rs[j] != 0.f ? fmaf(__uint_as_float(r0[j]), coef, fec) : -INFINITY;
-          z[j + 32] = rs[j + 32] != 0.f ? fmaf(__uint_as_float(r1[j]), coef, fec) : -INFINITY;
-          mz = fmaxf(mz, fmaxf(z[j], z[j + 32]));
-        }
-        float Rn = R;
-        if (mz > R + 8.f) Rn = mz;
-        alpha = (Rn == R) ? 1.f : exp2f(R - Rn);  // R = -inf -> 0
-        need_rescale = (Rn != R) && !first_in_seg;
-        const float lsc = ldexpf(1.0f, -ec);
-        float lsum = 0.f;
-        uint32_t pk[kCh / 2];
-#pragma unroll
-        for (int j = 0; j < kCh; j += 2) {
-          const float e0 = z[j] == -INFINITY ? 0.f : exp2f(z[j] - Rn);
-          const float e1 = z[j + 1] == -INFINITY ? 0.f : exp2f(z[j + 1] - Rn);
-          float r0f, r1f;
-          if (f16) {
-            __half2 h = __floats2half2_rn(e0, e1);
-            pk[j / 2] = *reinterpret_cast<uint32_t *>(&h);
-            const float2 back = __half22float2(h);
-            r0f = back.x;
-            r1f = back.y;
-          } else {
-            pk[j / 2] = pack_bf16x2(e0, e1);
-            r0f = __uint_as_float(pk[j / 2] << 16);
-            r1f = __uint_as_float(pk[j / 2] & 0xFFFF0000u);
-          }
-          lsum += r0f + r1f;  // the denominator uses the rounded P, like the numerator
-        }
-        l_run = l_run * alpha + lsum * lsc;
-        R = Rn;
-#pragma unroll
-        for (int c = 0; c < 8; ++c)
-          *reinterpret_cast<uint4 *>(S.p + sw128_offset(head, c)) =
-              make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      }
-      // O rows (lanes 0..15) take their head's rescale factor from lane + 16
-      const float alpha_o = __shfl_sync(0xFFFFFFFFu, alpha, (lane & 15) + 16);
-      const bool any = __any_sync(0xFFFFFFFFu, need_rescale);
-      if (any) {
-        for (int col = 0; col < kD; col += 32) {
-          uint32_t r[32];
-          const uint32_t addr = tmem + (static_cast<uint32_t>(quad * 32) << 16) + col;
-          tmem_ld32(addr, r);
-          tmem_ld_wait();
-          if (lane < 16) {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) r[i] = __float_as_uint(__uint_as_float(r[i]) * alpha_o);
-          }
-          tmem_st32(addr, r);
-        }
-        tmem_st_wait();
-      }
-    }
-    if (!ok && lane == 0) S.abort_flag = 1;
-    tc_fence_before();
-    fence_proxy_async_smem();
-    __syncthreads();
-    if (S.abort_flag) break;
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t pa = smem_u32(S.p), ka = smem_u32(&S.k[kb][0][0]);
-#pragma unroll
-      for (int nh = 0; nh < 2; ++nh)
-#pragma unroll
-        for (int ks = 0; ks < kCh / 16; ++ks)
-          mma_bf16(tmem + nh * 256, sw128_desc(pa + ks * 32, 16, 1024),
-                   sw128_desc(ka + nh * 4 * kAtom + ks * 2048, kAtom, 1024), idesc2,
-                   (!first_in_seg || ks > 0) ? 1u : 0u);
-      mma_commit(&S.bar_o);
-    }
-    ok = mbar_wait(&S.bar_o, static_cast<uint32_t>(it & 1), &S.abort_flag);
-    ok = __all_sync(0xFFFFFFFFu, ok);
-    tc_fence_after();
-    first_in_seg = false;
-    const bool seg_end = (g + 1 == c1) || (find_seq(prefix, p.B, g + 1) != b);
-    if (seg_end && ok) {
-      const size_t slot = static_cast<size_t>(b) + blockIdx.x;
-      if (smax_thread) {
-        float *ml = P.part_ml + (slot * kH + head) * 2;
-        ml[0] = R;
-        ml[1] = l_run;
-      }
-      // all 8 warps read O: warps 0-3 columns 0..255, warps 4-7 columns 256..511
-      const int colbase = (warp >> 2) * 256;
-      float *po = P.part_o + (slot * kH + head) * kD;
-      for (int col = colbase; col < colbase + 256; col += 32) {
-        uint32_t r[32];
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + col, r);
-        tmem_ld_wait();
-        if (lane < 16) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            *reinterpret_cast<float4 *>(po + col + i) = make_float4(
-                __uint_as_float(r[i]), __uint_as_float(r[i + 1]), __uint_as_float(r[i + 2]), __uint_as_float(r[i + 3]));
-        }
-      }
-      tc_fence_before();
-    }
-    if (!ok && lane == 0) S.abort_flag = 1;
-    __syncthreads();
-    if (S.abort_flag) break;
-  }
+  if (warp == kMetaWarp) meta_role(p, S, prefix, c0, c1);
+  else if (warp >= kGatherWarp0 && warp < kGatherWarp0 + 4) gather_role(p, S, prefix, c0, c1);
+  else if (warp == kMmaWarp) {
+    if ((tid & 31) == 0) mma_role(p, S, prefix, c0, c1, tmem);
+  } else softmax_role(P, S, prefix, c0, c1, tmem);
 
   if (tid == 0 && S.abort_flag) report(p.d_status, DSV4_DEV_TIMEOUT);
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
 }
 
-// Merge the partials of every sequence, inverse RoPE, store. grid (B, H / 8), 256 threads.
+// Merge the partials of every sequence, inverse RoPE, store. grid (B, H / 8), 256 threads:
+// warp w owns head h0 + w for the weights; for the sum every thread owns 4 float4 columns
+// of the CTA's 8 heads and keeps their loads of several partials in flight together.
 __global__ void __launch_bounds__(256) mqa_merge_kernel(const MqaTcParams P, int grid_ctas) {
   const MqaLaunch &p = P.a;
-  __shared__ int np_s;  // partials of this sequence
+  __shared__ int warp_cnt[8];
   __shared__ float cs[kD / 2], sn[kD / 2];
+  __shared__ float inv_l[8], lse_s[8];
   extern __shared__ __align__(16) uint8_t dyn[];
-  float *wgt = reinterpret_cast<float *>(dyn);  // [grid_ctas][8]: weight of each partial, per head
-  int *cta = reinterpret_cast<int *>(wgt + static_cast<size_t>(grid_ctas) * 8);  // [grid_ctas]
+  float *wgt = reinterpret_cast<float *>(dyn);                                  // [grid][8] weight
+  float *lv = wgt + static_cast<size_t>(grid_ctas) * 8;                         // [grid][8] partial sum
+  int *cta = reinterpret_cast<int *>(lv + static_cast<size_t>(grid_ctas) * 8);  // [grid]
   long long *prefix = reinterpret_cast<long long *>(cta + ((grid_ctas + 1) & ~1));  // [B + 1]
   long long *red = prefix + p.B + 1;                                             // [blockDim]
-  __shared__ float inv_l[8], lse_s[8];
-  const int b = blockIdx.x, h0 = blockIdx.y * 8, tid = threadIdx.x;
-  chunk_prefix(p, prefix, red, false);
-  if (tid == 0) {
-    // the CTAs of the main kernel whose (non-empty) chunk range meets this sequence; with
-    // fewer chunks than CTAs some ranges are empty and those CTAs wrote no partial
-    const long long acc = prefix[p.B], mine = prefix[b], cnt = prefix[b + 1] - prefix[b];
-    int n = 0;
-    for (int c = 0; c < grid_ctas && cnt > 0; ++c) {
-      const long long a0 = (acc * c) / grid_ctas, a1 = (acc * (c + 1)) / grid_ctas;
-      if (a0 < mine + cnt && a1 > mine && a1 > a0) cta[n++] = c;
-    }
-    np_s = n;
-  }
+  const int b = blockIdx.x, h0 = blockIdx.y * 8, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const KeyList L = key_list(p, b, false);
   const int half = p.rope_dims / 2;
-  for (int i = tid; i < half; i += 256) rope_cos_sin(L.pos, i, p.rope_dims, p.rope_base, &cs[i], &sn[i]);
-  __syncthreads();
-  const int np = np_s;
-  if (tid < 8) {
-    const int h = h0 + tid;
-    float M = -INFINITY;
-    for (int i = 0; i < np; ++i) {
-      const size_t slot = static_cast<size_t>(b) + cta[i];
-      M = fmaxf(M, P.part_ml[(slot * kH + h) * 2]);
+  for (int i = tid; i < half; i += 256) rope_cos_sin(L.pos, i, p.rope_theta1, &cs[i], &sn[i]);
+  chunk_prefix(p, prefix, red, false);
+  // the CTAs of the main kernel whose (non-empty) chunk range meets this sequence, in
+  // order; with fewer chunks than CTAs some ranges are empty and those CTAs wrote nothing
+  const long long acc = prefix[p.B], mine = prefix[b], cnt = prefix[b + 1] - prefix[b];
+  int n = 0;
+  for (int c0 = 0; c0 < grid_ctas; c0 += 256) {
+    const int c = c0 + tid;
+    bool hit = false;
+    if (c < grid_ctas && cnt > 0) {
+      const long long a0 = (acc * c) / grid_ctas, a1 = (acc * (c + 1)) / grid_ctas;
+      hit = a0 < mine + cnt && a1 > mine && a1 > a0;
     }
-    float Ls = 0.f;
-    for (int i = 0; i < np; ++i) {
-      const size_t slot = static_cast<size_t>(b) + cta[i];
-      const float mi = P.part_ml[(slot * kH + h) * 2], li = P.part_ml[(slot * kH + h) * 2 + 1];
-      const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
-      wgt[i * 8 + tid] = w;
-      Ls += w * li;
-    }
-    inv_l[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
-    lse_s[tid] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+    const unsigned bal = __ballot_sync(0xFFFFFFFFu, hit);
+    if (lane == 0) warp_cnt[warp] = __popc(bal);
+    __syncthreads();
+    int off = n;
+    for (int w = 0; w < warp; ++w) off += warp_cnt[w];
+    if (hit) cta[off + __popc(bal & ((1u << lane) - 1u))] = c;
+    for (int w = 0; w < 8; ++w) n += warp_cnt[w];
+    __syncthreads();
+  }
+  const int np = n;
+  for (int j = tid; j < np * 8; j += 256) {
+    const size_t slot = static_cast<size_t>(b) + cta[j >> 3];
+    const float2 ml = *reinterpret_cast<const float2 *>(P.part_ml + (slot * kH + h0 + (j & 7)) * 2);
+    wgt[j] = ml.x;
+    lv[j] = ml.y;
   }
   __syncthreads();
-  const int rope0 = kD - p.rope_dims;
-  for (int t = tid; t < 8 * (kD / 2); t += 256) {
-    const int hh = t / (kD / 2), pr = t % (kD / 2), h = h0 + hh;
-    float o0 = 0.f, o1 = 0.f;
-    for (int i = 0; i < np; ++i) {
-      const size_t slot = static_cast<size_t>(b) + cta[i];
-      const float2 v = *reinterpret_cast<const float2 *>(P.part_o + (slot * kH + h) * kD + 2 * pr);
-      o0 = fmaf(wgt[i * 8 + hh], v.x, o0);
-      o1 = fmaf(wgt[i * 8 + hh], v.y, o1);
+  {  // weights of head h0 + warp: 2^(m_i - M), M the largest partial reference
+    float M = -INFINITY;
+    for (int i = lane; i < np; i += 32) M = fmaxf(M, wgt[i * 8 + warp]);
+    M = warp_max(M);
+    float Ls = 0.f;
+    for (int i = lane; i < np; i += 32) {
+      const float mi = wgt[i * 8 + warp];
+      const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
+      wgt[i * 8 + warp] = w;
+      Ls += w * lv[i * 8 + warp];
     }
-    o0 *= inv_l[hh];
-    o1 *= inv_l[hh];
-    const int d = 2 * pr;
-    if (d >= rope0) {  // rotate by -pos
-      const int pi = (d - rope0) >> 1;
-      const float c = cs[pi], s = sn[pi];
-      const float y0 = o0 * c + o1 * s, y1 = -o0 * s + o1 * c;
-      o0 = y0;
-      o1 = y1;
+    Ls = warp_sum(Ls);
+    if (lane == 0) {
+      inv_l[warp] = Ls > 0.f ? 1.f / Ls : 0.f;
+      lse_s[warp] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+    }
+  }
+  __syncthreads();
+  constexpr int kPer = 8 * kD / 4 / 256;  // float4 columns per thread (4)
+  float4 o[kPer];
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) o[q] = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int i = 0; i < np; ++i) {
+    const size_t slot = static_cast<size_t>(b) + cta[i];
+    const float *base = P.part_o + (slot * kH + h0) * kD;
+    float4 v[kPer];
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) v[q] = __ldcs(reinterpret_cast<const float4 *>(base) + q * 256 + tid);
+#pragma unroll
+    for (int q = 0; q < kPer; ++q) {
+      const float w = wgt[i * 8 + (q * 256 + tid) / (kD / 4)];
+      o[q].x = fmaf(w, v[q].x, o[q].x);
+      o[q].y = fmaf(w, v[q].y, o[q].y);
+      o[q].z = fmaf(w, v[q].z, o[q].z);
+      o[q].w = fmaf(w, v[q].w, o[q].w);
+    }
+  }
+  const int rope0 = kD - p.rope_dims;
+#pragma unroll
+  for (int q = 0; q < kPer; ++q) {
+    const int e = q * 256 + tid, hh = e / (kD / 4), d = (e % (kD / 4)) * 4, h = h0 + hh;
+    float y[4] = {o[q].x * inv_l[hh], o[q].y * inv_l[hh], o[q].z * inv_l[hh], o[q].w * inv_l[hh]};
+#pragma unroll
+    for (int u = 0; u < 4; u += 2) {
+      if (d + u >= rope0) {  // rotate by -pos
+        const int pi = (d + u - rope0) >> 1;
+        const float c = cs[pi], sv = sn[pi];
+        const float y0 = y[u] * c + y[u + 1] * sv, y1 = -y[u] * sv + y[u + 1] * c;
+        y[u] = y0;
+        y[u + 1] = y1;
+      }
     }
     const size_t off = (static_cast<size_t>(b) * kH + h) * kD + d;
     if (p.out_dt == DSV4_F32) {
-      *reinterpret_cast<float2 *>(static_cast<float *>(p.out) + off) = make_float2(o0, o1);
+      *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off) = make_float4(y[0], y[1], y[2], y[3]);
     } else {
-      *reinterpret_cast<uint32_t *>(static_cast<uint16_t *>(p.out) + off) = pack_bf16x2(o0, o1);
+      *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.out) + off) =
+          make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
     }
   }
   if (p.lse && tid < 8) p.lse[static_cast<size_t>(b) * kH + h0 + tid] = lse_s[tid];
@@ -663,7 +857,7 @@ __global__ void __launch_bounds__(256) mqa_simt_kernel(const MqaLaunch p, float 
   __syncthreads();
   for (int i = tid; i < half; i += 256) {
     float c, s;
-    rope_cos_sin(L.pos, i, p.rope_dims, p.rope_base, &c, &s);
+    rope_cos_sin(L.pos, i, p.rope_theta1, &c, &s);
     const float x0 = qr[rope0 + 2 * i], x1 = qr[rope0 + 2 * i + 1];
     qr[rope0 + 2 * i] = x0 * c - x1 * s;
     qr[rope0 + 2 * i + 1] = x0 * s + x1 * c;
@@ -731,7 +925,7 @@ __global__ void __launch_bounds__(256) mqa_simt_kernel(const MqaLaunch p, float 
   __syncthreads();
   for (int i = tid; i < half; i += 256) {
     float c, s;
-    rope_cos_sin(L.pos, i, p.rope_dims, p.rope_base, &c, &s);
+    rope_cos_sin(L.pos, i, p.rope_theta1, &c, &s);
     const float x0 = ob[rope0 + 2 * i], x1 = ob[rope0 + 2 * i + 1];
     ob[rope0 + 2 * i] = x0 * c + x1 * s;
     ob[rope0 + 2 * i + 1] = -x0 * s + x1 * c;
@@ -756,8 +950,8 @@ float softmax_scale_log2(const MqaLaunch &p) {
 }  // namespace
 
 bool mqa_uses_tensor_cores(const MqaLaunch &p) {
-  return (p.kv_dt == DSV4_BF16 || p.kv_dt == DSV4_FP8E4M3) && p.D == kD && p.H == kH &&
-         (p.q_dt == DSV4_BF16 || p.q_dt == DSV4_F32) && p.rope_dims % 8 == 0 && p.B <= 1024;
+  return (p.kv_dt == DSV4_BF16 || p.kv_dt == DSV4_FP8E4M3) && p.D == kD && p.H == kH && p.q_dt == DSV4_BF16 &&
+         p.rope_dims % 8 == 0 && p.B <= 1024;
 }
 
 size_t mqa_workspace_bytes(const MqaLaunch &p) {
@@ -766,7 +960,9 @@ size_t mqa_workspace_bytes(const MqaLaunch &p) {
   return align_up(slots * kH * kD * sizeof(float), 256) + align_up(slots * kH * 2 * sizeof(float), 256);
 }
 
-cudaError_t launch_mqa(const MqaLaunch &p, void *ws, cudaStream_t st) {
+cudaError_t launch_mqa(const MqaLaunch &p0, void *ws, cudaStream_t st) {
+  MqaLaunch p = p0;
+  p.rope_theta1 = rope_theta1(p.rope_base, p.rope_dims);
   if (mqa_uses_tensor_cores(p)) {
     MqaTcParams P;
     P.a = p;
@@ -780,7 +976,7 @@ cudaError_t launch_mqa(const MqaLaunch &p, void *ws, cudaStream_t st) {
     mqa_tc_kernel<<<tc_grid(), kThreads, smem, st>>>(P);
     e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    const size_t msmem = static_cast<size_t>(tc_grid()) * 8 * sizeof(float) +
+    const size_t msmem = static_cast<size_t>(tc_grid()) * 16 * sizeof(float) +
                          static_cast<size_t>((tc_grid() + 1) & ~1) * sizeof(int) +
                          (static_cast<size_t>(p.B) + 1 + 256) * sizeof(long long);
     e = cudaFuncSetAttribute(mqa_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);

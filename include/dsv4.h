@@ -193,9 +193,9 @@ dsv4_status dsv4_swa_insert(const dsv4_swa_insert_args *args, dsv4_stream stream
  *   keys: paged cache with keys.dim == dim, dtype F32 or FP8E4M3;
  *   n_entries [batch] device int32 (<= keys.max_blocks * 256/keys.m);
  *   pos [batch] device int32 (used only when q_rope_dims > 0).
- * fp8 queries and keys with dim 128, heads 32 or 64, m == 4, k <= 512, no query RoPE and
- * batch <= 512 run on the tensor cores (tcgen05, fed by TMA); other shapes run on a
- * CUDA-core kernel. Both give the same entries.
+ * fp8 queries and keys with dim 128, heads 32 or 64, m == 4, no query RoPE and batch <= 512
+ * run on the tensor cores (tcgen05, fed by TMA); other shapes run on a CUDA-core kernel.
+ * Both give the same entries.
  */
 typedef struct {
   int32_t batch;
@@ -238,8 +238,8 @@ dsv4_status dsv4_indexer_topk(const dsv4_indexer_args *args, void *workspace,
  * make that first call before any stream capture begins.
  * Limit: if dsv4_indexer_workspace_size(args) > DSV4_NOALLOC_SCRATCH_BYTES the call returns
  * DSV4_ERR_SCRATCH_LIMIT and launches nothing (use dsv4_indexer_topk with a caller
- * workspace instead). With fp8 keys of 128 dims, k = 512 and 32768 visible entries per
- * sequence that admits about 13 sequences.
+ * workspace instead). The tensor-core path needs about 4 bytes per cache entry of every
+ * sequence: 16 MiB admits about 127 sequences of 32768 entries (a 131072-token context).
  * Zero state: nothing has to start at zero; the per-sequence candidate counts at the head
  * of the scratch are zeroed by the call itself, on `stream`, before its kernels run.
  * Concurrency: the scratch is shared by every call on a device. Calls ordered on one

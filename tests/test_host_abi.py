@@ -115,7 +115,7 @@ def test_validation_rejects_bad_calls(lib):
         assert lib.dsv4_indexer_topk(C.byref(a), C.c_void_p(FAKE), 1 << 30, None) == code, bad
     a = _indexer()
     need = lib.dsv4_indexer_workspace_size(C.byref(a))
-    assert need >= 2 * 8 * 512
+    assert need >= 2 * 512 * 4  # at least one float score per cache entry of each sequence
     assert lib.dsv4_indexer_topk(C.byref(a), C.c_void_p(FAKE), need - 1, None) == A.ERR_INVALID_ARG
 
 
@@ -171,7 +171,9 @@ def test_hybrid_validation_and_workspace(lib):
     S.kv_dtype, S.q_dtype, S.out_dtype = A.BF16, A.BF16, A.BF16
     S.idx_kv, S.idx_gate, S.q_idx, S.w = FAKE, FAKE, FAKE, FAKE
     S.q_idx_dtype, S.w_dtype = A.FP8, A.BF16
-    assert lib.dsv4_hybrid_decode(C.byref(L), C.byref(S), C.c_void_p(FAKE), ws - 1, None) == A.ERR_INVALID_ARG
+    # the layer-level size is the largest need over the step's dtype choices; a workspace
+    # below one score per cache entry of every sequence is too small for any of them
+    assert lib.dsv4_hybrid_decode(C.byref(L), C.byref(S), C.c_void_p(FAKE), 32 * 512 * 4 - 1, None) == A.ERR_INVALID_ARG
     S2 = A.Step.from_buffer_copy(S)
     S2.batch = 31  # disagrees with nothing yet, but a missing q must be caught
     S2.q = None

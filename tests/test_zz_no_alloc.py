@@ -31,7 +31,7 @@ def _args(batch, max_blocks, k=512):
 
 def test_noalloc_refuses_requests_beyond_the_scratch():
     lib = dsv4.load()
-    big = _args(batch=64, max_blocks=512)  # 131072 positions: 32768 entries per sequence
+    big = _args(batch=160, max_blocks=512)  # 131072 positions: 32768 entries per sequence
     assert lib.dsv4_indexer_workspace_size(C.byref(big)) > A.NOALLOC_SCRATCH_BYTES
     assert lib.dsv4_indexer_topk_noalloc(C.byref(big), None) == A.ERR_SCRATCH_LIMIT
     assert b"static scratch" in lib.dsv4_status_string(A.ERR_SCRATCH_LIMIT)
