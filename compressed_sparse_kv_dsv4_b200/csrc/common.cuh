@@ -97,6 +97,16 @@ __device__ __forceinline__ void rope_cos_sin(int64_t pos, int pair, double theta
 }
 
 // --------------------------------------------------------------------------------------
+// programmatic dependent launch: a kernel launched with programmatic stream serialization
+// may start while its predecessor on the stream still runs. pdl_wait() returns once every
+// prerequisite grid has completed and its memory is visible; before it a kernel may only
+// touch data no predecessor writes or reads. Each kernel calls pdl_launch_dependents()
+// after its own pdl_wait(), so a kernel's early part only ever overlaps its immediate
+// predecessor. Launched without the attribute, both are no-ops.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// --------------------------------------------------------------------------------------
 // reductions
 
 __device__ __forceinline__ float warp_sum(float v) {
@@ -215,14 +225,14 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t by
                : "memory");
 }
 
-// One probe of the phase. The thread is suspended (not spinning) until the phase completes
-// or the hint (ns) runs out, so waiting warps leave the issue slots to the working ones.
+// One probe of the phase (the hardware may hold the thread for a short, implementation-
+// defined time before answering false).
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
-      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(1000000u)
+      : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
 }
@@ -270,6 +280,15 @@ __device__ __forceinline__ void tma_load_2d(void *dst, const CUtensorMap *map, u
           smem_u32(dst)),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
       : "memory");
+}
+
+// 1-D bulk copy global -> shared of `bytes` (a multiple of 16; both addresses 16-byte
+// aligned), completing as transaction bytes on bar
+__device__ __forceinline__ void bulk_load(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
 __device__ __forceinline__ void prefetch_tensormap(const CUtensorMap *map) {

@@ -196,6 +196,8 @@ __device__ __forceinline__ int64_t compress_items(const SeqRange &r, int m) {
 }
 
 __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressLaunch p) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) float smem[];
   float *scratch = smem;             // 3 * kMaxD
   float *e = smem + 3 * kMaxD;       // kMaxD
@@ -252,6 +254,8 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressLaunch
 }
 
 __global__ void __launch_bounds__(kThreads) swa_insert_kernel(const SwaLaunch p) {
+  pdl_wait();
+  pdl_launch_dependents();
   __shared__ float e[kMaxD];
   __shared__ float red[32];
   const int s = blockIdx.y;
@@ -272,6 +276,8 @@ __global__ void __launch_bounds__(kThreads) swa_insert_kernel(const SwaLaunch p)
 // One decode step's updates. blockIdx.y: 0 = window insert, 1 = main compressor append,
 // 2 = indexer-key compressor append.
 __global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const PrologueLaunch p) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ __align__(16) float smem[];
   float *scratch = smem;
   float *e = smem + 3 * kMaxD;
@@ -328,16 +334,14 @@ cudaError_t launch_compress(const CompressLaunch &p0, cudaStream_t st) {
   const long long upper = static_cast<long long>(p.total_tokens) / p.m + p.B;
   const long long cap = static_cast<long long>(sm_count()) * 8;
   const int grid = static_cast<int>(upper < cap ? (upper > 0 ? upper : 1) : cap);
-  compress_kernel<<<grid, kThreads, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(compress_kernel, dim3(grid), dim3(kThreads), smem, st, 1, p);
 }
 
 cudaError_t launch_swa_insert(const SwaLaunch &p0, cudaStream_t st) {
   SwaLaunch p = p0;
   p.rope_theta1 = rope_theta1(p.rope_base, p.rope_dims);
   dim3 grid(p.W, p.B);
-  swa_insert_kernel<<<grid, kThreads, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(swa_insert_kernel, grid, dim3(kThreads), 0, st, 1, p);
 }
 
 cudaError_t launch_decode_prologue(const PrologueLaunch &p0, cudaStream_t st) {
@@ -348,8 +352,7 @@ cudaError_t launch_decode_prologue(const PrologueLaunch &p0, cudaStream_t st) {
       cudaFuncSetAttribute(decode_prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPoolSmem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.B, p.idx_D > 0 ? 3 : 2);
-  decode_prologue_kernel<<<grid, kThreads, kPoolSmem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(decode_prologue_kernel, grid, dim3(kThreads), kPoolSmem, st, 1, p);
 }
 
 }  // namespace dsv4

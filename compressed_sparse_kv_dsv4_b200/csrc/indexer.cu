@@ -68,6 +68,8 @@ __device__ __forceinline__ int64_t visible_entries(const int32_t *n_entries, con
 
 __global__ void __launch_bounds__(256) indexer_simt_kernel(const IndexerLaunch p, unsigned long long *cand,
                                                            int64_t stride, int *cand_count) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ float sq[];  // [H][Dq] query, then [H] coefficients
   const int b = blockIdx.y;
   const int per_page = DSV4_PAGE_POSITIONS / p.m;
@@ -201,8 +203,8 @@ struct StageIter {
   }
 };
 
-// Page ids of the next kBatchStages stages, one per lane (lane = 4 * stage + page): the
-// block-table loads of a whole batch are in flight together, a batch ahead of their use.
+// Block-table entries of the next kBatchStages stages, one per lane (lane = 4 * stage +
+// page): the loads of a whole batch are in flight together, a batch ahead of their use.
 __device__ __forceinline__ int load_page_batch(const TcParams &p, const long long *prefix, const int64_t *nvis,
                                                StageIter &ahead, int lane) {
   int sb_l = -1;
@@ -218,13 +220,10 @@ __device__ __forceinline__ int load_page_batch(const TcParams &p, const long lon
       first_l = lt0 * kTile + static_cast<int64_t>(lane & 3) * kPerPage;
     }
   }
-  int pid = -1;
-  if (sb_l >= 0 && first_l < nvis[sb_l]) {
-    const int pg = p.block_table[static_cast<size_t>(sb_l) * p.max_blocks + first_l / kPerPage];
-    if (pg >= 0 && pg < p.num_pages) pid = pg;
-    else report(p.d_status, DSV4_DEV_BAD_PAGE);
-  }
-  return pid;
+  // the raw table entry; no page (-1) when the slot has no tile or starts past the visible
+  // entries. It is validated where it is used, so the load is not waited for here.
+  return sb_l >= 0 && first_l < nvis[sb_l] ? p.block_table[static_cast<size_t>(sb_l) * p.max_blocks + first_l / kPerPage]
+                                           : -1;
 }
 
 template <int H>
@@ -239,7 +238,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   // ---- setup: barriers, TMEM, tile prefix over sequences
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], 1); }
-    for (int i = 0; i < kSlots; ++i) { mbar_init(&S.sfull[i], 32); mbar_init(&S.sempty[i], kGroupThreads / 32); }
+    for (int i = 0; i < kSlots; ++i) { mbar_init(&S.sfull[i], 1); mbar_init(&S.sempty[i], kGroupThreads / 32); }
     for (int i = 0; i < kGroups; ++i) { mbar_init(&S.tfull[i], 1); mbar_init(&S.tempty[i], kGroupThreads / 32); }
     for (int i = 0; i < 2; ++i) { mbar_init(&S.qfull[i], 1); mbar_init(&S.qempty[i], 1); }
     S.abort_flag = 0;
@@ -270,6 +269,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
     }
     if (lane == 0) prefix[p.B] = carry;
   }
+  pdl_wait();  // keys, scales and the score buffer may be in use by the kernel before
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -281,8 +282,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   if (warp == 0) {
     // ---------------- producer. Lane 0 issues the key TMA of stage k (one box per 64-row
     // page; an invalid page, or one past the visible entries, takes a zero-filled
-    // out-of-range box). All 32 lanes copy the stage's key scales with cp.async, each
-    // arriving on the slot's barrier when its copies land.
+    // out-of-range box) and one bulk copy of the key scales per page, both completing as
+    // transaction bytes on their barriers.
     const int oob_row = p.num_pages * kPerPage;
     StageIter it, ahead;
     it.init(prefix, p.B, t0, t1);
@@ -301,35 +302,42 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
         batch_next = load_page_batch(p, prefix, nvis, ahead, lane);
       }
       const int slot = static_cast<int>(k % kSlots);
-      int ok = 1;
-      if (lane == 0 && k >= kSlots &&
-          !mbar_wait(&S.sempty[slot], static_cast<uint32_t>((k / kSlots - 1) & 1), &S.abort_flag))
-        ok = 0;
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
-      if (!ok) break;
-      {  // scales of stage k: lane l copies 2 x 16 bytes of page l / 8
-        const int pg_slot = lane >> 3;
-        const int my_pid = __shfl_sync(0xFFFFFFFFu, batch_cur, bs * kStagePages + pg_slot);
-        float *dst = &S.sig[slot][pg_slot * kPerPage + (lane & 7) * 8];
-        if (my_pid >= 0) {
-          const float *src = p.k_scales + static_cast<size_t>(my_pid) * kPerPage + (lane & 7) * 8;
-          cp_async16(dst, src);
-          cp_async16(dst + 4, src + 4);
-          cp_async_arrive(&S.sfull[slot]);
-        } else {
-          reinterpret_cast<float4 *>(dst)[0] = make_float4(0.f, 0.f, 0.f, 0.f);
-          reinterpret_cast<float4 *>(dst)[1] = make_float4(0.f, 0.f, 0.f, 0.f);
-          mbar_arrive(&S.sfull[slot]);
-        }
+      // this stage's pages (lanes 0..3), validated: an entry outside the pool is reported and
+      // treated as no page
+      int pid = __shfl_sync(0xFFFFFFFFu, batch_cur, (bs * kStagePages + lane) & 31);
+      if (lane < kStagePages && pid != -1 && (pid < 0 || pid >= p.num_pages)) {
+        report(p.d_status, DSV4_DEV_BAD_PAGE);
+        pid = -1;
       }
+      if (lane >= kStagePages) pid = -1;
       int rows[kStagePages];
 #pragma unroll
       for (int i = 0; i < kStagePages; ++i) {
-        const int v = __shfl_sync(0xFFFFFFFFu, batch_cur, bs * kStagePages + i);
+        const int v = __shfl_sync(0xFFFFFFFFu, pid, i);
         rows[i] = v >= 0 ? v * kPerPage : oob_row;
       }
+      int ok = 1;
       if (lane == 0) {
-        if (new_seg) {
+        if (k >= kSlots && !mbar_wait(&S.sempty[slot], static_cast<uint32_t>((k / kSlots - 1) & 1), &S.abort_flag))
+          ok = 0;
+        if (ok) {  // key scales: one 256-byte bulk copy per valid page, zeros for the others
+          uint32_t bytes = 0;
+#pragma unroll
+          for (int i = 0; i < kStagePages; ++i) bytes += rows[i] != oob_row ? kPerPage * 4 : 0;
+          float4 *z = reinterpret_cast<float4 *>(S.sig[slot]);
+#pragma unroll
+          for (int i = 0; i < kStagePages; ++i)
+            if (rows[i] == oob_row)
+              for (int u = 0; u < kPerPage / 4; ++u) z[i * kPerPage / 4 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
+          fence_proxy_async_smem();  // the slot is written by bulk copies too
+          mbar_arrive_expect_tx(&S.sfull[slot], bytes);
+#pragma unroll
+          for (int i = 0; i < kStagePages; ++i)
+            if (rows[i] != oob_row)
+              bulk_load(&S.sig[slot][i * kPerPage], p.k_scales + static_cast<size_t>(rows[i]), kPerPage * 4,
+                        &S.sfull[slot]);
+        }
+        if (ok && new_seg) {
           ++seg;
           const int qs = seg & 1;
           if (seg >= 2 && !mbar_wait(&S.qempty[qs], ((seg >> 1) - 1) & 1, &S.abort_flag)) ok = 0;
@@ -353,7 +361,6 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
       if (!ok) break;
       ++k;
     }
-    asm volatile("cp.async.wait_all;" ::: "memory");
     if (lane == 0 && S.abort_flag) {
       // let key loads already in flight land before the CTA leaves
       const long long from = k > kStages ? k - kStages : 0;
@@ -509,8 +516,8 @@ __device__ __forceinline__ void cluster_sync_all() {
 __device__ __forceinline__ int ld_cluster(const int *p, uint32_t rank) {
   uint32_t ra;
   int v;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p)), "r"(rank));
-  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(ra) : "memory");
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p)), "r"(rank));
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(ra));
   return v;
 }
 __device__ __forceinline__ int warp_sum_int(int v) {
@@ -534,6 +541,8 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
   const int64_t n = visible_entries(n_entries, pos, m, b, capacity, d_status, rank == 0 && tid == 0);
   const int64_t lo = static_cast<int64_t>(rank) * slice;
   const int cnt = static_cast<int>(n > lo ? (n - lo < slice ? n - lo : slice) : 0);
+  pdl_wait();  // the scores come from the kernel before
+  pdl_launch_dependents();
   const float *src = scores + static_cast<size_t>(b) * ld + lo;
   for (int i = tid * 4; i < cnt; i += kTkThreads * 4) {
     float v[4];
@@ -556,20 +565,18 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
   auto pass = [&](int shift, int par) {
     for (int i = tid; i < 256; i += kTkThreads) hist[par][i] = 0;
     __syncthreads();
-    for (int i0 = 0; i0 < cnt; i0 += kTkThreads) {
-      const int i = i0 + tid;
-      int bin = 256;
-      if (i < cnt) {
-        const uint32_t key = keys[i];
-        if (key != 0u && (key & mask) == prefix) bin = static_cast<int>((key >> shift) & 0xFF);
-      }
-      const unsigned peers = __match_any_sync(0xFFFFFFFFu, bin);
-      if (bin < 256 && lane == __ffs(peers) - 1) atomicAdd(&hist[par][bin], __popc(peers));
+    for (int i = tid; i < cnt; i += kTkThreads) {
+      const uint32_t key = keys[i];
+      if (key != 0u && (key & mask) == prefix) atomicAdd(&hist[par][(key >> shift) & 0xFF], 1);
     }
     cluster_sync_all();
-    if (tid < 256) {
+    if (tid < 256) {  // all remote loads in flight before the first is used
+      int v[kTkMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kTkMaxCluster; ++r) v[r] = r < static_cast<int>(cs) ? ld_cluster(&hist[par][tid], r) : 0;
       int s = 0;
-      for (uint32_t r = 0; r < cs; ++r) s += ld_cluster(&hist[par][tid], r);
+#pragma unroll
+      for (int r = 0; r < kTkMaxCluster; ++r) s += v[r];
       ghist[tid] = s;
     }
     __syncthreads();
@@ -639,10 +646,10 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
       xch[0] = run;
     }
     cluster_sync_all();
-    if (tid == 0) {
-      int before = 0;
-      for (uint32_t r = 0; r < rank; ++r) before += ld_cluster(&xch[0], r);
-      bcast = before;
+    if (warp == 0) {  // lane r reads CTA r
+      int v = lane < static_cast<int>(rank) ? ld_cluster(&xch[0], lane) : 0;
+      v = warp_sum_int(v);
+      if (lane == 0) bcast = v;
     }
     __syncthreads();
   }
@@ -679,15 +686,13 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
     xch[1] = run;
   }
   cluster_sync_all();
-  if (tid == 0) {
-    int before = 0, all = 0;
-    for (uint32_t r = 0; r < cs; ++r) {
-      const int v = ld_cluster(&xch[1], r);
-      if (r < rank) before += v;
-      all += v;
+  if (warp == 0) {  // lane r reads CTA r
+    const int v = lane < static_cast<int>(cs) ? ld_cluster(&xch[1], lane) : 0;
+    const int before = warp_sum_int(lane < static_cast<int>(rank) ? v : 0), all = warp_sum_int(v);
+    if (lane == 0) {
+      sel_above = before;
+      sel_count = all;
     }
-    sel_above = before;
-    sel_count = all;
   }
   __syncthreads();
   walk(true, sel_above + warp_base[warp]);
@@ -707,6 +712,8 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const unsigned long long *cand, int64_t stride,
                                                                   const int *cand_count, int k, int32_t *idx,
                                                                   float *scores, uint32_t *d_status, int smem_keys) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ unsigned long long skeys[];  // [smem_keys] staged candidates, then [kp2] selected
   __shared__ int hist[256];
   __shared__ int sel_digit, sel_above, sel_count, kept;
@@ -872,8 +879,7 @@ cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st) {
   const size_t smem = sizeof(TcSmem<H>) + 1024 + (2 * static_cast<size_t>(p.B) + 1) * 8;
   cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  indexer_tc_kernel<H><<<tc_grid(), kIxThreads, smem, st>>>(tp);
-  return cudaGetLastError();
+  return launch_pdl(indexer_tc_kernel<H>, dim3(tc_grid()), dim3(kIxThreads), smem, st, 1, tp);
 }
 
 }  // namespace
@@ -913,20 +919,9 @@ cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t 
       e = cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
       if (e != cudaSuccess) return e;
     }
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B));
-    cfg.blockDim = dim3(kTkThreads);
-    cfg.dynamicSmemBytes = tsmem;
-    cfg.stream = st;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeClusterDimension;
-    attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
-    attr[0].val.clusterDim.y = 1;
-    attr[0].val.clusterDim.z = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, topk_scores_kernel, static_cast<const float *>(scores), score_ld(p),
-                              p.n_entries, p.pos, p.m, capacity_of(p), p.k, slice, p.idx, p.scores, p.d_status);
+    return launch_pdl(topk_scores_kernel, dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B)),
+                      dim3(kTkThreads), tsmem, st, cs, static_cast<const float *>(scores), score_ld(p), p.n_entries,
+                      p.pos, p.m, capacity_of(p), p.k, slice, p.idx, p.scores, p.d_status);
   } else {
     e = cudaMemsetAsync(cand_count, 0, static_cast<size_t>(p.B) * sizeof(int), st);
     if (e != cudaSuccess) return e;
@@ -935,8 +930,7 @@ cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t 
     const size_t smem = (static_cast<size_t>(p.H) * p.Dq + p.H) * sizeof(float);
     e = cudaFuncSetAttribute(indexer_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    indexer_simt_kernel<<<grid, 256, smem, st>>>(p, cand, stride, cand_count);
-    e = cudaGetLastError();
+    e = launch_pdl(indexer_simt_kernel, grid, dim3(256), smem, st, 1, p, cand, stride, cand_count);
     if (e != cudaSuccess) return e;
   }
   // merge candidate lists: stage up to ~200 KB of candidates in shared memory
@@ -944,9 +938,9 @@ cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t 
   const size_t ssmem = static_cast<size_t>(smem_keys) * sizeof(unsigned long long);
   e = cudaFuncSetAttribute(topk_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
   if (e != cudaSuccess) return e;
-  topk_select_kernel<<<p.B, kSelThreads, ssmem, st>>>(cand, stride, cand_count, p.k, p.idx, p.scores, p.d_status,
-                                                      smem_keys);
-  return cudaGetLastError();
+  return launch_pdl(topk_select_kernel, dim3(p.B), dim3(kSelThreads), ssmem, st, 1,
+                    static_cast<const unsigned long long *>(cand), stride, static_cast<const int *>(cand_count), p.k,
+                    p.idx, p.scores, p.d_status, smem_keys);
 }
 
 }  // namespace dsv4

@@ -172,6 +172,8 @@ struct MqaTcParams {
   float scale_log2;
   float *part_o;   // [B + G][H][D]
   float *part_ml;  // [B + G][H][2]
+  uint16_t *qp;    // [B][H][D] query rotated by RoPE_pos, fp16 (scaled per head) or bf16
+  float *qinv;     // [B][H] 2^-e undoing the per-head scale (1 for bf16)
 };
 
 // Operands of the two MMAs. fp8 caches: fp16 (e4m3 -> fp16 is exact, and fp16 keeps 11
@@ -291,13 +293,77 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const long long *prefi
   }
 }
 
-// ---- warps 4-7 (gw = 0..3): query of a new segment and the key tiles.
-// Query: warp gw owns heads 16gw .. 16gw+15; lane l owns 16-byte runs (8 dims) l and l + 32
-// of each. The raw bf16 runs are copied into their swizzled homes, then rotated by RoPE_pos
-// and stored as bf16, or as fp16 scaled per head by a power of two (qinv undoes it in the
-// logits) so that |q| < 2^14 whatever the input range. RoPE pairs never straddle a run.
-__device__ __forceinline__ void query_issue(const MqaLaunch &p, MqaSmem &S, int b, int gw, int lane) {
-  const uint16_t *q = static_cast<const uint16_t *>(p.q) + static_cast<size_t>(b) * kH * kD;
+// ---- the query of every sequence, rotated by RoPE_pos once: bf16, or fp16 scaled per
+// head by a power of two (qinv undoes it in the logits) so that |q| < 2^14 whatever the
+// input range. grid (B), 256 threads: thread t owns dims 128 (t & 3) .. +127 of head t / 4.
+// It reads only the caller's query and writes only qp/qinv, which nothing before it on the
+// stream reads, so it runs before its pdl_wait(), beside the kernel before it.
+__global__ void __launch_bounds__(256) mqa_query_kernel(const MqaTcParams P) {
+  const MqaLaunch &p = P.a;
+  __shared__ float cs[kD / 2], sn[kD / 2];
+  const int b = blockIdx.x, t = threadIdx.x, h = t >> 2, d0 = (t & 3) * 128;
+  const bool f16 = fp16_operands(p);
+  const int half = p.rope_dims / 2, rope0 = kD - p.rope_dims;
+  const int64_t pos = p.pos[b];
+  for (int i = t; i < half; i += 256) rope_cos_sin(pos, i, p.rope_theta1, &cs[i], &sn[i]);
+  const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) +
+                                                     (static_cast<size_t>(b) * kH + h) * kD + d0);
+  uint4 raw[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) raw[i] = __ldg(src + i);
+  __syncthreads();
+  auto rotated = [&](int i, float *x) {  // the 8 values of run i, rotated where they are rope dims
+    const uint32_t v[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      x[2 * u] = __uint_as_float(v[u] << 16);
+      x[2 * u + 1] = __uint_as_float(v[u] & 0xFFFF0000u);
+      const int d = d0 + i * 8 + 2 * u;
+      if (d >= rope0) {
+        const float c = cs[(d - rope0) >> 1], sv = sn[(d - rope0) >> 1];
+        const float x0 = x[2 * u], x1 = x[2 * u + 1];
+        x[2 * u] = x0 * c - x1 * sv;
+        x[2 * u + 1] = x0 * sv + x1 * c;
+      }
+    }
+  };
+  float qs = 1.0f, qi = 1.0f;
+  if (f16) {
+    float am = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float x[8];
+      rotated(i, x);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) am = fmaxf(am, fabsf(x[u]));
+    }
+    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
+    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
+    int e = 0;
+    if (am > 0.f) frexpf(am, &e);  // am < 2^e
+    qi = am > 0.f ? ldexpf(1.0f, e - 14) : 1.0f;
+    qs = am > 0.f ? ldexpf(1.0f, 14 - e) : 1.0f;
+  }
+  uint4 *dst = reinterpret_cast<uint4 *>(P.qp + (static_cast<size_t>(b) * kH + h) * kD + d0);
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float x[8];
+    rotated(i, x);
+    dst[i] = f16 ? make_uint4(pack_f16x2(x[0] * qs, x[1] * qs), pack_f16x2(x[2] * qs, x[3] * qs),
+                              pack_f16x2(x[4] * qs, x[5] * qs), pack_f16x2(x[6] * qs, x[7] * qs))
+                 : make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
+                              pack_bf16x2(x[6], x[7]));
+  }
+  if ((t & 3) == 0) P.qinv[static_cast<size_t>(b) * kH + h] = qi;
+  pdl_wait();
+  pdl_launch_dependents();
+}
+
+// ---- warps 4-7 (gw = 0..3): query of a new segment and the key tiles. Query: warp gw
+// copies the prepared rows of heads 16gw .. 16gw+15 into their swizzled homes (lane l owns
+// 16-byte runs l and l + 32 of each) and their scales.
+__device__ __forceinline__ void query_issue(const MqaTcParams &P, MqaSmem &S, int b, int gw, int lane) {
+  const uint16_t *q = P.qp + static_cast<size_t>(b) * kH * kD;
 #pragma unroll 4
   for (int hh = 0; hh < 16; ++hh) {
     const int h = gw * 16 + hh;
@@ -310,64 +376,9 @@ __device__ __forceinline__ void query_issue(const MqaLaunch &p, MqaSmem &S, int 
   cp_async_commit();
 }
 
-__device__ __forceinline__ void query_finish(const MqaLaunch &p, MqaSmem &S, int64_t pos, int par, int gw, int lane) {
-  const bool f16 = fp16_operands(p);
-  const int rope0 = kD - p.rope_dims;
-  float c[2][4], sn[2][4];
-#pragma unroll
-  for (int r = 0; r < 2; ++r) {
-    const int d0 = (lane + 32 * r) * 8;
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      c[r][u] = 1.f;
-      sn[r][u] = 0.f;
-      if (d0 >= rope0) rope_cos_sin(pos, (d0 + 2 * u - rope0) >> 1, p.rope_theta1, &c[r][u], &sn[r][u]);
-    }
-  }
+__device__ __forceinline__ void query_finish(const MqaTcParams &P, MqaSmem &S, int b, int par, int gw, int lane) {
+  if (lane < 16) S.qinv[par][gw * 16 + lane] = P.qinv[static_cast<size_t>(b) * kH + gw * 16 + lane];
   cp_async_wait_all();
-  __syncwarp();
-#pragma unroll 1
-  for (int hh = 0; hh < 16; ++hh) {
-    const int h = gw * 16 + hh;
-    float x[2][8];
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int seg = lane + 32 * r;
-      const uint4 w = *reinterpret_cast<const uint4 *>(&S.q[seg >> 3][0] + sw128_offset(h, seg & 7));
-      const uint32_t v[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const float x0 = __uint_as_float(v[u] << 16), x1 = __uint_as_float(v[u] & 0xFFFF0000u);
-        x[r][2 * u] = x0 * c[r][u] - x1 * sn[r][u];
-        x[r][2 * u + 1] = x0 * sn[r][u] + x1 * c[r][u];
-      }
-    }
-    float qs = 1.0f, qi = 1.0f;
-    if (f16) {
-      float am = 0.f;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) am = fmaxf(am, fmaxf(fabsf(x[0][u]), fabsf(x[1][u])));
-      am = warp_max(am);
-      int e = 0;
-      if (am > 0.f) frexpf(am, &e);  // am < 2^e
-      qi = am > 0.f ? ldexpf(1.0f, e - 14) : 1.0f;
-      qs = am > 0.f ? ldexpf(1.0f, 14 - e) : 1.0f;
-    }
-    if (lane == 0) S.qinv[par][h] = qi;
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int seg = lane + 32 * r;
-      uint4 o;
-      if (f16) {
-        o = make_uint4(pack_f16x2(x[r][0] * qs, x[r][1] * qs), pack_f16x2(x[r][2] * qs, x[r][3] * qs),
-                       pack_f16x2(x[r][4] * qs, x[r][5] * qs), pack_f16x2(x[r][6] * qs, x[r][7] * qs));
-      } else {
-        o = make_uint4(pack_bf16x2(x[r][0], x[r][1]), pack_bf16x2(x[r][2], x[r][3]), pack_bf16x2(x[r][4], x[r][5]),
-                       pack_bf16x2(x[r][6], x[r][7]));
-      }
-      *reinterpret_cast<uint4 *>(&S.q[seg >> 3][0] + sw128_offset(h, seg & 7)) = o;
-    }
-  }
 }
 
 // Key tile of one chunk: warp gw fills rows 16gw .. 16gw+15. fp8 rows (32 runs of 16
@@ -421,7 +432,8 @@ __device__ __forceinline__ void gather_store_fp8(MqaSmem &S, uint8_t *kt, int ms
   }
 }
 
-__device__ void gather_role(const MqaLaunch &p, MqaSmem &S, const long long *prefix, long long c0, long long c1) {
+__device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const long long *prefix, long long c0, long long c1) {
+  const MqaLaunch &p = P.a;
   const int lane = threadIdx.x & 31, gw = (threadIdx.x >> 5) - kGatherWarp0;
   const bool fp8 = p.kv_dt == DSV4_FP8E4M3;
   int seg = -1;
@@ -433,7 +445,7 @@ __device__ void gather_role(const MqaLaunch &p, MqaSmem &S, const long long *pre
     if (ok && cp.first) {
       ++seg;
       if (seg >= 1) ok = mbar_wait(&S.q_empty, static_cast<uint32_t>((seg - 1) & 1), &S.abort_flag);
-      if (ok) query_issue(p, S, cp.b, gw, lane);
+      if (ok) query_issue(P, S, cp.b, gw, lane);
     }
     if (ok && n >= 2) ok = mbar_wait(&S.k_empty[s], static_cast<uint32_t>((n / 2 - 1) & 1), &S.abort_flag);
     if (!__all_sync(0xFFFFFFFFu, ok)) {
@@ -464,7 +476,7 @@ __device__ void gather_role(const MqaLaunch &p, MqaSmem &S, const long long *pre
       mbar_arrive(&S.meta_empty[ms]);
     }
     if (cp.first) {
-      query_finish(p, S, key_list(p, cp.b, false).pos, seg & 1, gw, lane);
+      query_finish(P, S, cp.b, seg & 1, gw, lane);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.q_full);
@@ -654,16 +666,19 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const long long *
       }
       float *po = P.part_o + (slot * kH + head) * kD;
 #pragma unroll 1
-      for (int col = 0; col < kD; col += 32) {
-        uint32_t o[32];
-        tmem_ld32(lane_base + col, o);
+      for (int col = 0; col < kD; col += 128) {  // four loads in flight per wait
+        uint32_t o[4][32];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + col + 32 * c, o[c]);
         tmem_ld_wait();
         if (!hi) {
 #pragma unroll
-          for (int i = 0; i < 32; i += 4)
-            __stcg(reinterpret_cast<float4 *>(po + col + i),
-                   make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]), __uint_as_float(o[i + 2]),
-                               __uint_as_float(o[i + 3])));
+          for (int c = 0; c < 4; ++c)
+#pragma unroll
+            for (int i = 0; i < 32; i += 4)
+              __stcg(reinterpret_cast<float4 *>(po + col + 32 * c + i),
+                     make_float4(__uint_as_float(o[c][i]), __uint_as_float(o[c][i + 1]), __uint_as_float(o[c][i + 2]),
+                                 __uint_as_float(o[c][i + 3])));
         }
       }
       tc_fence_before();
@@ -704,6 +719,8 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     tmem_relinquish();
   }
   chunk_prefix(p, prefix, prefix + p.B + 1, blockIdx.x == 0);
+  pdl_wait();  // the selection (idx) and the caches come from the kernels before
+  pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -712,7 +729,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
   const long long c0 = (T * blockIdx.x) / G, c1 = (T * (blockIdx.x + 1)) / G;
 
   if (warp == kMetaWarp) meta_role(p, S, prefix, c0, c1);
-  else if (warp >= kGatherWarp0 && warp < kGatherWarp0 + 4) gather_role(p, S, prefix, c0, c1);
+  else if (warp >= kGatherWarp0 && warp < kGatherWarp0 + 4) gather_role(P, S, prefix, c0, c1);
   else if (warp == kMmaWarp) {
     if ((tid & 31) == 0) mma_role(p, S, prefix, c0, c1, tmem);
   } else softmax_role(P, S, prefix, c0, c1, tmem);
@@ -766,6 +783,8 @@ __global__ void __launch_bounds__(256) mqa_merge_kernel(const MqaTcParams P, int
     __syncthreads();
   }
   const int np = n;
+  pdl_wait();  // the partials come from the kernel before
+  pdl_launch_dependents();
   for (int j = tid; j < np * 8; j += 256) {
     const size_t slot = static_cast<size_t>(b) + cta[j >> 3];
     const float2 ml = *reinterpret_cast<const float2 *>(P.part_ml + (slot * kH + h0 + (j & 7)) * 2);
@@ -843,6 +862,8 @@ __global__ void __launch_bounds__(256) mqa_merge_kernel(const MqaTcParams P, int
 constexpr int kSimtChunk = 256;
 
 __global__ void __launch_bounds__(256) mqa_simt_kernel(const MqaLaunch p, float scale_log2) {
+  pdl_wait();
+  pdl_launch_dependents();
   extern __shared__ float sm[];
   float *qr = sm;                      // [D]
   float *xs = qr + p.D;                // [chunk]
@@ -957,7 +978,9 @@ bool mqa_uses_tensor_cores(const MqaLaunch &p) {
 size_t mqa_workspace_bytes(const MqaLaunch &p) {
   if (!mqa_uses_tensor_cores(p)) return 0;
   const size_t slots = static_cast<size_t>(p.B) + tc_grid();
-  return align_up(slots * kH * kD * sizeof(float), 256) + align_up(slots * kH * 2 * sizeof(float), 256);
+  return align_up(slots * kH * kD * sizeof(float), 256) + align_up(slots * kH * 2 * sizeof(float), 256) +
+         align_up(static_cast<size_t>(p.B) * kH * kD * sizeof(uint16_t), 256) +
+         align_up(static_cast<size_t>(p.B) * kH * sizeof(float), 256);
 }
 
 cudaError_t launch_mqa(const MqaLaunch &p0, void *ws, cudaStream_t st) {
@@ -968,28 +991,33 @@ cudaError_t launch_mqa(const MqaLaunch &p0, void *ws, cudaStream_t st) {
     P.a = p;
     P.scale_log2 = softmax_scale_log2(p);
     const size_t slots = static_cast<size_t>(p.B) + tc_grid();
-    P.part_o = static_cast<float *>(ws);
-    P.part_ml = reinterpret_cast<float *>(static_cast<char *>(ws) + align_up(slots * kH * kD * sizeof(float), 256));
-    const size_t smem = sizeof(MqaSmem) + 1024 + (static_cast<size_t>(p.B) + 1 + kThreads) * sizeof(long long);
-    cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    char *w = static_cast<char *>(ws);
+    P.part_o = reinterpret_cast<float *>(w);
+    w += align_up(slots * kH * kD * sizeof(float), 256);
+    P.part_ml = reinterpret_cast<float *>(w);
+    w += align_up(slots * kH * 2 * sizeof(float), 256);
+    P.qp = reinterpret_cast<uint16_t *>(w);
+    w += align_up(static_cast<size_t>(p.B) * kH * kD * sizeof(uint16_t), 256);
+    P.qinv = reinterpret_cast<float *>(w);
+    cudaError_t e = launch_pdl(mqa_query_kernel, dim3(p.B), dim3(256), 0, st, 1, P);
     if (e != cudaSuccess) return e;
-    mqa_tc_kernel<<<tc_grid(), kThreads, smem, st>>>(P);
-    e = cudaGetLastError();
+    const size_t smem = sizeof(MqaSmem) + 1024 + (static_cast<size_t>(p.B) + 1 + kThreads) * sizeof(long long);
+    e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = launch_pdl(mqa_tc_kernel, dim3(tc_grid()), dim3(kThreads), smem, st, 1, P);
     if (e != cudaSuccess) return e;
     const size_t msmem = static_cast<size_t>(tc_grid()) * 16 * sizeof(float) +
                          static_cast<size_t>((tc_grid() + 1) & ~1) * sizeof(int) +
                          (static_cast<size_t>(p.B) + 1 + 256) * sizeof(long long);
     e = cudaFuncSetAttribute(mqa_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     if (e != cudaSuccess) return e;
-    mqa_merge_kernel<<<dim3(p.B, kH / 8), 256, msmem, st>>>(P, tc_grid());
-    return cudaGetLastError();
+    return launch_pdl(mqa_merge_kernel, dim3(p.B, kH / 8), dim3(256), msmem, st, 1, P, tc_grid());
   }
   const size_t smem = (2 * static_cast<size_t>(p.D) + 2 * kSimtChunk + 32) * sizeof(float) +
                       kSimtChunk * sizeof(void *) + 16;
   cudaError_t e = cudaFuncSetAttribute(mqa_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  mqa_simt_kernel<<<dim3(p.H, p.B), 256, smem, st>>>(p, softmax_scale_log2(p));
-  return cudaGetLastError();
+  return launch_pdl(mqa_simt_kernel, dim3(p.H, p.B), dim3(256), smem, st, 1, p, softmax_scale_log2(p));
 }
 
 }  // namespace dsv4
