@@ -90,59 +90,10 @@ __device__ __forceinline__ const uint8_t *key_row(const MqaLaunch &p, int b, con
   return static_cast<const uint8_t *>(p.pages) + row * p.D * esz;
 }
 
-// prefix[b] = number of 64-key chunks of sequences 0..b-1, prefix[B] = total; computed by
-// every thread of the CTA (contiguous slices of sequences, then a two-level shuffle scan of
-// the slice sums). red: 32 scratch values. blockDim.x is a multiple of 32.
-__device__ void chunk_prefix(const MqaLaunch &p, long long *prefix, long long *red, bool report_it) {
-  const int nt = blockDim.x, t = threadIdx.x, lane = t & 31, warp = t >> 5;
-  const int lo = static_cast<int>((static_cast<long long>(p.B) * t) / nt);
-  const int hi = static_cast<int>((static_cast<long long>(p.B) * (t + 1)) / nt);
-  long long mine = 0;
-  for (int b = lo; b < hi; ++b) {
-    const KeyList L = key_list(p, b, report_it);
-    const long long c = (L.nw + L.nsel + 63) / 64;
-    prefix[b] = c;
-    mine += c;
-  }
-  long long v = mine;  // inclusive scan within the warp
-#pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const long long u = __shfl_up_sync(0xFFFFFFFFu, v, o);
-    if (lane >= o) v += u;
-  }
-  if (lane == 31) red[warp] = v;
-  __syncthreads();
-  if (warp == 0) {
-    long long w = lane < (nt >> 5) ? red[lane] : 0;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const long long u = __shfl_up_sync(0xFFFFFFFFu, w, o);
-      if (lane >= o) w += u;
-    }
-    red[lane] = w;
-  }
-  __syncthreads();
-  long long acc = v - mine + (warp > 0 ? red[warp - 1] : 0);
-  if (t == nt - 1) prefix[p.B] = acc + mine;
-  for (int b = lo; b < hi; ++b) {
-    const long long c = prefix[b];
-    prefix[b] = acc;
-    acc += c;
-  }
-  __syncthreads();
-}
-
-__device__ __forceinline__ int find_seq(const long long *prefix, int B, long long g) {
-  int lo = 0, hi = B - 1;
-  while (lo < hi) {
-    const int mid = (lo + hi + 1) >> 1;
-    if (prefix[mid] <= g) lo = mid; else hi = mid - 1;
-  }
-  return lo;
-}
-
 // ------------------------------------------------------------------------------------
-// tensor-core kernel
+// tensor-core kernel: one thread-block cluster of cs CTAs per sequence; CTA r takes a
+// contiguous run of the sequence's 64-key chunks, and the cluster merges the CTAs' partial
+// results in distributed shared memory.
 
 constexpr int kH = 64, kD = 512, kCh = 64;
 constexpr int kAtom = kCh * 128;  // one 64-dim column block of a 64-row tile: 8 KB
@@ -151,18 +102,24 @@ constexpr int kMetaSlots = 4;     // chunks whose key metadata is resolved ahead
 // MMA issue (and TMEM allocation), warp 9 key metadata
 constexpr int kSoftWarp0 = 0, kGatherWarp0 = 4, kMmaWarp = 8, kMetaWarp = 9;
 constexpr int kThreads = 320;
+constexpr int kMaxCluster = 16;
 
 struct alignas(1024) MqaSmem {
-  uint8_t q[kD / 64][kH * 128];      // 64 KB, K-major SW128, 8 atoms of 64 dims
-  uint8_t k[2][kD / 64][kCh * 128];  // 2 x 64 KB key tiles (stage = chunk parity)
-  uint8_t p[kH * 128];               // 8 KB: P[64 heads][64 keys], K-major SW128
+  uint8_t q[kD / 64][kH * 128];  // 64 KB, K-major SW128, 8 atoms of 64 dims
+  union {
+    uint8_t k[2][kD / 64][kCh * 128];  // 2 x 64 KB key tiles (stage = chunk parity)
+    float obuf[kH][kD];                // after the last MMA: this CTA's weighted O (swizzled runs)
+  };
+  uint8_t p[kH * 128];                   // 8 KB: P[64 heads][64 keys], K-major SW128
   const uint8_t *mrow[kMetaSlots][kCh];  // row address of each key of a chunk (nullptr: none)
   float mscale[kMetaSlots][kCh];         // its row scale
   float rscale[2][kCh];                  // row scale per key of a staged tile (0: no key)
   int ec[2];                             // tile exponent: K rows hold code * scale * 2^-ec
-  float qinv[2][kH];                     // 2^-e of the per-head query scale, by segment parity
+  float qinv[kH];                        // 2^-e of the per-head query scale
+  float red_m[kH], red_l[kH];            // this CTA's reference max and sum per head (read by the cluster)
+  float wgt[kH], inv_l[kH], lse[kH];     // its weight in the merge, 1 / total sum, log-sum-exp
   uint64_t meta_full[kMetaSlots], meta_empty[kMetaSlots];
-  uint64_t k_full[2], k_empty[2], q_full, q_empty, s_full, s_empty, p_full, o_full, o_empty;
+  uint64_t k_full[2], k_empty[2], q_full, s_full, s_empty, p_full, o_full;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -170,8 +127,6 @@ struct alignas(1024) MqaSmem {
 struct MqaTcParams {
   MqaLaunch a;
   float scale_log2;
-  float *part_o;   // [B + G][H][D]
-  float *part_ml;  // [B + G][H][2]
   uint16_t *qp;    // [B][H][D] query rotated by RoPE_pos, fp16 (scaled per head) or bf16
   float *qinv;     // [B][H] 2^-e undoing the per-head scale (1 for bf16)
 };
@@ -185,33 +140,59 @@ __device__ __forceinline__ uint32_t pack_f16x2(float a, float b) {
   return *reinterpret_cast<uint32_t *>(&h);
 }
 
-// where chunk g sits: its sequence, and whether it opens / closes this CTA's run of it
-struct ChunkPos {
-  int b;
-  bool first, last;
-};
-__device__ __forceinline__ ChunkPos chunk_pos(const long long *prefix, int B, long long g, long long c0,
-                                              long long c1) {
-  ChunkPos c;
-  c.b = find_seq(prefix, B, g);
-  c.first = g == c0 || prefix[c.b] == g;
-  c.last = g + 1 == c1 || prefix[c.b + 1] == g + 1;
-  return c;
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
 }
+__device__ __forceinline__ uint32_t cluster_size() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
+  return r;
+}
+// every thread of every CTA of the cluster; orders shared-memory writes before it with reads after it
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// address of the same shared variable in CTA `rank` of this cluster
+__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
+  uint32_t ra;
+  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p)), "r"(rank));
+  return ra;
+}
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
+  return v;
+}
+// 16-byte run c of row h of obuf: runs are XOR-swizzled by h so that the 16 rows a warp
+// writes at once land in different banks
+__device__ __forceinline__ int obuf_run(int h, int c) { return c ^ (h & 7); }
+
+// This CTA's chunks of its sequence: [lo, hi) of the sequence's C chunks.
+struct ChunkRange {
+  int b;
+  long long lo, hi;
+};
 
 // ---- warp 9: row address and scale of every key of up to kMetaSlots chunks at a time.
 // The idx -> block table -> scale chain is staged over all keys of the batch, so its three
 // memory latencies are paid once per batch.
-__device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const long long *prefix, long long c0, long long c1) {
-  const int lane = threadIdx.x & 31;
+__device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const KeyList &L, const ChunkRange &cr) {
+  const int lane = threadIdx.x & 31, b = cr.b;
   const int per_page = DSV4_PAGE_POSITIONS / p.m;
   const size_t esz = dtype_size(p.kv_dt);
   constexpr int kKeys = kMetaSlots * 2;  // keys per lane per batch
-  for (long long g0 = c0; g0 < c1; g0 += kMetaSlots) {
-    const int nb = static_cast<int>(c1 - g0 < kMetaSlots ? c1 - g0 : kMetaSlots);
+  for (long long g0 = cr.lo; g0 < cr.hi; g0 += kMetaSlots) {
+    const int nb = static_cast<int>(cr.hi - g0 < kMetaSlots ? cr.hi - g0 : kMetaSlots);
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
-      const long long n = g0 + i - c0;
+      const long long n = g0 + i - cr.lo;
       if (n >= kMetaSlots && lane == 0 &&
           !mbar_wait(&S.meta_empty[n % kMetaSlots], static_cast<uint32_t>((n / kMetaSlots - 1) & 1), &S.abort_flag))
         ok = false;
@@ -220,26 +201,14 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const long long *prefi
       if (lane == 0) S.abort_flag = 1;
       return;
     }
-    int bc[kMetaSlots];
-    KeyList Lc[kMetaSlots];
-#pragma unroll
-    for (int i = 0; i < kMetaSlots; ++i) {
-      bc[i] = i < nb ? find_seq(prefix, p.B, g0 + i) : 0;
-      if (i < nb) Lc[i] = key_list(p, bc[i], false);
-    }
-    int bseq[kKeys];
     int64_t j[kKeys];  // >= 0: entry index; -1: none; -2 - slot: window ring slot
     int32_t page[kKeys];
 #pragma unroll
     for (int u = 0; u < kKeys; ++u) {  // stage 1: key list position -> entry index (idx load)
       const int i = u >> 1;
       j[u] = -1;
-      bseq[u] = 0;
       if (i < nb) {
-        const int b = bc[i];
-        const KeyList &L = Lc[i];
-        const int64_t t = (g0 + i - prefix[b]) * kCh + lane + 32 * (u & 1);
-        bseq[u] = b;
+        const int64_t t = (g0 + i) * kCh + lane + 32 * (u & 1);
         if (t < L.nw) {
           const int64_t pw = L.pos - L.nw + 1 + t;
           j[u] = -2 - (static_cast<int64_t>(b) * p.W + pw % p.W);
@@ -261,7 +230,7 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const long long *prefi
     for (int u = 0; u < kKeys; ++u) {  // stage 2: entry -> physical page (block table load)
       page[u] = -1;
       if (j[u] >= 0) {
-        page[u] = p.block_table[static_cast<size_t>(bseq[u]) * p.max_blocks + j[u] / per_page];
+        page[u] = p.block_table[static_cast<size_t>(b) * p.max_blocks + j[u] / per_page];
         if (page[u] < 0 || page[u] >= p.num_pages) {
           report(p.d_status, DSV4_DEV_BAD_PAGE);
           page[u] = -1;
@@ -283,62 +252,62 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const long long *prefi
         rp = static_cast<const uint8_t *>(p.pages) + row * p.D * esz;
         sc = p.kv_dt == DSV4_FP8E4M3 ? p.scales[row] : 1.0f;
       }
-      const int slot = static_cast<int>((g0 + i - c0) % kMetaSlots);
+      const int slot = static_cast<int>((g0 + i - cr.lo) % kMetaSlots);
       S.mrow[slot][lane + 32 * (u & 1)] = rp;
       S.mscale[slot][lane + 32 * (u & 1)] = rp ? sc : 0.f;
     }
     __syncwarp();
     if (lane == 0)
-      for (int i = 0; i < nb; ++i) mbar_arrive(&S.meta_full[(g0 + i - c0) % kMetaSlots]);
+      for (int i = 0; i < nb; ++i) mbar_arrive(&S.meta_full[(g0 + i - cr.lo) % kMetaSlots]);
   }
 }
 
 // ---- the query of every sequence, rotated by RoPE_pos once: bf16, or fp16 scaled per
 // head by a power of two (qinv undoes it in the logits) so that |q| < 2^14 whatever the
-// input range. grid (B), 256 threads: thread t owns dims 128 (t & 3) .. +127 of head t / 4.
-// It reads only the caller's query and writes only qp/qinv, which nothing before it on the
-// stream reads, so it runs before its pdl_wait(), beside the kernel before it.
+// input range. grid (B, H / 16), 256 threads: thread t owns dims 32 (t & 15) .. +31 of head
+// 16 blockIdx.y + t / 16. It reads only the caller's query and writes only qp/qinv, which
+// nothing before it on the stream reads, so it runs before its pdl_wait(), beside the
+// kernel before it.
 __global__ void __launch_bounds__(256) mqa_query_kernel(const MqaTcParams P) {
   const MqaLaunch &p = P.a;
   __shared__ float cs[kD / 2], sn[kD / 2];
-  const int b = blockIdx.x, t = threadIdx.x, h = t >> 2, d0 = (t & 3) * 128;
+  const int b = blockIdx.x, t = threadIdx.x, h = blockIdx.y * 16 + (t >> 4), d0 = (t & 15) * 32;
   const bool f16 = fp16_operands(p);
   const int half = p.rope_dims / 2, rope0 = kD - p.rope_dims;
   const int64_t pos = p.pos[b];
   for (int i = t; i < half; i += 256) rope_cos_sin(pos, i, p.rope_theta1, &cs[i], &sn[i]);
   const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) +
                                                      (static_cast<size_t>(b) * kH + h) * kD + d0);
-  uint4 raw[16];
+  uint4 raw[4];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) raw[i] = __ldg(src + i);
+  for (int i = 0; i < 4; ++i) raw[i] = __ldg(src + i);
   __syncthreads();
-  auto rotated = [&](int i, float *x) {  // the 8 values of run i, rotated where they are rope dims
+  float x[4][8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // the 8 values of run i, rotated where they are rope dims
     const uint32_t v[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      x[2 * u] = __uint_as_float(v[u] << 16);
-      x[2 * u + 1] = __uint_as_float(v[u] & 0xFFFF0000u);
+      x[i][2 * u] = __uint_as_float(v[u] << 16);
+      x[i][2 * u + 1] = __uint_as_float(v[u] & 0xFFFF0000u);
       const int d = d0 + i * 8 + 2 * u;
       if (d >= rope0) {
         const float c = cs[(d - rope0) >> 1], sv = sn[(d - rope0) >> 1];
-        const float x0 = x[2 * u], x1 = x[2 * u + 1];
-        x[2 * u] = x0 * c - x1 * sv;
-        x[2 * u + 1] = x0 * sv + x1 * c;
+        const float x0 = x[i][2 * u], x1 = x[i][2 * u + 1];
+        x[i][2 * u] = x0 * c - x1 * sv;
+        x[i][2 * u + 1] = x0 * sv + x1 * c;
       }
     }
-  };
+  }
   float qs = 1.0f, qi = 1.0f;
   if (f16) {
     float am = 0.f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float x[8];
-      rotated(i, x);
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int u = 0; u < 8; ++u) am = fmaxf(am, fabsf(x[u]));
-    }
-    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 1));
-    am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, 2));
+      for (int u = 0; u < 8; ++u) am = fmaxf(am, fabsf(x[i][u]));
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) am = fmaxf(am, __shfl_xor_sync(0xFFFFFFFFu, am, o));
     int e = 0;
     if (am > 0.f) frexpf(am, &e);  // am < 2^e
     qi = am > 0.f ? ldexpf(1.0f, e - 14) : 1.0f;
@@ -346,15 +315,12 @@ __global__ void __launch_bounds__(256) mqa_query_kernel(const MqaTcParams P) {
   }
   uint4 *dst = reinterpret_cast<uint4 *>(P.qp + (static_cast<size_t>(b) * kH + h) * kD + d0);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    float x[8];
-    rotated(i, x);
-    dst[i] = f16 ? make_uint4(pack_f16x2(x[0] * qs, x[1] * qs), pack_f16x2(x[2] * qs, x[3] * qs),
-                              pack_f16x2(x[4] * qs, x[5] * qs), pack_f16x2(x[6] * qs, x[7] * qs))
-                 : make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
-                              pack_bf16x2(x[6], x[7]));
-  }
-  if ((t & 3) == 0) P.qinv[static_cast<size_t>(b) * kH + h] = qi;
+  for (int i = 0; i < 4; ++i)
+    dst[i] = f16 ? make_uint4(pack_f16x2(x[i][0] * qs, x[i][1] * qs), pack_f16x2(x[i][2] * qs, x[i][3] * qs),
+                              pack_f16x2(x[i][4] * qs, x[i][5] * qs), pack_f16x2(x[i][6] * qs, x[i][7] * qs))
+                 : make_uint4(pack_bf16x2(x[i][0], x[i][1]), pack_bf16x2(x[i][2], x[i][3]),
+                              pack_bf16x2(x[i][4], x[i][5]), pack_bf16x2(x[i][6], x[i][7]));
+  if ((t & 15) == 0) P.qinv[static_cast<size_t>(b) * kH + h] = qi;
   pdl_wait();
   pdl_launch_dependents();
 }
@@ -376,8 +342,8 @@ __device__ __forceinline__ void query_issue(const MqaTcParams &P, MqaSmem &S, in
   cp_async_commit();
 }
 
-__device__ __forceinline__ void query_finish(const MqaTcParams &P, MqaSmem &S, int b, int par, int gw, int lane) {
-  if (lane < 16) S.qinv[par][gw * 16 + lane] = P.qinv[static_cast<size_t>(b) * kH + gw * 16 + lane];
+__device__ __forceinline__ void query_finish(const MqaTcParams &P, MqaSmem &S, int b, int gw, int lane) {
+  if (lane < 16) S.qinv[gw * 16 + lane] = P.qinv[static_cast<size_t>(b) * kH + gw * 16 + lane];
   cp_async_wait_all();
 }
 
@@ -432,28 +398,22 @@ __device__ __forceinline__ void gather_store_fp8(MqaSmem &S, uint8_t *kt, int ms
   }
 }
 
-__device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const long long *prefix, long long c0, long long c1) {
+__device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &cr) {
   const MqaLaunch &p = P.a;
   const int lane = threadIdx.x & 31, gw = (threadIdx.x >> 5) - kGatherWarp0;
   const bool fp8 = p.kv_dt == DSV4_FP8E4M3;
-  int seg = -1;
-  for (long long g = c0; g < c1; ++g) {
-    const long long n = g - c0;
+  if (cr.lo < cr.hi) query_issue(P, S, cr.b, gw, lane);
+  for (long long g = cr.lo; g < cr.hi; ++g) {
+    const long long n = g - cr.lo;
     const int s = static_cast<int>(n & 1), ms = static_cast<int>(n % kMetaSlots);
-    const ChunkPos cp = chunk_pos(prefix, p.B, g, c0, c1);
     bool ok = mbar_wait(&S.meta_full[ms], static_cast<uint32_t>((n / kMetaSlots) & 1), &S.abort_flag);
-    if (ok && cp.first) {
-      ++seg;
-      if (seg >= 1) ok = mbar_wait(&S.q_empty, static_cast<uint32_t>((seg - 1) & 1), &S.abort_flag);
-      if (ok) query_issue(P, S, cp.b, gw, lane);
-    }
     if (ok && n >= 2) ok = mbar_wait(&S.k_empty[s], static_cast<uint32_t>((n / 2 - 1) & 1), &S.abort_flag);
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) S.abort_flag = 1;
       break;
     }
-    // the query copy (if any) and the key rows are in flight together; the tile is finished
-    // first, then the query
+    // the query copy (first chunk) and the key rows are in flight together; the tile is
+    // finished first, then the query
     uint8_t *kt = &S.k[s][0][0];
     // chunk exponent (every warp derives the same one) and the scales softmax reads
     const float smax = warp_max(fmaxf(S.mscale[ms][lane], S.mscale[ms][lane + 32]));
@@ -475,8 +435,8 @@ __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const long long *p
       mbar_arrive(&S.k_full[s]);
       mbar_arrive(&S.meta_empty[ms]);
     }
-    if (cp.first) {
-      query_finish(P, S, cp.b, seg & 1, gw, lane);
+    if (n == 0) {
+      query_finish(P, S, cr.b, gw, lane);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.q_full);
@@ -487,93 +447,79 @@ __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const long long *p
 
 // ---- warp 8, one thread: MMA1 S = Q K^T into TMEM lanes 16..31, MMA2 O += P K into lanes
 // 0..15 (all 512 columns; the same swizzled key tile read MN-major serves as V = K).
-__device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const long long *prefix, long long c0, long long c1,
-                         uint32_t tmem) {
+__device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const ChunkRange &cr, uint32_t tmem) {
   const bool f16 = fp16_operands(p);
   const uint32_t idesc1 = f16 ? idesc_f16(kH, kCh, 0, 0) : idesc_bf16(kH, kCh, 0, 0);
   const uint32_t idesc2 = f16 ? idesc_f16(kH, 256, 0, 1) : idesc_bf16(kH, 256, 0, 1);
   const uint32_t s_tmem = tmem + (16u << 16);
-  int seg = -1;
+  const uint64_t qd = sw128_desc(smem_u32(&S.q[0][0]), 16, 1024);
+  const uint64_t pd = sw128_desc(smem_u32(S.p), 16, 1024);
   long long n = 0;
-  for (long long g = c0; g < c1; ++g, ++n) {
+  for (long long g = cr.lo; g < cr.hi; ++g, ++n) {
     const int s = static_cast<int>(n & 1);
-    const ChunkPos cp = chunk_pos(prefix, p.B, g, c0, c1);
-    if (cp.first) {
-      ++seg;
-      if (!mbar_wait(&S.q_full, static_cast<uint32_t>(seg & 1), &S.abort_flag)) break;
-    }
+    if (n == 0 && !mbar_wait(&S.q_full, 0u, &S.abort_flag)) break;
     if (!mbar_wait(&S.k_full[s], static_cast<uint32_t>((n / 2) & 1), &S.abort_flag)) break;
     if (n >= 1 && !mbar_wait(&S.s_empty, static_cast<uint32_t>((n - 1) & 1), &S.abort_flag)) break;
     tc_fence_after();
-    const uint32_t qa = smem_u32(&S.q[0][0]), ka = smem_u32(&S.k[s][0][0]);
-#pragma unroll 4
-    for (int kk = 0; kk < kD / 16; ++kk) {
-      const uint32_t off = (kk >> 2) * (kH * 128) + (kk & 3) * 32;
-      const uint32_t offk = (kk >> 2) * kAtom + (kk & 3) * 32;
-      mma_bf16(s_tmem, sw128_desc(qa + off, 16, 1024), sw128_desc(ka + offk, 16, 1024), idesc1, kk > 0 ? 1u : 0u);
+    const uint32_t ka = smem_u32(&S.k[s][0][0]);
+    const uint64_t kd = sw128_desc(ka, 16, 1024);
+#pragma unroll
+    for (int kk = 0; kk < kD / 16; ++kk) {  // descriptor start advances in 16-byte units
+      const uint32_t off = ((kk >> 2) * (kH * 128) + (kk & 3) * 32) >> 4;
+      const uint32_t offk = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
+      mma_bf16(s_tmem, qd + off, kd + offk, idesc1, kk > 0 ? 1u : 0u);
     }
     mma_commit(&S.s_full);
-    if (cp.last) mma_commit(&S.q_empty);
     if (!mbar_wait(&S.p_full, static_cast<uint32_t>(n & 1), &S.abort_flag)) break;
-    if (cp.first && seg >= 1 && !mbar_wait(&S.o_empty, static_cast<uint32_t>((seg - 1) & 1), &S.abort_flag)) break;
     tc_fence_after();
-    const uint32_t pa = smem_u32(S.p);
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh)
 #pragma unroll
       for (int ks = 0; ks < kCh / 16; ++ks)
-        mma_bf16(tmem + nh * 256, sw128_desc(pa + ks * 32, 16, 1024),
-                 sw128_desc(ka + nh * 4 * kAtom + ks * 2048, kAtom, 1024), idesc2,
-                 (!cp.first || ks > 0) ? 1u : 0u);
+        mma_bf16(tmem + nh * 256, pd + ks * 2, sw128_desc(ka + nh * 4 * kAtom + ks * 2048, kAtom, 1024), idesc2,
+                 (n > 0 || ks > 0) ? 1u : 0u);
     mma_commit(&S.k_empty[s]);
     mma_commit(&S.o_full);
   }
-  // let the last MMAs finish before the CTA frees its TMEM
+  // let the last MMAs finish before anyone reads or frees the TMEM
   if (n > 0) {
     volatile int dummy = 0;
     mbar_wait(&S.o_full, static_cast<uint32_t>((n - 1) & 1), &dummy);
   }
 }
 
-// ---- warps 0-3 (quad = warp): online softmax and the partial output. Head h = 16 quad +
-// (lane & 15): its S row is TMEM lane 32 quad + 16 + (lane & 15); lanes 16..31 take keys
-// 0..31 of it, lanes 0..15 keys 32..63 (by shuffle), and both keep the head's running state.
-// Lanes 0..15 also own the head's O row (TMEM lane 32 quad + lane) for rescaling and output.
+// ---- warps 0-3 (quad = warp): online softmax. Head h = 16 quad + (lane & 15): its S row is
+// TMEM lane 32 quad + 16 + (lane & 15); lanes 16..31 take keys 0..31 of it, lanes 0..15
+// keys 32..63 (by shuffle), and both keep the head's running state. Lanes 0..15 also own the
+// head's O row (TMEM lane 32 quad + lane) for rescaling.
 // Online softmax in log2 units: with z_j = x_j + ec (x_j the logit of key j), the
 // accumulators hold O = sum_j 2^(z_j - R) * Krow_j and l = sum_j 2^(z_j - R) * 2^-ec, both
 // from the same rounded P, in units of 2^R; R is raised lazily (only when a chunk's max z
 // exceeds it by more than 8), so P stays <= 2^8 and O is rescaled rarely.
-__device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const long long *prefix, long long c0, long long c1,
-                             uint32_t tmem) {
+// Leaves (R, l) of each head in red_m / red_l.
+__device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &cr, uint32_t tmem) {
   const MqaLaunch &p = P.a;
   const int lane = threadIdx.x & 31, quad = (threadIdx.x >> 5) - kSoftWarp0;
   const int head = quad * 16 + (lane & 15);
-  const bool hi = lane >= 16;            // keys 0..31 (S row owner) vs keys 32..63
+  const bool hi = lane >= 16;  // keys 0..31 (S row owner) vs keys 32..63
   const int key0 = hi ? 0 : 32;
   const bool f16 = fp16_operands(p);
   const uint32_t lane_base = tmem + (static_cast<uint32_t>(quad * 32) << 16);
   float R = -INFINITY, l_half = 0.f;
-  int seg = -1;
   long long n = 0;
-  for (long long g = c0; g < c1; ++g, ++n) {
+  bool done = true;
+  for (long long g = cr.lo; g < cr.hi; ++g, ++n) {
     const int s = static_cast<int>(n & 1);
-    const ChunkPos cp = chunk_pos(prefix, p.B, g, c0, c1);
-    if (cp.first) {
-      ++seg;
-      R = -INFINITY;
-      l_half = 0.f;
-    }
     bool ok = mbar_wait(&S.k_full[s], static_cast<uint32_t>((n / 2) & 1), &S.abort_flag);
     ok = ok && mbar_wait(&S.s_full, static_cast<uint32_t>(n & 1), &S.abort_flag);
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) S.abort_flag = 1;
+      done = false;
       break;
     }
-    // read the query scale before releasing S: once S is free the query of a later segment
-    // (same parity) may be written
     const int ec = S.ec[s];
     // logit in log2 units of key j: acc * tau*log2(e) * qinv[h] * (fp8: 2^ec; bf16: 1)
-    const float coef = P.scale_log2 * S.qinv[seg & 1][head] * ldexpf(1.0f, ec);
+    const float coef = P.scale_log2 * S.qinv[head] * ldexpf(1.0f, ec);
     const float fec = static_cast<float>(ec);
     tc_fence_after();
     uint32_t r0[32], r1[32];
@@ -597,7 +543,7 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const long long *
     float Rn = R;
     if (mz > R + 8.f) Rn = mz;
     const float alpha = (Rn == R) ? 1.f : exp2f(R - Rn);  // R = -inf -> 0
-    const bool need_rescale = (Rn != R) && !cp.first;
+    const bool need_rescale = (Rn != R) && n > 0;
     const float lsc = ldexpf(1.0f, -ec);
     float lsum = 0.f;
     uint32_t pk[16];
@@ -625,6 +571,7 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const long long *
     ok = n == 0 || mbar_wait(&S.o_full, static_cast<uint32_t>((n - 1) & 1), &S.abort_flag);
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) S.abort_flag = 1;
+      done = false;
       break;
     }
     tc_fence_after();
@@ -650,50 +597,22 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const long long *
     fence_proxy_async_smem();
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.p_full);
-    if (cp.last) {
-      const float l = l_half + __shfl_xor_sync(0xFFFFFFFFu, l_half, 16);
-      ok = mbar_wait(&S.o_full, static_cast<uint32_t>(n & 1), &S.abort_flag);
-      if (!__all_sync(0xFFFFFFFFu, ok)) {
-        if (lane == 0) S.abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      const size_t slot = static_cast<size_t>(cp.b) + blockIdx.x;
-      if (hi) {
-        float *ml = P.part_ml + (slot * kH + head) * 2;
-        ml[0] = R;
-        ml[1] = l;
-      }
-      float *po = P.part_o + (slot * kH + head) * kD;
-#pragma unroll 1
-      for (int col = 0; col < kD; col += 128) {  // four loads in flight per wait
-        uint32_t o[4][32];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(lane_base + col + 32 * c, o[c]);
-        tmem_ld_wait();
-        if (!hi) {
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-#pragma unroll
-            for (int i = 0; i < 32; i += 4)
-              __stcg(reinterpret_cast<float4 *>(po + col + 32 * c + i),
-                     make_float4(__uint_as_float(o[c][i]), __uint_as_float(o[c][i + 1]), __uint_as_float(o[c][i + 2]),
-                                 __uint_as_float(o[c][i + 3])));
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&S.o_empty);
-    }
+  }
+  const float l = l_half + __shfl_xor_sync(0xFFFFFFFFu, l_half, 16);
+  if (hi) {
+    S.red_m[head] = done ? R : -INFINITY;
+    S.red_l[head] = done ? l : 0.f;
   }
 }
 
 __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_constant__ MqaTcParams P) {
   extern __shared__ uint8_t smem_raw[];
   MqaSmem &S = *reinterpret_cast<MqaSmem *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ float rcs[kD / 2], rsn[kD / 2];  // inverse-RoPE factors of this sequence
   const MqaLaunch &p = P.a;
-  long long *prefix = reinterpret_cast<long long *>(&S + 1);  // [B + 1] chunks before sequence b
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const uint32_t rank = cluster_rank(), cs = cluster_size();
+  const int b = blockIdx.y;
 
   if (tid == 0) {
     for (int i = 0; i < kMetaSlots; ++i) {
@@ -705,12 +624,10 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
       mbar_init(&S.k_empty[i], 1);
     }
     mbar_init(&S.q_full, 4);
-    mbar_init(&S.q_empty, 1);
     mbar_init(&S.s_full, 1);
     mbar_init(&S.s_empty, 4);
     mbar_init(&S.p_full, 4);
     mbar_init(&S.o_full, 1);
-    mbar_init(&S.o_empty, 4);
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -718,141 +635,136 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     tmem_alloc(&S.tmem_base, 512);
     tmem_relinquish();
   }
-  chunk_prefix(p, prefix, prefix + p.B + 1, blockIdx.x == 0);
-  pdl_wait();  // the selection (idx) and the caches come from the kernels before
+  const KeyList L = key_list(p, b, rank == 0 && tid == 0);
+  const int half = p.rope_dims / 2;
+  for (int i = tid; i < half; i += kThreads) rope_cos_sin(L.pos, i, p.rope_theta1, &rcs[i], &rsn[i]);
+  const long long C = (L.nw + L.nsel + kCh - 1) / kCh;  // the sequence's chunks
+  ChunkRange cr;
+  cr.b = b;
+  cr.lo = C * rank / cs;
+  cr.hi = C * (rank + 1) / cs;
+  pdl_wait();  // the selection (idx), the caches and the prepared query come from the kernels before
   pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
-  const long long T = prefix[p.B], G = gridDim.x;
-  const long long c0 = (T * blockIdx.x) / G, c1 = (T * (blockIdx.x + 1)) / G;
 
-  if (warp == kMetaWarp) meta_role(p, S, prefix, c0, c1);
-  else if (warp >= kGatherWarp0 && warp < kGatherWarp0 + 4) gather_role(P, S, prefix, c0, c1);
+  if (warp == kMetaWarp) meta_role(p, S, L, cr);
+  else if (warp >= kGatherWarp0 && warp < kGatherWarp0 + 4) gather_role(P, S, cr);
   else if (warp == kMmaWarp) {
-    if ((tid & 31) == 0) mma_role(p, S, prefix, c0, c1, tmem);
-  } else softmax_role(P, S, prefix, c0, c1, tmem);
+    if (lane == 0) mma_role(p, S, cr, tmem);
+  } else softmax_role(P, S, cr, tmem);
 
-  if (tid == 0 && S.abort_flag) report(p.d_status, DSV4_DEV_TIMEOUT);
+  // ---- merge of the cluster's partials: the weight of each CTA's (R, l) per head
   tc_fence_before();
   __syncthreads();
+  tc_fence_after();
+  cluster_sync_all();
+  if (tid < kH) {
+    float m[kMaxCluster], l[kMaxCluster];
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) {
+      m[r] = r < static_cast<int>(cs) ? ld_cluster_f32(cluster_addr(&S.red_m[tid], r)) : -INFINITY;
+      l[r] = r < static_cast<int>(cs) ? ld_cluster_f32(cluster_addr(&S.red_l[tid], r)) : 0.f;
+    }
+    float M = -INFINITY;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) M = fmaxf(M, m[r]);
+    float Ls = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxCluster; ++r) Ls += m[r] == -INFINITY ? 0.f : exp2f(m[r] - M) * l[r];
+    const float mine = S.red_m[tid];
+    S.wgt[tid] = mine == -INFINITY ? 0.f : exp2f(mine - M);
+    S.inv_l[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
+    S.lse[tid] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+  }
+  __syncthreads();
+  // this CTA's O times its weight into obuf (the key tiles are free): warp w reads TMEM
+  // lanes of quadrant w % 4, columns 256 (w / 4) .. +255
+  if (warp < 8) {
+    const int quad = warp & 3, h = quad * 16 + (lane & 15), col0 = (warp >> 2) * 256;
+    const bool has = cr.lo < cr.hi && !S.abort_flag;
+    const float w = S.wgt[h];
+#pragma unroll 1
+    for (int col = col0; col < col0 + 256; col += 64) {
+      uint32_t o[2][32];
+      if (has) {
+        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + col, o[0]);
+        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + col + 32, o[1]);
+        tmem_ld_wait();
+      }
+      if (lane < 16) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int i = 0; i < 32; i += 4) {
+            const int run = (col + 32 * c + i) >> 2;
+            const float4 v = has ? make_float4(__uint_as_float(o[c][i]) * w, __uint_as_float(o[c][i + 1]) * w,
+                                               __uint_as_float(o[c][i + 2]) * w, __uint_as_float(o[c][i + 3]) * w)
+                                 : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(&S.obuf[h][obuf_run(h, run) * 4]) = v;
+          }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  // CTA r finishes columns [r * Dc, (r + 1) * Dc): the sum over the cluster, / l, inverse
+  // RoPE, store
+  {
+    const int Dc = kD / static_cast<int>(cs), runs = Dc / 4, rope0 = kD - p.rope_dims;
+    for (int e = tid; e < kH * runs; e += kThreads) {
+      const int h = e / runs, d = static_cast<int>(rank) * Dc + (e % runs) * 4;
+      const uint32_t a = smem_u32(&S.obuf[h][obuf_run(h, d >> 2) * 4]);
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      float4 v[kMaxCluster];
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) {
+        if (r < static_cast<int>(cs)) {
+          uint32_t ra;
+          asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(r));
+          v[r] = ld_cluster_v4(ra);
+        }
+      }
+#pragma unroll
+      for (int r = 0; r < kMaxCluster; ++r) {
+        if (r < static_cast<int>(cs)) {
+          acc.x += v[r].x;
+          acc.y += v[r].y;
+          acc.z += v[r].z;
+          acc.w += v[r].w;
+        }
+      }
+      const float il = S.inv_l[h];
+      float y[4] = {acc.x * il, acc.y * il, acc.z * il, acc.w * il};
+#pragma unroll
+      for (int u = 0; u < 4; u += 2) {
+        if (d + u >= rope0) {  // rotate by -pos
+          const int pi = (d + u - rope0) >> 1;
+          const float c = rcs[pi], sv = rsn[pi];
+          const float y0 = y[u] * c + y[u + 1] * sv, y1 = -y[u] * sv + y[u + 1] * c;
+          y[u] = y0;
+          y[u + 1] = y1;
+        }
+      }
+      const size_t off = (static_cast<size_t>(b) * kH + h) * kD + d;
+      if (p.out_dt == DSV4_F32) {
+        *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off) = make_float4(y[0], y[1], y[2], y[3]);
+      } else {
+        *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.out) + off) =
+            make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
+      }
+    }
+    if (rank == 0 && p.lse && tid < kH) p.lse[static_cast<size_t>(b) * kH + tid] = S.lse[tid];
+  }
+  if (tid == 0 && S.abort_flag) report(p.d_status, DSV4_DEV_TIMEOUT);
+  cluster_sync_all();  // no CTA leaves while another may still read its shared memory
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
   }
-}
-
-// Merge the partials of every sequence, inverse RoPE, store. grid (B, H / 8), 256 threads:
-// warp w owns head h0 + w for the weights; for the sum every thread owns 4 float4 columns
-// of the CTA's 8 heads and keeps their loads of several partials in flight together.
-__global__ void __launch_bounds__(256) mqa_merge_kernel(const MqaTcParams P, int grid_ctas) {
-  const MqaLaunch &p = P.a;
-  __shared__ int warp_cnt[8];
-  __shared__ float cs[kD / 2], sn[kD / 2];
-  __shared__ float inv_l[8], lse_s[8];
-  extern __shared__ __align__(16) uint8_t dyn[];
-  float *wgt = reinterpret_cast<float *>(dyn);                                  // [grid][8] weight
-  float *lv = wgt + static_cast<size_t>(grid_ctas) * 8;                         // [grid][8] partial sum
-  int *cta = reinterpret_cast<int *>(lv + static_cast<size_t>(grid_ctas) * 8);  // [grid]
-  long long *prefix = reinterpret_cast<long long *>(cta + ((grid_ctas + 1) & ~1));  // [B + 1]
-  long long *red = prefix + p.B + 1;                                             // [blockDim]
-  const int b = blockIdx.x, h0 = blockIdx.y * 8, tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const KeyList L = key_list(p, b, false);
-  const int half = p.rope_dims / 2;
-  for (int i = tid; i < half; i += 256) rope_cos_sin(L.pos, i, p.rope_theta1, &cs[i], &sn[i]);
-  chunk_prefix(p, prefix, red, false);
-  // the CTAs of the main kernel whose (non-empty) chunk range meets this sequence, in
-  // order; with fewer chunks than CTAs some ranges are empty and those CTAs wrote nothing
-  const long long acc = prefix[p.B], mine = prefix[b], cnt = prefix[b + 1] - prefix[b];
-  int n = 0;
-  for (int c0 = 0; c0 < grid_ctas; c0 += 256) {
-    const int c = c0 + tid;
-    bool hit = false;
-    if (c < grid_ctas && cnt > 0) {
-      const long long a0 = (acc * c) / grid_ctas, a1 = (acc * (c + 1)) / grid_ctas;
-      hit = a0 < mine + cnt && a1 > mine && a1 > a0;
-    }
-    const unsigned bal = __ballot_sync(0xFFFFFFFFu, hit);
-    if (lane == 0) warp_cnt[warp] = __popc(bal);
-    __syncthreads();
-    int off = n;
-    for (int w = 0; w < warp; ++w) off += warp_cnt[w];
-    if (hit) cta[off + __popc(bal & ((1u << lane) - 1u))] = c;
-    for (int w = 0; w < 8; ++w) n += warp_cnt[w];
-    __syncthreads();
-  }
-  const int np = n;
-  pdl_wait();  // the partials come from the kernel before
-  pdl_launch_dependents();
-  for (int j = tid; j < np * 8; j += 256) {
-    const size_t slot = static_cast<size_t>(b) + cta[j >> 3];
-    const float2 ml = *reinterpret_cast<const float2 *>(P.part_ml + (slot * kH + h0 + (j & 7)) * 2);
-    wgt[j] = ml.x;
-    lv[j] = ml.y;
-  }
-  __syncthreads();
-  {  // weights of head h0 + warp: 2^(m_i - M), M the largest partial reference
-    float M = -INFINITY;
-    for (int i = lane; i < np; i += 32) M = fmaxf(M, wgt[i * 8 + warp]);
-    M = warp_max(M);
-    float Ls = 0.f;
-    for (int i = lane; i < np; i += 32) {
-      const float mi = wgt[i * 8 + warp];
-      const float w = (mi == -INFINITY) ? 0.f : exp2f(mi - M);
-      wgt[i * 8 + warp] = w;
-      Ls += w * lv[i * 8 + warp];
-    }
-    Ls = warp_sum(Ls);
-    if (lane == 0) {
-      inv_l[warp] = Ls > 0.f ? 1.f / Ls : 0.f;
-      lse_s[warp] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
-    }
-  }
-  __syncthreads();
-  constexpr int kPer = 8 * kD / 4 / 256;  // float4 columns per thread (4)
-  float4 o[kPer];
-#pragma unroll
-  for (int q = 0; q < kPer; ++q) o[q] = make_float4(0.f, 0.f, 0.f, 0.f);
-  for (int i = 0; i < np; ++i) {
-    const size_t slot = static_cast<size_t>(b) + cta[i];
-    const float *base = P.part_o + (slot * kH + h0) * kD;
-    float4 v[kPer];
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) v[q] = __ldcs(reinterpret_cast<const float4 *>(base) + q * 256 + tid);
-#pragma unroll
-    for (int q = 0; q < kPer; ++q) {
-      const float w = wgt[i * 8 + (q * 256 + tid) / (kD / 4)];
-      o[q].x = fmaf(w, v[q].x, o[q].x);
-      o[q].y = fmaf(w, v[q].y, o[q].y);
-      o[q].z = fmaf(w, v[q].z, o[q].z);
-      o[q].w = fmaf(w, v[q].w, o[q].w);
-    }
-  }
-  const int rope0 = kD - p.rope_dims;
-#pragma unroll
-  for (int q = 0; q < kPer; ++q) {
-    const int e = q * 256 + tid, hh = e / (kD / 4), d = (e % (kD / 4)) * 4, h = h0 + hh;
-    float y[4] = {o[q].x * inv_l[hh], o[q].y * inv_l[hh], o[q].z * inv_l[hh], o[q].w * inv_l[hh]};
-#pragma unroll
-    for (int u = 0; u < 4; u += 2) {
-      if (d + u >= rope0) {  // rotate by -pos
-        const int pi = (d + u - rope0) >> 1;
-        const float c = cs[pi], sv = sn[pi];
-        const float y0 = y[u] * c + y[u + 1] * sv, y1 = -y[u] * sv + y[u + 1] * c;
-        y[u] = y0;
-        y[u + 1] = y1;
-      }
-    }
-    const size_t off = (static_cast<size_t>(b) * kH + h) * kD + d;
-    if (p.out_dt == DSV4_F32) {
-      *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off) = make_float4(y[0], y[1], y[2], y[3]);
-    } else {
-      *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.out) + off) =
-          make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
-    }
-  }
-  if (p.lse && tid < 8) p.lse[static_cast<size_t>(b) * kH + h0 + tid] = lse_s[tid];
 }
 
 // ------------------------------------------------------------------------------------
@@ -961,8 +873,6 @@ __global__ void __launch_bounds__(256) mqa_simt_kernel(const MqaLaunch p, float 
     p.lse[static_cast<size_t>(b) * p.H + h] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
 }
 
-int tc_grid() { return sm_count(); }
-
 float softmax_scale_log2(const MqaLaunch &p) {
   const float s = p.softmax_scale > 0.f ? p.softmax_scale : 1.0f / sqrtf(static_cast<float>(p.D));
   return s * kLog2e;
@@ -977,10 +887,35 @@ bool mqa_uses_tensor_cores(const MqaLaunch &p) {
 
 size_t mqa_workspace_bytes(const MqaLaunch &p) {
   if (!mqa_uses_tensor_cores(p)) return 0;
-  const size_t slots = static_cast<size_t>(p.B) + tc_grid();
-  return align_up(slots * kH * kD * sizeof(float), 256) + align_up(slots * kH * 2 * sizeof(float), 256) +
-         align_up(static_cast<size_t>(p.B) * kH * kD * sizeof(uint16_t), 256) +
+  return align_up(static_cast<size_t>(p.B) * kH * kD * sizeof(uint16_t), 256) +
          align_up(static_cast<size_t>(p.B) * kH * sizeof(float), 256);
+}
+
+// CTAs per sequence: as many as keep the batch within one wave of SMs (a power of two, at
+// most 16, and at most 8 where the device cannot co-schedule 16 of these CTAs)
+int mqa_cluster(const MqaLaunch &p, size_t smem) {
+  int cs = 1;
+  while (cs < kMaxCluster && static_cast<long long>(cs) * 2 * p.B <= sm_count()) cs <<= 1;
+  if (cs > 8) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(cs);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess ||
+        cudaOccupancyMaxActiveClusters(&n, mqa_tc_kernel, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      cs = 8;
+    }
+  }
+  return cs;
 }
 
 cudaError_t launch_mqa(const MqaLaunch &p0, void *ws, cudaStream_t st) {
@@ -990,28 +925,18 @@ cudaError_t launch_mqa(const MqaLaunch &p0, void *ws, cudaStream_t st) {
     MqaTcParams P;
     P.a = p;
     P.scale_log2 = softmax_scale_log2(p);
-    const size_t slots = static_cast<size_t>(p.B) + tc_grid();
     char *w = static_cast<char *>(ws);
-    P.part_o = reinterpret_cast<float *>(w);
-    w += align_up(slots * kH * kD * sizeof(float), 256);
-    P.part_ml = reinterpret_cast<float *>(w);
-    w += align_up(slots * kH * 2 * sizeof(float), 256);
     P.qp = reinterpret_cast<uint16_t *>(w);
     w += align_up(static_cast<size_t>(p.B) * kH * kD * sizeof(uint16_t), 256);
     P.qinv = reinterpret_cast<float *>(w);
-    cudaError_t e = launch_pdl(mqa_query_kernel, dim3(p.B), dim3(256), 0, st, 1, P);
+    cudaError_t e = launch_pdl(mqa_query_kernel, dim3(p.B, kH / 16), dim3(256), 0, st, 1, P);
     if (e != cudaSuccess) return e;
-    const size_t smem = sizeof(MqaSmem) + 1024 + (static_cast<size_t>(p.B) + 1 + kThreads) * sizeof(long long);
+    const size_t smem = sizeof(MqaSmem) + 1024;
     e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    e = launch_pdl(mqa_tc_kernel, dim3(tc_grid()), dim3(kThreads), smem, st, 1, P);
-    if (e != cudaSuccess) return e;
-    const size_t msmem = static_cast<size_t>(tc_grid()) * 16 * sizeof(float) +
-                         static_cast<size_t>((tc_grid() + 1) & ~1) * sizeof(int) +
-                         (static_cast<size_t>(p.B) + 1 + 256) * sizeof(long long);
-    e = cudaFuncSetAttribute(mqa_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(mqa_merge_kernel, dim3(p.B, kH / 8), dim3(256), msmem, st, 1, P, tc_grid());
+    const int cs = mqa_cluster(p, smem);
+    return launch_pdl(mqa_tc_kernel, dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B)), dim3(kThreads),
+                      smem, st, cs, P);
   }
   const size_t smem = (2 * static_cast<size_t>(p.D) + 2 * kSimtChunk + 32) * sizeof(float) +
                       kSimtChunk * sizeof(void *) + 16;
