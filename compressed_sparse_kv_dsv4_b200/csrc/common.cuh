@@ -106,6 +106,14 @@ __device__ __forceinline__ void rope_cos_sin(int64_t pos, int pair, double theta
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// 2^x by the hardware approximation (one MUFU op; relative error ~2^-22, far below the
+// fp16/bf16 rounding the softmax weights receive next); 2^-inf = 0
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 // --------------------------------------------------------------------------------------
 // reductions
 
@@ -238,16 +246,23 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete. Returns false (and raises *abort)
-// if the wait exceeded kWaitLimitNs or another role already raised *abort.
+// if the wait exceeded kWaitLimitNs or another role already raised *abort. Between polls
+// the thread sleeps (32 ns, doubling to 128 ns), so a waiting warp leaves the issue slots
+// of its SM sub-partition to the warps doing work; the limit is checked every 16 polls.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
-  for (;;) {
+  uint32_t ns = 32;
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(ns);
+    if (ns < 128) ns <<= 1;
     if (mbar_try_wait(bar, parity)) return true;
-    if (*abort) return false;
-    if (globaltimer() - t0 > kWaitLimitNs) {
-      *abort = 1;
-      return false;
+    if ((i & 15) == 0) {
+      if (*abort) return false;
+      if (globaltimer() - t0 > kWaitLimitNs) {
+        *abort = 1;
+        return false;
+      }
     }
   }
 }

@@ -547,10 +547,11 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange 
     const float lsc = ldexpf(1.0f, -ec);
     float lsum = 0.f;
     uint32_t pk[16];
+    const float ref = Rn == -INFINITY ? 0.f : Rn;  // a chunk with no key at all: every z is -inf
 #pragma unroll
     for (int j = 0; j < 32; j += 2) {
-      const float e0 = z[j] == -INFINITY ? 0.f : exp2f(z[j] - Rn);
-      const float e1 = z[j + 1] == -INFINITY ? 0.f : exp2f(z[j + 1] - Rn);
+      const float e0 = ex2_approx(z[j] - ref);  // z = -inf gives 0
+      const float e1 = ex2_approx(z[j + 1] - ref);
       float a0, a1;
       if (f16) {
         __half2 h2 = __floats2half2_rn(e0, e1);
