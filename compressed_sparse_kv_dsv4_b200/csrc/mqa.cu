@@ -7,18 +7,21 @@
 // Keys of sequence s (V = K): window positions max(0,p-W+1)..p, then the selected entries
 // idx[s][0..k) (C4) or all visible entries (C128).
 //
-// Tensor-core path (bf16/fp8 caches, D = 512, H = 64): split-K over 64-key chunks of the
-// flattened (sequence, chunk) space, one persistent CTA per SM. Per chunk:
-//   gather: 64 key rows (16-byte loads; fp8 -> bf16 is exact) into a 128B-swizzled tile,
-//   MMA1:   S[64 heads x 64 keys] = Q K^T   (tcgen05 kind::f16, M = 64, accum at TMEM lane 16)
-//   softmax per head in one thread (the S row sits in that thread's TMEM lane), online
-//           with a lazy reference max (rescale only when the max grows by > 2^8),
-//           P' = exp2(x - m) * scale_j as bf16 (the fp8 row scale folded into P),
-//   MMA2:   O[64 x 512] += P' K               (M = 64, N = 256 x 2, K MN-major from the
-//           same swizzled tile, accum at TMEM lane 0, all 512 columns).
-// The gather of chunk i+1 overlaps MMA1 of chunk i. Each (CTA, sequence) segment writes
-// an unnormalized partial (O, m, l); a merge kernel combines partials with their
-// log-sum-exp weights, applies the inverse RoPE and stores the output.
+// Tensor-core path (bf16/fp8 caches, D = 512, H = 64):
+//   mqa_query_kernel: the query rotated by RoPE_pos once per sequence, as fp16 scaled per
+//     head by a power of two (fp8 caches) or bf16;
+//   mqa_tc_kernel: one thread-block cluster of cs CTAs per sequence, CTA r on a contiguous
+//     run of the sequence's 64-key chunks, with warp roles connected by mbarriers:
+//       metadata warp: row address + scale of every key (idx -> block table -> scale);
+//       gather warps:  64 rows into a 128B-swizzled K-major tile (fp8 -> fp16 exact, the
+//                      row scale folded in; bf16 copied), and the prepared query;
+//       MMA warp:      S[64 heads x 64 keys] = Q K^T (tcgen05 kind::f16, M = 64, TMEM lanes
+//                      16..31), then O[64 x 512] += P K (the same tile read MN-major, lanes 0..15);
+//       softmax warps: online softmax in log2 units with a lazy reference max, P to smem.
+//     At the end the cluster merges its partials in distributed shared memory: (max, sum)
+//     exchanged per head, each CTA's weighted O staged in its freed tile buffers, and CTA r
+//     summing, normalizing, inverse-rotating and storing columns [r * 512/cs, (r+1) * 512/cs).
+// CUDA-core path (any dtype, D <= 1024): mqa_simt_kernel, one CTA per (head, sequence).
 #include "common.cuh"
 #include "internal.h"
 
