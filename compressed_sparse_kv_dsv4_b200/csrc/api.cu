@@ -462,6 +462,7 @@ dsv4_status dsv4_hybrid_decode(const dsv4_layer *layer, const dsv4_step *step, v
   if (hp.c4) {
     int32_t *idx = step->topk_idx ? step->topk_idx : reinterpret_cast<int32_t *>(w);
     hp.ix.idx = idx;
+    hp.ix.after_append = true;  // the prologue appended at most each sequence's last entry
     e = launch_indexer_topk(hp.ix, w + hp.idx_bytes, st);
     if (e != cudaSuccess) return to_status(e);
     hp.mq.idx = idx;

@@ -139,6 +139,7 @@ struct TcParams {
   float *scores;  // [B][ld]; -inf where the entry has no valid page
   int64_t ld;
   uint32_t *d_status;
+  int after_append;  // wait for the kernel before only ahead of each sequence's last tile
 };
 
 // The tensor-core path serves C4 layers: 64 entries per page, a 128-entry tile = 2 pages,
@@ -269,7 +270,10 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
     }
     if (lane == 0) prefix[p.B] = carry;
   }
-  pdl_wait();  // keys, scales and the score buffer may be in use by the kernel before
+  // Keys and scales may be written by the kernel before. In general every read waits for
+  // it; after a decode-step append (which touches only each sequence's last entry) only
+  // the stages holding a sequence's last tile do (the producer waits ahead of them).
+  if (!p.after_append) pdl_wait();
   pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
@@ -318,6 +322,9 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
       }
       int ok = 1;
       if (lane == 0) {
+        // the stage holding a sequence's last tile waits for the kernel before (it may have
+        // just written that entry's key and scale)
+        if (p.after_append && seg_end && lt0 + nt == prefix[sb + 1] - prefix[sb]) pdl_wait();
         if (k >= kSlots && !mbar_wait(&S.sempty[slot], static_cast<uint32_t>((k / kSlots - 1) & 1), &S.abort_flag))
           ok = 0;
         if (ok) {  // key scales: one 256-byte bulk copy per valid page, zeros for the others
@@ -876,6 +883,7 @@ cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st) {
   tp.scores = scores;
   tp.ld = score_ld(p);
   tp.d_status = p.d_status;
+  tp.after_append = p.after_append ? 1 : 0;
   const size_t smem = sizeof(TcSmem<H>) + 1024 + (2 * static_cast<size_t>(p.B) + 1) * 8;
   cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

@@ -125,6 +125,10 @@ struct IndexerLaunch {
   int32_t *idx;
   float *scores;
   uint32_t *d_status;
+  // The kernel before it on the stream wrote at most the last visible entry of each
+  // sequence (the decode step's prologue): the other keys may be read before that kernel
+  // has finished.
+  bool after_append = false;
 };
 bool indexer_uses_tensor_cores(const IndexerLaunch &p);
 size_t indexer_workspace_bytes(const IndexerLaunch &p);
