@@ -147,14 +147,13 @@ struct TcParams {
 constexpr int kPerPage = 64;
 constexpr int kStageTiles = 2;
 constexpr int kStagePages = kStageTiles * kTile / kPerPage;  // 4
-constexpr int kStages = 5;       // key stages in flight (160 KB)
 constexpr int kSlots = 8;        // key-scale ring, one slot per stage
 constexpr int kBatchStages = 32 / kStagePages;  // stages whose page ids one warp load covers (8)
 constexpr int kGroups = 2;       // epilogue warp groups, alternating stages
 constexpr int kGroupThreads = 128;
 constexpr int kIxThreads = 64 + kGroups * kGroupThreads;
 
-template <int H>  // H in {32, 64}
+template <int H, int kStages>  // H in {32, 64}; kStages key stages of 32 KB in flight
 struct alignas(1024) TcSmem {
   uint8_t stage[kStages][kStageTiles][kTile * kRowBytes];  // key tiles (rows = entries)
   uint8_t q[2][H * kRowBytes];
@@ -227,10 +226,11 @@ __device__ __forceinline__ int load_page_batch(const TcParams &p, const long lon
                                            : -1;
 }
 
-template <int H>
+template <int H, int kStages>
 __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_constant__ TcParams p) {
   extern __shared__ uint8_t smem_raw[];
-  TcSmem<H> &S = *reinterpret_cast<TcSmem<H> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  TcSmem<H, kStages> &S =
+      *reinterpret_cast<TcSmem<H, kStages> *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   long long *prefix = reinterpret_cast<long long *>(&S + 1);       // [B + 1] tiles before sequence b
   int64_t *nvis = reinterpret_cast<int64_t *>(prefix + p.B + 1);  // [B] visible entries
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -502,7 +502,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
 
 constexpr int kTkThreads = 1024;
 constexpr int kTkWarps = kTkThreads / 32;
-constexpr int kTkSlice = 49152;  // largest slice per CTA (192 KB of keys)
+constexpr int kTkSlice = 24 * kTkThreads;  // largest slice of a cluster CTA: 24 keys per thread
+constexpr int kTkSolo = 16 * 1024;         // largest sequence one CTA takes alone (1024 threads x 16 keys)
 constexpr int kTkMaxCluster = 16;
 
 __device__ __forceinline__ uint32_t cluster_rank() {
@@ -533,15 +534,15 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
-__global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float *scores, int64_t ld,
+template <int KPT, int NT>  // NT threads of KPT keys each: a CTA holds up to NT * KPT keys, all in registers
+__global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores, int64_t ld,
                                                                    const int32_t *n_entries, const int32_t *pos,
                                                                    int m, int64_t capacity, int k, int slice,
                                                                    int32_t *idx, float *out_scores, uint32_t *d_status) {
-  extern __shared__ uint32_t keys[];  // [slice]
-  __shared__ int hist[2][256];        // this CTA's histogram of the current pass (double buffered)
-  __shared__ int ghist[256];          // the cluster's
-  __shared__ int xch[2];              // read by the other CTAs: class members, kept keys
-  __shared__ int warp_cnt[kTkWarps], warp_base[kTkWarps];
+  __shared__ int hist[2][256];  // this CTA's histogram of the current pass (double buffered)
+  __shared__ int ghist[256];    // the cluster's
+  __shared__ int xch[2];        // read by the other CTAs: class members, kept keys
+  __shared__ int warp_cnt[(NT / 32)], warp_base[(NT / 32)];
   __shared__ int sel_digit, sel_above, sel_count, bcast;
   const int b = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const uint32_t rank = cluster_rank(), cs = cluster_size();
@@ -550,32 +551,26 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
   const int cnt = static_cast<int>(n > lo ? (n - lo < slice ? n - lo : slice) : 0);
   pdl_wait();  // the scores come from the kernel before
   pdl_launch_dependents();
+  // warp w owns the contiguous run [w * 32 * KPT, (w + 1) * 32 * KPT) of the slice; its
+  // lane l holds key r at position w * 32 * KPT + 32 r + l (coalesced loads, and the rounds
+  // of the index-order walks below are the register index r)
+  const int wbase = warp * 32 * KPT;
   const float *src = scores + static_cast<size_t>(b) * ld + lo;
-  for (int i = tid * 4; i < cnt; i += kTkThreads * 4) {
-    float v[4];
-    if (i + 4 <= cnt) {
-      const float4 f = __ldcs(reinterpret_cast<const float4 *>(src + i));
-      v[0] = f.x; v[1] = f.y; v[2] = f.z; v[3] = f.w;
-    } else {
+  uint32_t key[KPT];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) v[u] = i + u < cnt ? src[i + u] : -INFINITY;
-    }
-#pragma unroll
-    for (int u = 0; u < 4; ++u) keys[i + u] = isfinite(v[u]) ? float_order_key(v[u]) : 0u;
+  for (int r = 0; r < KPT; ++r) {
+    const int i = wbase + 32 * r + lane;
+    const float v = i < cnt ? __ldcs(src + i) : -INFINITY;
+    key[r] = isfinite(v) ? float_order_key(v) : 0u;
   }
-  const int seg = (cnt + kTkWarps * 32 - 1) / (kTkWarps * 32) * 32;  // keys per warp, a multiple of 32
-  const int w0 = warp * seg, w1 = min(cnt, w0 + seg);
-  // one radix pass: the cluster histogram of digit `shift` over keys matching prefix/mask;
-  // returns (in sel_*) the digit holding the need-th largest key
   uint32_t prefix = 0, mask = 0;
   int need = 0, total_valid = 0, kk = 0;
-  auto pass = [&](int shift, int par) {
-    for (int i = tid; i < 256; i += kTkThreads) hist[par][i] = 0;
+  auto pass = [&](int shift, int par) {  // the cluster histogram of digit `shift` of the matching keys
+    for (int i = tid; i < 256; i += NT) hist[par][i] = 0;
     __syncthreads();
-    for (int i = tid; i < cnt; i += kTkThreads) {
-      const uint32_t key = keys[i];
-      if (key != 0u && (key & mask) == prefix) atomicAdd(&hist[par][(key >> shift) & 0xFF], 1);
-    }
+#pragma unroll
+    for (int r = 0; r < KPT; ++r)
+      if (key[r] != 0u && (key[r] & mask) == prefix) atomicAdd(&hist[par][(key[r] >> shift) & 0xFF], 1);
     cluster_sync_all();
     if (tid < 256) {  // all remote loads in flight before the first is used
       int v[kTkMaxCluster];
@@ -616,9 +611,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
   };
   // first pass: also counts the valid keys of the whole sequence
   pass(24, 0);
-  if (tid == 0) sel_count = -1;
-  __syncthreads();
-  pick(1 << 30);  // total in bcast; the digit choice is redone below once k is known
+  pick(1 << 30);  // the total, in bcast; the digit is chosen below once k is known
   total_valid = bcast;
   kk = total_valid < k ? total_valid : k;
   need = kk;
@@ -638,18 +631,19 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
       pick(need);
     }
   }
-  auto above = [&](uint32_t key) { return key != 0u && (!partial || (key & mask) > prefix); };
-  auto in_class = [&](uint32_t key) { return partial && key != 0u && (key & mask) == prefix; };
+  auto above = [&](uint32_t kv) { return kv != 0u && (!partial || (kv & mask) > prefix); };
+  auto in_class = [&](uint32_t kv) { return partial && kv != 0u && (kv & mask) == prefix; };
   // class members before this CTA and before each warp
   {
     int e = 0;
-    for (int i = w0 + lane; i < w1; i += 32) e += in_class(keys[i]);
+#pragma unroll
+    for (int r = 0; r < KPT; ++r) e += in_class(key[r]);
     e = warp_sum_int(e);
     if (lane == 0) warp_cnt[warp] = e;
     __syncthreads();
     if (tid == 0) {
       int run = 0;
-      for (int w = 0; w < kTkWarps; ++w) { warp_base[w] = run; run += warp_cnt[w]; }
+      for (int w = 0; w < (NT / 32); ++w) { warp_base[w] = run; run += warp_cnt[w]; }
       xch[0] = run;
     }
     cluster_sync_all();
@@ -662,34 +656,33 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
   }
   const int eq_before = bcast + warp_base[warp];
   __syncthreads();
-  // kept keys of each warp, then of the CTA, then the CTA's offset in the cluster
-  auto walk = [&](bool write, int out0) {
+  // kept keys of each warp in index order (round r, then lane): counted, then written
+  auto walk = [&](bool write, int at) {
     int e = eq_before, kept = 0;
-    for (int i0 = w0; i0 < w1; i0 += 32) {
-      const int i = i0 + lane;
-      const uint32_t key = i < w1 ? keys[i] : 0u;
-      const bool cl = in_class(key);
+#pragma unroll
+    for (int r = 0; r < KPT; ++r) {
+      const bool cl = in_class(key[r]);
       const unsigned clb = __ballot_sync(0xFFFFFFFFu, cl);
-      const bool keep = above(key) || (cl && e + __popc(clb & ((1u << lane) - 1u)) < need);
+      const bool keep = above(key[r]) || (cl && e + __popc(clb & ((1u << lane) - 1u)) < need);
       e += __popc(clb);
       const unsigned kb = __ballot_sync(0xFFFFFFFFu, keep);
       if (write && keep) {
-        const int at = out0 + kept + __popc(kb & ((1u << lane) - 1u));
-        if (at < k) {
-          idx[static_cast<size_t>(b) * k + at] = static_cast<int32_t>(lo + i);
-          if (out_scores) out_scores[static_cast<size_t>(b) * k + at] = order_key_to_float(key);
+        const int o = at + kept + __popc(kb & ((1u << lane) - 1u));
+        if (o < k) {
+          idx[static_cast<size_t>(b) * k + o] = static_cast<int32_t>(lo + wbase + 32 * r + lane);
+          if (out_scores) out_scores[static_cast<size_t>(b) * k + o] = order_key_to_float(key[r]);
         }
       }
       kept += __popc(kb);
     }
     return kept;
   };
-  const int my_kept = walk(false, 0);
-  if (lane == 0) warp_cnt[warp] = my_kept;
+  const int kept = walk(false, 0);
+  if (lane == 0) warp_cnt[warp] = kept;
   __syncthreads();
   if (tid == 0) {
     int run = 0;
-    for (int w = 0; w < kTkWarps; ++w) { warp_base[w] = run; run += warp_cnt[w]; }
+    for (int w = 0; w < (NT / 32); ++w) { warp_base[w] = run; run += warp_cnt[w]; }
     xch[1] = run;
   }
   cluster_sync_all();
@@ -704,7 +697,7 @@ __global__ void __launch_bounds__(kTkThreads, 1) topk_scores_kernel(const float 
   __syncthreads();
   walk(true, sel_above + warp_base[warp]);
   if (rank == 0) {
-    for (int i = sel_count + tid; i < k; i += kTkThreads) {
+    for (int i = sel_count + tid; i < k; i += NT) {
       idx[static_cast<size_t>(b) * k + i] = -1;
       if (out_scores) out_scores[static_cast<size_t>(b) * k + i] = -INFINITY;
     }
@@ -844,16 +837,17 @@ int64_t score_ld(const IndexerLaunch &p) { return (capacity_of(p) + 3) / 4 * 4; 
 
 // CTAs per sequence of the top-k cluster: enough for a slice to fit in shared memory, and
 // as many as keep the batch within one wave of SMs (a power of two, at most 16)
+// CTAs per sequence of the top-k: one while the sequence's entries fit in one CTA's
+// registers (no cluster barriers at all), else the smallest power-of-two cluster that fits
 int tk_cluster(const IndexerLaunch &p) {
+  if (capacity_of(p) <= kTkSolo) return 1;
   int need = 1;
   while (static_cast<int64_t>(need) * kTkSlice < capacity_of(p)) need <<= 1;
-  int par = 1;
-  while (par < 8 && static_cast<int64_t>(par) * 2 * p.B <= sm_count()) par <<= 1;
-  return need > par ? need : par;
+  return need;
 }
 int tk_slice(const IndexerLaunch &p) {
   const int cs = tk_cluster(p);
-  return static_cast<int>((capacity_of(p) + cs - 1) / cs + 3) / 4 * 4;
+  return static_cast<int>((capacity_of(p) + cs - 1) / cs);
 }
 
 // candidate list length per sequence (CUDA-core path: every entry)
@@ -884,10 +878,18 @@ cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st) {
   tp.ld = score_ld(p);
   tp.d_status = p.d_status;
   tp.after_append = p.after_append ? 1 : 0;
-  const size_t smem = sizeof(TcSmem<H>) + 1024 + (2 * static_cast<size_t>(p.B) + 1) * 8;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // six stages in flight where shared memory allows, else five
+  const size_t tail = 1024 + (2 * static_cast<size_t>(p.B) + 1) * 8;
+  if (sizeof(TcSmem<H, 6>) + tail <= 227 * 1024) {
+    const size_t smem = sizeof(TcSmem<H, 6>) + tail;
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(indexer_tc_kernel<H, 6>, dim3(tc_grid()), dim3(kIxThreads), smem, st, 1, tp);
+  }
+  const size_t smem = sizeof(TcSmem<H, 5>) + tail;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(indexer_tc_kernel<H>, dim3(tc_grid()), dim3(kIxThreads), smem, st, 1, tp);
+  return launch_pdl(indexer_tc_kernel<H, 5>, dim3(tc_grid()), dim3(kIxThreads), smem, st, 1, tp);
 }
 
 }  // namespace
@@ -920,16 +922,18 @@ cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t 
     e = p.H == 32 ? launch_tc<32>(p, scores, st) : launch_tc<64>(p, scores, st);
     if (e != cudaSuccess) return e;
     const int cs = tk_cluster(p), slice = tk_slice(p);
-    const size_t tsmem = static_cast<size_t>(slice) * sizeof(uint32_t);
-    e = cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem);
-    if (e != cudaSuccess) return e;
-    if (cs > 8) {
-      e = cudaFuncSetAttribute(topk_scores_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
-      if (e != cudaSuccess) return e;
-    }
-    return launch_pdl(topk_scores_kernel, dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B)),
-                      dim3(kTkThreads), tsmem, st, cs, static_cast<const float *>(scores), score_ld(p), p.n_entries,
-                      p.pos, p.m, capacity_of(p), p.k, slice, p.idx, p.scores, p.d_status);
+    auto launch_k = [&](auto kern, int nt) -> cudaError_t {
+      if (cs > 8) {
+        const cudaError_t a = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+        if (a != cudaSuccess) return a;
+      }
+      return launch_pdl(kern, dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B)), dim3(nt), 0, st, cs,
+                        static_cast<const float *>(scores), score_ld(p), p.n_entries, p.pos, p.m, capacity_of(p), p.k,
+                        slice, p.idx, p.scores, p.d_status);
+    };
+    if (slice <= 8 * kTkThreads) return launch_k(topk_scores_kernel<8, kTkThreads>, kTkThreads);
+    if (slice <= 16 * kTkThreads) return launch_k(topk_scores_kernel<16, kTkThreads>, kTkThreads);
+    return launch_k(topk_scores_kernel<24, kTkThreads>, kTkThreads);
   } else {
     e = cudaMemsetAsync(cand_count, 0, static_cast<size_t>(p.B) * sizeof(int), st);
     if (e != cudaSuccess) return e;
