@@ -540,6 +540,7 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
                                                                    int m, int64_t capacity, int k, int slice,
                                                                    int32_t *idx, float *out_scores, uint32_t *d_status) {
   __shared__ int hist[2][256];  // this CTA's histogram of the current pass (double buffered)
+  __shared__ int whist[NT / 32][256];  // first pass: one histogram per warp (no collisions between warps)
   __shared__ int ghist[256];    // the cluster's
   __shared__ int xch[2];        // read by the other CTAs: class members, kept keys
   __shared__ int warp_cnt[(NT / 32)], warp_base[(NT / 32)];
@@ -565,12 +566,28 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
   }
   uint32_t prefix = 0, mask = 0;
   int need = 0, total_valid = 0, kk = 0;
+  bool whole_class = true;  // every key of the k-th key's class is kept (no ranks needed)
   auto pass = [&](int shift, int par) {  // the cluster histogram of digit `shift` of the matching keys
-    for (int i = tid; i < 256; i += NT) hist[par][i] = 0;
-    __syncthreads();
+    if (shift == 24) {  // every key takes part: per-warp histograms, then summed
+      for (int i = lane; i < 256; i += 32) whist[warp][i] = 0;
+      __syncwarp();
 #pragma unroll
-    for (int r = 0; r < KPT; ++r)
-      if (key[r] != 0u && (key[r] & mask) == prefix) atomicAdd(&hist[par][(key[r] >> shift) & 0xFF], 1);
+      for (int r = 0; r < KPT; ++r)
+        if (key[r] != 0u) atomicAdd(&whist[warp][key[r] >> 24], 1);
+      __syncthreads();
+      for (int i = tid; i < 256; i += NT) {
+        int t = 0;
+#pragma unroll 8
+        for (int w = 0; w < NT / 32; ++w) t += whist[w][i];
+        hist[par][i] = t;
+      }
+    } else {
+      for (int i = tid; i < 256; i += NT) hist[par][i] = 0;
+      __syncthreads();
+#pragma unroll
+      for (int r = 0; r < KPT; ++r)
+        if (key[r] != 0u && (key[r] & mask) == prefix) atomicAdd(&hist[par][(key[r] >> shift) & 0xFF], 1);
+    }
     cluster_sync_all();
     if (tid < 256) {  // all remote loads in flight before the first is used
       int v[kTkMaxCluster];
@@ -625,7 +642,8 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
       need -= sel_above;
       const int cntd = sel_count;
       __syncthreads();
-      if (cntd == need || shift == 0) break;  // the whole class is taken, or the key is exact
+      whole_class = cntd == need;
+      if (whole_class || shift == 0) break;  // the whole class is taken, or the key is exact
       par ^= 1;
       pass(shift - 8, par);
       pick(need);
@@ -633,8 +651,8 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
   }
   auto above = [&](uint32_t kv) { return kv != 0u && (!partial || (kv & mask) > prefix); };
   auto in_class = [&](uint32_t kv) { return partial && kv != 0u && (kv & mask) == prefix; };
-  // class members before this CTA and before each warp
-  {
+  // class members before this CTA and before each warp (only needed when the class is split)
+  if (partial && !whole_class) {
     int e = 0;
 #pragma unroll
     for (int r = 0; r < KPT; ++r) e += in_class(key[r]);
@@ -654,7 +672,7 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
     }
     __syncthreads();
   }
-  const int eq_before = bcast + warp_base[warp];
+  const int eq_before = partial && !whole_class ? bcast + warp_base[warp] : 0;
   __syncthreads();
   // kept keys of each warp in index order (round r, then lane): counted, then written
   auto walk = [&](bool write, int at) {
@@ -662,9 +680,12 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
 #pragma unroll
     for (int r = 0; r < KPT; ++r) {
       const bool cl = in_class(key[r]);
-      const unsigned clb = __ballot_sync(0xFFFFFFFFu, cl);
-      const bool keep = above(key[r]) || (cl && e + __popc(clb & ((1u << lane) - 1u)) < need);
-      e += __popc(clb);
+      bool keep = above(key[r]) || (cl && whole_class);
+      if (!whole_class) {  // uniform: the class is split, members are ranked in index order
+        const unsigned clb = __ballot_sync(0xFFFFFFFFu, cl);
+        keep = keep || (cl && e + __popc(clb & ((1u << lane) - 1u)) < need);
+        e += __popc(clb);
+      }
       const unsigned kb = __ballot_sync(0xFFFFFFFFu, keep);
       if (write && keep) {
         const int o = at + kept + __popc(kb & ((1u << lane) - 1u));
