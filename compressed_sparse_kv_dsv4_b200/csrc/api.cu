@@ -457,17 +457,23 @@ dsv4_status dsv4_hybrid_decode(const dsv4_layer *layer, const dsv4_step *step, v
   if (need > 0 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))) return DSV4_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char *w = static_cast<char *>(ws);
+  // prologue -> query preparation -> (C4: indexer -> top-k) -> attention; the query kernel
+  // depends on no kernel of the step, so it runs beside the prologue and the indexer
+  void *mq_ws = w + hp.idx_bytes + hp.ix_bytes;
   cudaError_t e = launch_decode_prologue(hp.pro, st);
+  if (e != cudaSuccess) return to_status(e);
+  e = launch_mqa_query(hp.mq, mq_ws, st);
   if (e != cudaSuccess) return to_status(e);
   if (hp.c4) {
     int32_t *idx = step->topk_idx ? step->topk_idx : reinterpret_cast<int32_t *>(w);
     hp.ix.idx = idx;
     hp.ix.after_append = true;  // the prologue appended at most each sequence's last entry
+    hp.ix.release_next = true;  // the attention follows in this call
     e = launch_indexer_topk(hp.ix, w + hp.idx_bytes, st);
     if (e != cudaSuccess) return to_status(e);
     hp.mq.idx = idx;
   }
-  e = launch_mqa(hp.mq, w + hp.idx_bytes + hp.ix_bytes, st);
+  e = launch_mqa_attention(hp.mq, mq_ws, st);
   return to_status(e);
 }
 

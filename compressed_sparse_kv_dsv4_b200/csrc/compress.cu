@@ -196,8 +196,7 @@ __device__ __forceinline__ int64_t compress_items(const SeqRange &r, int m) {
 }
 
 __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressLaunch p) {
-  pdl_wait();
-  pdl_launch_dependents();
+  pdl_wait();  // the only kernel of its call: it releases nothing early
   extern __shared__ __align__(16) float smem[];
   float *scratch = smem;             // 3 * kMaxD
   float *e = smem + 3 * kMaxD;       // kMaxD
@@ -254,8 +253,7 @@ __global__ void __launch_bounds__(kThreads) compress_kernel(const CompressLaunch
 }
 
 __global__ void __launch_bounds__(kThreads) swa_insert_kernel(const SwaLaunch p) {
-  pdl_wait();
-  pdl_launch_dependents();
+  pdl_wait();  // the only kernel of its call: it releases nothing early
   __shared__ float e[kMaxD];
   __shared__ float red[32];
   const int s = blockIdx.y;

@@ -538,7 +538,8 @@ template <int KPT, int NT>  // NT threads of KPT keys each: a CTA holds up to NT
 __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores, int64_t ld,
                                                                    const int32_t *n_entries, const int32_t *pos,
                                                                    int m, int64_t capacity, int k, int slice,
-                                                                   int32_t *idx, float *out_scores, uint32_t *d_status) {
+                                                                   int32_t *idx, float *out_scores, uint32_t *d_status,
+                                                                   int release) {
   __shared__ int hist[2][256];  // this CTA's histogram of the current pass (double buffered)
   __shared__ int whist[NT / 32][256];  // first pass: one histogram per warp (no collisions between warps)
   __shared__ int ghist[256];    // the cluster's
@@ -551,7 +552,7 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
   const int64_t lo = static_cast<int64_t>(rank) * slice;
   const int cnt = static_cast<int>(n > lo ? (n - lo < slice ? n - lo : slice) : 0);
   pdl_wait();  // the scores come from the kernel before
-  pdl_launch_dependents();
+  if (release) pdl_launch_dependents();  // only when a kernel of the same call follows
   // warp w owns the contiguous run [w * 32 * KPT, (w + 1) * 32 * KPT) of the slice; its
   // lane l holds key r at position w * 32 * KPT + 32 r + l (coalesced loads, and the rounds
   // of the index-order walks below are the register index r)
@@ -732,9 +733,10 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
 
 __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const unsigned long long *cand, int64_t stride,
                                                                   const int *cand_count, int k, int32_t *idx,
-                                                                  float *scores, uint32_t *d_status, int smem_keys) {
+                                                                  float *scores, uint32_t *d_status, int smem_keys,
+                                                                  int release) {
   pdl_wait();
-  pdl_launch_dependents();
+  if (release) pdl_launch_dependents();  // only when a kernel of the same call follows
   extern __shared__ unsigned long long skeys[];  // [smem_keys] staged candidates, then [kp2] selected
   __shared__ int hist[256];
   __shared__ int sel_digit, sel_above, sel_count, kept;
@@ -864,6 +866,7 @@ int tk_cluster(const IndexerLaunch &p) {
   if (capacity_of(p) <= kTkSolo) return 1;
   int need = 1;
   while (static_cast<int64_t>(need) * kTkSlice < capacity_of(p)) need <<= 1;
+  while (need < 8 && static_cast<int64_t>(need) * 2 * p.B <= sm_count()) need <<= 1;  // more CTAs while they fit one wave
   return need;
 }
 int tk_slice(const IndexerLaunch &p) {
@@ -950,7 +953,7 @@ cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t 
       }
       return launch_pdl(kern, dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B)), dim3(nt), 0, st, cs,
                         static_cast<const float *>(scores), score_ld(p), p.n_entries, p.pos, p.m, capacity_of(p), p.k,
-                        slice, p.idx, p.scores, p.d_status);
+                        slice, p.idx, p.scores, p.d_status, p.release_next ? 1 : 0);
     };
     if (slice <= 8 * kTkThreads) return launch_k(topk_scores_kernel<8, kTkThreads>, kTkThreads);
     if (slice <= 16 * kTkThreads) return launch_k(topk_scores_kernel<16, kTkThreads>, kTkThreads);
@@ -973,7 +976,7 @@ cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t 
   if (e != cudaSuccess) return e;
   return launch_pdl(topk_select_kernel, dim3(p.B), dim3(kSelThreads), ssmem, st, 1,
                     static_cast<const unsigned long long *>(cand), stride, static_cast<const int *>(cand_count), p.k,
-                    p.idx, p.scores, p.d_status, smem_keys);
+                    p.idx, p.scores, p.d_status, smem_keys, p.release_next ? 1 : 0);
 }
 
 }  // namespace dsv4

@@ -129,6 +129,10 @@ struct IndexerLaunch {
   // sequence (the decode step's prologue): the other keys may be read before that kernel
   // has finished.
   bool after_append = false;
+  // Another kernel of the same call follows: the last kernel releases it early. When the
+  // indexer ends its call, its last kernel does not (the next call's kernels might read
+  // what it writes).
+  bool release_next = false;
 };
 bool indexer_uses_tensor_cores(const IndexerLaunch &p);
 size_t indexer_workspace_bytes(const IndexerLaunch &p);
@@ -163,6 +167,10 @@ struct MqaLaunch {
 bool mqa_uses_tensor_cores(const MqaLaunch &p);
 size_t mqa_workspace_bytes(const MqaLaunch &p);
 cudaError_t launch_mqa(const MqaLaunch &p, void *ws, cudaStream_t st);
+// the two halves of launch_mqa, for callers that schedule other kernels between them:
+// the query preparation (tensor-core path only) and the attention
+cudaError_t launch_mqa_query(const MqaLaunch &p, void *ws, cudaStream_t st);
+cudaError_t launch_mqa_attention(const MqaLaunch &p, void *ws, cudaStream_t st);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 

@@ -267,18 +267,19 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const KeyList &L, cons
 
 // ---- the query of every sequence, rotated by RoPE_pos once: bf16, or fp16 scaled per
 // head by a power of two (qinv undoes it in the logits) so that |q| < 2^14 whatever the
-// input range. grid (B, H / 16), 256 threads: thread t owns dims 32 (t & 15) .. +31 of head
-// 16 blockIdx.y + t / 16. It reads only the caller's query and writes only qp/qinv, which
-// nothing before it on the stream reads, so it runs before its pdl_wait(), beside the
-// kernel before it.
-__global__ void __launch_bounds__(256) mqa_query_kernel(const MqaTcParams P) {
+// input range. grid (B, H / 8), 128 threads (small enough to share an SM with the indexer):
+// thread t owns dims 32 (t & 15) .. +31 of head 8 blockIdx.y + t / 16. It reads only the
+// caller's query and writes only qp/qinv, which no kernel before it in the same call reads,
+// so it releases the next kernel at once and runs before its own pdl_wait().
+__global__ void __launch_bounds__(128) mqa_query_kernel(const MqaTcParams P) {
+  pdl_launch_dependents();
   const MqaLaunch &p = P.a;
   __shared__ float cs[kD / 2], sn[kD / 2];
-  const int b = blockIdx.x, t = threadIdx.x, h = blockIdx.y * 16 + (t >> 4), d0 = (t & 15) * 32;
+  const int b = blockIdx.x, t = threadIdx.x, h = blockIdx.y * 8 + (t >> 4), d0 = (t & 15) * 32;
   const bool f16 = fp16_operands(p);
   const int half = p.rope_dims / 2, rope0 = kD - p.rope_dims;
   const int64_t pos = p.pos[b];
-  for (int i = t; i < half; i += 256) rope_cos_sin(pos, i, p.rope_theta1, &cs[i], &sn[i]);
+  for (int i = t; i < half; i += 128) rope_cos_sin(pos, i, p.rope_theta1, &cs[i], &sn[i]);
   const uint4 *src = reinterpret_cast<const uint4 *>(static_cast<const uint16_t *>(p.q) +
                                                      (static_cast<size_t>(b) * kH + h) * kD + d0);
   uint4 raw[4];
@@ -324,8 +325,7 @@ __global__ void __launch_bounds__(256) mqa_query_kernel(const MqaTcParams P) {
                  : make_uint4(pack_bf16x2(x[i][0], x[i][1]), pack_bf16x2(x[i][2], x[i][3]),
                               pack_bf16x2(x[i][4], x[i][5]), pack_bf16x2(x[i][6], x[i][7]));
   if ((t & 15) == 0) P.qinv[static_cast<size_t>(b) * kH + h] = qi;
-  pdl_wait();
-  pdl_launch_dependents();
+  pdl_wait();  // completes only after the kernel before it: the chain of waits stays unbroken
 }
 
 // ---- warps 4-7 (gw = 0..3): query of a new segment and the key tiles. Query: warp gw
@@ -648,7 +648,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
   cr.lo = C * rank / cs;
   cr.hi = C * (rank + 1) / cs;
   pdl_wait();  // the selection (idx), the caches and the prepared query come from the kernels before
-  pdl_launch_dependents();
+  // (the last kernel of its call: it does not release the next call's kernels early)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -779,7 +779,6 @@ constexpr int kSimtChunk = 256;
 
 __global__ void __launch_bounds__(256) mqa_simt_kernel(const MqaLaunch p, float scale_log2) {
   pdl_wait();
-  pdl_launch_dependents();
   extern __shared__ float sm[];
   float *qr = sm;                      // [D]
   float *xs = qr + p.D;                // [chunk]
@@ -897,7 +896,7 @@ size_t mqa_workspace_bytes(const MqaLaunch &p) {
 
 // CTAs per sequence: as many as keep the batch within one wave of SMs (a power of two, at
 // most 16, and at most 8 where the device cannot co-schedule 16 of these CTAs)
-int mqa_cluster(const MqaLaunch &p, size_t smem) {
+static int mqa_cluster(const MqaLaunch &p, size_t smem) {
   int cs = 1;
   while (cs < kMaxCluster && static_cast<long long>(cs) * 2 * p.B <= sm_count()) cs <<= 1;
   if (cs > 8) {
@@ -922,21 +921,30 @@ int mqa_cluster(const MqaLaunch &p, size_t smem) {
   return cs;
 }
 
-cudaError_t launch_mqa(const MqaLaunch &p0, void *ws, cudaStream_t st) {
+static MqaTcParams tc_params(const MqaLaunch &p0, void *ws) {
+  MqaTcParams P;
+  P.a = p0;
+  P.a.rope_theta1 = rope_theta1(p0.rope_base, p0.rope_dims);
+  P.scale_log2 = softmax_scale_log2(P.a);
+  char *w = static_cast<char *>(ws);
+  P.qp = reinterpret_cast<uint16_t *>(w);
+  w += align_up(static_cast<size_t>(p0.B) * kH * kD * sizeof(uint16_t), 256);
+  P.qinv = reinterpret_cast<float *>(w);
+  return P;
+}
+
+cudaError_t launch_mqa_query(const MqaLaunch &p, void *ws, cudaStream_t st) {
+  if (!mqa_uses_tensor_cores(p)) return cudaSuccess;
+  return launch_pdl(mqa_query_kernel, dim3(p.B, kH / 8), dim3(128), 0, st, 1, tc_params(p, ws));
+}
+
+cudaError_t launch_mqa_attention(const MqaLaunch &p0, void *ws, cudaStream_t st) {
   MqaLaunch p = p0;
   p.rope_theta1 = rope_theta1(p.rope_base, p.rope_dims);
   if (mqa_uses_tensor_cores(p)) {
-    MqaTcParams P;
-    P.a = p;
-    P.scale_log2 = softmax_scale_log2(p);
-    char *w = static_cast<char *>(ws);
-    P.qp = reinterpret_cast<uint16_t *>(w);
-    w += align_up(static_cast<size_t>(p.B) * kH * kD * sizeof(uint16_t), 256);
-    P.qinv = reinterpret_cast<float *>(w);
-    cudaError_t e = launch_pdl(mqa_query_kernel, dim3(p.B, kH / 16), dim3(256), 0, st, 1, P);
-    if (e != cudaSuccess) return e;
+    const MqaTcParams P = tc_params(p0, ws);
     const size_t smem = sizeof(MqaSmem) + 1024;
-    e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = cudaFuncSetAttribute(mqa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     const int cs = mqa_cluster(p, smem);
     return launch_pdl(mqa_tc_kernel, dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B)), dim3(kThreads),
@@ -947,6 +955,12 @@ cudaError_t launch_mqa(const MqaLaunch &p0, void *ws, cudaStream_t st) {
   cudaError_t e = cudaFuncSetAttribute(mqa_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(mqa_simt_kernel, dim3(p.H, p.B), dim3(256), smem, st, 1, p, softmax_scale_log2(p));
+}
+
+cudaError_t launch_mqa(const MqaLaunch &p, void *ws, cudaStream_t st) {
+  const cudaError_t e = launch_mqa_query(p, ws, st);
+  if (e != cudaSuccess) return e;
+  return launch_mqa_attention(p, ws, st);
 }
 
 }  // namespace dsv4
