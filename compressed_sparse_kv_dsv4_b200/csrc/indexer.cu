@@ -501,7 +501,6 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
 // output is in ascending entry order and does not depend on thread timing.
 
 constexpr int kTkThreads = 1024;
-constexpr int kTkWarps = kTkThreads / 32;
 constexpr int kTkSlice = 24 * kTkThreads;  // largest slice of a cluster CTA: 24 keys per thread
 constexpr int kTkSolo = 16 * 1024;         // largest sequence one CTA takes alone (1024 threads x 16 keys)
 constexpr int kTkMaxCluster = 16;

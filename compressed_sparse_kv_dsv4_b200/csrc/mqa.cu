@@ -18,9 +18,12 @@
 //       MMA warp:      S[64 heads x 64 keys] = Q K^T (tcgen05 kind::f16, M = 64, TMEM lanes
 //                      16..31), then O[64 x 512] += P K (the same tile read MN-major, lanes 0..15);
 //       softmax warps: online softmax in log2 units with a lazy reference max, P to smem.
-//     At the end the cluster merges its partials in distributed shared memory: (max, sum)
-//     exchanged per head, each CTA's weighted O staged in its freed tile buffers, and CTA r
-//     summing, normalizing, inverse-rotating and storing columns [r * 512/cs, (r+1) * 512/cs).
+//     The MMA warp issues S of chunk n + 1 (two S buffers in TMEM) while the softmax warps
+//     work on chunk n. At the end the cluster merges its partials: (max, sum) exchanged
+//     per head and each CTA's O staged per owner in its freed tile buffers, both passed
+//     through global memory (L2 moves them several times faster than the cluster's
+//     shared-memory network); CTA r weighs and sums its slabs, normalizes, inverse-rotates
+//     and stores columns [r * 512/cs, (r+1) * 512/cs).
 // CUDA-core path (any dtype, D <= 1024): mqa_simt_kernel, one CTA per (head, sequence).
 #include "common.cuh"
 #include "internal.h"
@@ -111,7 +114,7 @@ struct alignas(1024) MqaSmem {
   uint8_t q[kD / 64][kH * 128];  // 64 KB, K-major SW128, 8 atoms of 64 dims
   union {
     uint8_t k[2][kD / 64][kCh * 128];  // 2 x 64 KB key tiles (stage = chunk parity)
-    float obuf[kH][kD];                // after the last MMA: this CTA's weighted O (swizzled runs)
+    float rbuf[kH * kD];               // after the last MMA: this CTA's weighted O, one slab per owner
   };
   uint8_t p[kH * 128];                   // 8 KB: P[64 heads][64 keys], K-major SW128
   const uint8_t *mrow[kMetaSlots][kCh];  // row address of each key of a chunk (nullptr: none)
@@ -120,18 +123,23 @@ struct alignas(1024) MqaSmem {
   int ec[2];                             // tile exponent: K rows hold code * scale * 2^-ec
   float qinv[kH];                        // 2^-e of the per-head query scale
   float red_m[kH], red_l[kH];            // this CTA's reference max and sum per head (read by the cluster)
-  float wgt[kH], inv_l[kH], lse[kH];     // its weight in the merge, 1 / total sum, log-sum-exp
+  float inv_l[kH], lse[kH];              // 1 / the cluster's total sum, log-sum-exp, per head
+  float wsrc[kMaxCluster][kH];           // weight 2^(R - M) of each cluster CTA's partial, per head
   uint64_t meta_full[kMetaSlots], meta_empty[kMetaSlots];
-  uint64_t k_full[2], k_empty[2], q_full, s_full, s_empty, p_full, o_full;
+  uint64_t k_full[2], k_empty[2], q_full, s_full[2], s_empty[2], p_full, o_full, mma_done, part_full;
   uint32_t tmem_base;
   int abort_flag;
 };
+
+static_assert(sizeof(MqaSmem) + 1024 <= 227 * 1024, "attention shared memory exceeds one SM");
 
 struct MqaTcParams {
   MqaLaunch a;
   float scale_log2;
   uint16_t *qp;    // [B][H][D] query rotated by RoPE_pos, fp16 (scaled per head) or bf16
   float *qinv;     // [B][H] 2^-e undoing the per-head scale (1 for bf16)
+  float *part;     // [B][cs][cs - 1] slabs [H][D / cs]: CTA src's O for owner dst != src
+  float *red;      // [B][cs][2][H]: each CTA's reference max R and sum l per head
 };
 
 // Operands of the two MMAs. fp8 caches: fp16 (e4m3 -> fp16 is exact, and fp16 keeps 11
@@ -153,29 +161,13 @@ __device__ __forceinline__ uint32_t cluster_size() {
   asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(r));
   return r;
 }
-// every thread of every CTA of the cluster; orders shared-memory writes before it with reads after it
+// every thread of every CTA of the cluster; orders the memory writes before it with the reads after it
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-// address of the same shared variable in CTA `rank` of this cluster
-__device__ __forceinline__ uint32_t cluster_addr(const void *p, uint32_t rank) {
-  uint32_t ra;
-  asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(smem_u32(p)), "r"(rank));
-  return ra;
-}
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr));
-  return v;
-}
-__device__ __forceinline__ float4 ld_cluster_v4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr));
-  return v;
-}
-// 16-byte run c of row h of obuf: runs are XOR-swizzled by h so that the 16 rows a warp
+// 16-byte run c of row h of a merge slab: runs are XOR-swizzled by h so that the 16 rows a warp
 // writes at once land in different banks
-__device__ __forceinline__ int obuf_run(int h, int c) { return c ^ (h & 7); }
+__device__ __forceinline__ int slab_run(int h, int c) { return c ^ (h & 7); }
 
 // This CTA's chunks of its sequence: [lo, hi) of the sequence's C chunks.
 struct ChunkRange {
@@ -204,60 +196,62 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const KeyList &L, cons
       if (lane == 0) S.abort_flag = 1;
       return;
     }
-    int64_t j[kKeys];  // >= 0: entry index; -1: none; -2 - slot: window ring slot
-    int32_t page[kKeys];
+    // Three stages, each with the loads of all kKeys keys issued together: every load reads
+    // a clamped, always-valid address and the result is selected afterwards, so no branch
+    // separates them. kind: 0 none, 1 window row, 2 selected entry.
+    int kind[kKeys];
+    int64_t t_u[kKeys], j[kKeys];
 #pragma unroll
-    for (int u = 0; u < kKeys; ++u) {  // stage 1: key list position -> entry index (idx load)
+    for (int u = 0; u < kKeys; ++u) {
       const int i = u >> 1;
-      j[u] = -1;
-      if (i < nb) {
-        const int64_t t = (g0 + i) * kCh + lane + 32 * (u & 1);
-        if (t < L.nw) {
-          const int64_t pw = L.pos - L.nw + 1 + t;
-          j[u] = -2 - (static_cast<int64_t>(b) * p.W + pw % p.W);
-        } else if (t - L.nw < L.nsel) {
-          const int64_t uu = t - L.nw;
-          int64_t e = uu;
-          if (p.idx) {
-            e = p.idx[static_cast<size_t>(b) * p.k + uu];
-            if (e >= L.n_entries) {
-              report(p.d_status, DSV4_DEV_BAD_INDEX);
-              e = -1;
-            }
-          }
-          j[u] = e < 0 ? -1 : e;
-        }
-      }
+      t_u[u] = (g0 + i) * kCh + lane + 32 * (u & 1);
+      kind[u] = i >= nb ? 0 : (t_u[u] < L.nw ? 1 : (t_u[u] - L.nw < L.nsel ? 2 : 0));
     }
 #pragma unroll
+    for (int u = 0; u < kKeys; ++u) {  // stage 1: list position -> entry index (idx load)
+      const int64_t uu = kind[u] == 2 ? t_u[u] - L.nw : 0;
+      j[u] = uu;
+      if (p.idx) j[u] = p.idx[static_cast<size_t>(b) * p.k + uu];
+    }
+    int32_t page[kKeys];
+#pragma unroll
     for (int u = 0; u < kKeys; ++u) {  // stage 2: entry -> physical page (block table load)
-      page[u] = -1;
-      if (j[u] >= 0) {
-        page[u] = p.block_table[static_cast<size_t>(b) * p.max_blocks + j[u] / per_page];
-        if (page[u] < 0 || page[u] >= p.num_pages) {
-          report(p.d_status, DSV4_DEV_BAD_PAGE);
-          page[u] = -1;
-        }
+      bool ok = kind[u] == 2 && j[u] >= 0;
+      if (ok && j[u] >= L.n_entries) {
+        report(p.d_status, DSV4_DEV_BAD_INDEX);
+        ok = false;
       }
+      if (!ok && kind[u] == 2) kind[u] = 0;  // padding or a bad index: no key
+      page[u] = p.block_table[static_cast<size_t>(b) * p.max_blocks + (ok ? j[u] / per_page : 0)];
     }
 #pragma unroll
     for (int u = 0; u < kKeys; ++u) {  // stage 3: row address and scale
       const int i = u >> 1;
-      if (i >= nb) continue;
-      const uint8_t *rp = nullptr;
-      float sc = 0.f;
-      if (j[u] <= -2) {
-        const size_t slot = static_cast<size_t>(-2 - j[u]);
-        rp = static_cast<const uint8_t *>(p.ring_rows) + slot * p.D * esz;
-        sc = p.kv_dt == DSV4_FP8E4M3 ? p.ring_scales[slot] : 1.0f;
-      } else if (page[u] >= 0) {
-        const size_t row = static_cast<size_t>(page[u]) * per_page + static_cast<size_t>(j[u] % per_page);
-        rp = static_cast<const uint8_t *>(p.pages) + row * p.D * esz;
-        sc = p.kv_dt == DSV4_FP8E4M3 ? p.scales[row] : 1.0f;
+      size_t slot_or_row = 0;
+      if (kind[u] == 1) {
+        const int64_t pw = L.pos - L.nw + 1 + t_u[u];
+        slot_or_row = static_cast<size_t>(b) * p.W + static_cast<size_t>(pw % p.W);
+      } else if (kind[u] == 2) {
+        if (page[u] < 0 || page[u] >= p.num_pages) {
+          report(p.d_status, DSV4_DEV_BAD_PAGE);
+          kind[u] = 0;
+        } else {
+          slot_or_row = static_cast<size_t>(page[u]) * per_page + static_cast<size_t>(j[u] % per_page);
+        }
       }
-      const int slot = static_cast<int>((g0 + i - cr.lo) % kMetaSlots);
-      S.mrow[slot][lane + 32 * (u & 1)] = rp;
-      S.mscale[slot][lane + 32 * (u & 1)] = rp ? sc : 0.f;
+      float sc = 1.0f;
+      if (p.kv_dt == DSV4_FP8E4M3) sc = (kind[u] == 1 ? p.ring_scales : p.scales)[kind[u] == 0 ? 0 : slot_or_row];
+      const uint8_t *rp = kind[u] == 0 ? nullptr
+                                       : static_cast<const uint8_t *>(kind[u] == 1 ? p.ring_rows : p.pages) +
+                                             slot_or_row * p.D * esz;
+      if (i < nb) {
+        const int slot = static_cast<int>((g0 + i - cr.lo) % kMetaSlots);
+        S.mrow[slot][lane + 32 * (u & 1)] = rp;
+        S.mscale[slot][lane + 32 * (u & 1)] = rp ? sc : 0.f;
+        // the gather of this CTA's third and later chunks waits for a free tile stage: their
+        // rows travel to L2 meanwhile
+        if (rp && g0 + i - cr.lo >= 2) bulk_prefetch_l2(rp, static_cast<uint32_t>(p.D * esz));
+      }
     }
     __syncwarp();
     if (lane == 0)
@@ -448,8 +442,11 @@ __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &
   cp_async_wait_all();
 }
 
-// ---- warp 8, one thread: MMA1 S = Q K^T into TMEM lanes 16..31, MMA2 O += P K into lanes
-// 0..15 (all 512 columns; the same swizzled key tile read MN-major serves as V = K).
+// ---- warp 8, one thread: MMA1 S = Q K^T into TMEM lanes 16..31 (columns 64 (n & 1) ..
+// +63: two S buffers), MMA2 O += P K into lanes 0..15 (all 512 columns; the same swizzled key
+// tile read MN-major serves as V = K). MMA1 of chunk n + 1 goes out as soon as its tile and
+// its S buffer are ready, ahead of MMA2 of chunk n when P of chunk n is not yet written, so
+// the softmax of chunk n overlaps the tensor-core work of chunk n + 1.
 __device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const ChunkRange &cr, uint32_t tmem) {
   const bool f16 = fp16_operands(p);
   const uint32_t idesc1 = f16 ? idesc_f16(kH, kCh, 0, 0) : idesc_bf16(kH, kCh, 0, 0);
@@ -457,37 +454,64 @@ __device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const ChunkRange &cr, u
   const uint32_t s_tmem = tmem + (16u << 16);
   const uint64_t qd = sw128_desc(smem_u32(&S.q[0][0]), 16, 1024);
   const uint64_t pd = sw128_desc(smem_u32(S.p), 16, 1024);
-  long long n = 0;
-  for (long long g = cr.lo; g < cr.hi; ++g, ++n) {
-    const int s = static_cast<int>(n & 1);
-    if (n == 0 && !mbar_wait(&S.q_full, 0u, &S.abort_flag)) break;
-    if (!mbar_wait(&S.k_full[s], static_cast<uint32_t>((n / 2) & 1), &S.abort_flag)) break;
-    if (n >= 1 && !mbar_wait(&S.s_empty, static_cast<uint32_t>((n - 1) & 1), &S.abort_flag)) break;
+  const long long nc = cr.hi - cr.lo;
+  // chunk m may take MMA1 once the query (chunk 0) and its tile are staged and the softmax
+  // has read S of chunk m - 2
+  auto s_ready = [&](long long m) {
+    return (m > 0 || mbar_try_wait(&S.q_full, 0u)) &&
+           mbar_try_wait(&S.k_full[m & 1], static_cast<uint32_t>((m >> 1) & 1)) &&
+           (m < 2 || mbar_try_wait(&S.s_empty[m & 1], static_cast<uint32_t>(((m - 2) >> 1) & 1)));
+  };
+  auto issue_s = [&](long long m) {
     tc_fence_after();
-    const uint32_t ka = smem_u32(&S.k[s][0][0]);
-    const uint64_t kd = sw128_desc(ka, 16, 1024);
+    const uint64_t kd = sw128_desc(smem_u32(&S.k[m & 1][0][0]), 16, 1024);
+    const uint32_t dt = s_tmem + 64u * static_cast<uint32_t>(m & 1);
 #pragma unroll
     for (int kk = 0; kk < kD / 16; ++kk) {  // descriptor start advances in 16-byte units
       const uint32_t off = ((kk >> 2) * (kH * 128) + (kk & 3) * 32) >> 4;
       const uint32_t offk = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
-      mma_bf16(s_tmem, qd + off, kd + offk, idesc1, kk > 0 ? 1u : 0u);
+      mma_bf16(dt, qd + off, kd + offk, idesc1, kk > 0 ? 1u : 0u);
     }
-    mma_commit(&S.s_full);
-    if (!mbar_wait(&S.p_full, static_cast<uint32_t>(n & 1), &S.abort_flag)) break;
+    mma_commit(&S.s_full[m & 1]);
+  };
+  long long next = 0;  // the next chunk to take MMA1
+  bool ok = true;
+  for (long long n = 0; ok && n < nc; ++n) {
+    // P of chunk n (which needs MMA1 of chunk n); meanwhile MMA1 of chunks n and n + 1 as
+    // soon as they can go
+    const uint64_t t0 = globaltimer();
+    uint32_t ns = 32;
+    for (uint32_t i = 1;; ++i) {
+      if (next <= n + 1 && next < nc && s_ready(next)) {
+        issue_s(next++);
+        continue;
+      }
+      if (mbar_try_wait(&S.p_full, static_cast<uint32_t>(n & 1))) break;
+      __nanosleep(ns);
+      if (ns < 128) ns <<= 1;
+      if ((i & 15) == 0 && (S.abort_flag || globaltimer() - t0 > kWaitLimitNs)) {
+        S.abort_flag = 1;
+        ok = false;
+        break;
+      }
+    }
+    if (!ok) break;
     tc_fence_after();
+    const uint32_t ka = smem_u32(&S.k[n & 1][0][0]);
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh)
 #pragma unroll
       for (int ks = 0; ks < kCh / 16; ++ks)
         mma_bf16(tmem + nh * 256, pd + ks * 2, sw128_desc(ka + nh * 4 * kAtom + ks * 2048, kAtom, 1024), idesc2,
                  (n > 0 || ks > 0) ? 1u : 0u);
-    mma_commit(&S.k_empty[s]);
+    mma_commit(&S.k_empty[n & 1]);
     mma_commit(&S.o_full);
   }
-  // let the last MMAs finish before anyone reads or frees the TMEM
-  if (n > 0) {
+  // let every MMA issued here finish (also after an abort) before anyone reads or frees the TMEM
+  if (next > 0) {
+    mma_commit(&S.mma_done);
     volatile int dummy = 0;
-    mbar_wait(&S.o_full, static_cast<uint32_t>((n - 1) & 1), &dummy);
+    mbar_wait(&S.mma_done, 0u, &dummy);
   }
 }
 
@@ -514,7 +538,7 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange 
   for (long long g = cr.lo; g < cr.hi; ++g, ++n) {
     const int s = static_cast<int>(n & 1);
     bool ok = mbar_wait(&S.k_full[s], static_cast<uint32_t>((n / 2) & 1), &S.abort_flag);
-    ok = ok && mbar_wait(&S.s_full, static_cast<uint32_t>(n & 1), &S.abort_flag);
+    ok = ok && mbar_wait(&S.s_full[s], static_cast<uint32_t>((n >> 1) & 1), &S.abort_flag);
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) S.abort_flag = 1;
       done = false;
@@ -525,13 +549,13 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange 
     const float coef = P.scale_log2 * S.qinv[head] * ldexpf(1.0f, ec);
     const float fec = static_cast<float>(ec);
     tc_fence_after();
-    uint32_t r0[32], r1[32];
-    tmem_ld32(lane_base + 0, r0);
-    tmem_ld32(lane_base + 32, r1);
+    uint32_t r0[32], r1[32];  // (lanes 0..15 read O columns here and discard them)
+    tmem_ld32(lane_base + 64 * s, r0);
+    tmem_ld32(lane_base + 64 * s + 32, r1);
     tmem_ld_wait();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&S.s_empty);
+    if (lane == 0) mbar_arrive(&S.s_empty[s]);
     const float *rs = S.rscale[s] + key0;
     float z[32];
     float mz = -INFINITY;
@@ -580,16 +604,17 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange 
     }
     tc_fence_after();
     if (__any_sync(0xFFFFFFFFu, need_rescale)) {
+      // O rows only (lanes 0..15 of the quadrant): lanes 16..31 hold S, which MMA1 of a later
+      // chunk may be writing now. Thread t takes head 16 quad + t % 16, columns
+      // col + 32 (t / 16) .. +31; alpha is the same in lanes t and t ^ 16.
 #pragma unroll 1
-      for (int col = 0; col < kD; col += 32) {
+      for (int col = 0; col < kD; col += 64) {
         uint32_t o[32];
-        tmem_ld32(lane_base + col, o);
+        tmem_ld16x2(lane_base + col, o);
         tmem_ld_wait();
-        if (!hi) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-        }
-        tmem_st32(lane_base + col, o);
+        for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+        tmem_st16x2(lane_base + col, o);
       }
       tmem_st_wait();
     }
@@ -628,10 +653,14 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
       mbar_init(&S.k_empty[i], 1);
     }
     mbar_init(&S.q_full, 4);
-    mbar_init(&S.s_full, 1);
-    mbar_init(&S.s_empty, 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&S.s_full[i], 1);
+      mbar_init(&S.s_empty[i], 4);
+    }
     mbar_init(&S.p_full, 4);
     mbar_init(&S.o_full, 1);
+    mbar_init(&S.mma_done, 1);
+    mbar_init(&S.part_full, 1);
     S.abort_flag = 0;
     fence_mbar_init();
   }
@@ -660,36 +689,22 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     if (lane == 0) mma_role(p, S, cr, tmem);
   } else softmax_role(P, S, cr, tmem);
 
-  // ---- merge of the cluster's partials: the weight of each CTA's (R, l) per head
+  // ---- merge of the cluster's partials. CTA q owns output columns [q Dc, (q + 1) Dc). As
+  // soon as its own chunks are done, each CTA stages its O (in units of its 2^R) in rbuf as
+  // one [kH][Dc] slab per owner (16-byte runs swizzled by row), bulk-copies the other
+  // owners' slabs to global memory and writes its (R, l) there too; after one cluster barrier
+  // each owner bulk-loads the cs - 1 slabs made for it into the freed slots and adds all cs
+  // slabs with the weights 2^(R - M). Nothing crosses the cluster's shared-memory network
+  // (L2 moves the slabs several times faster).
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  cluster_sync_all();
-  if (tid < kH) {
-    float m[kMaxCluster], l[kMaxCluster];
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) {
-      m[r] = r < static_cast<int>(cs) ? ld_cluster_f32(cluster_addr(&S.red_m[tid], r)) : -INFINITY;
-      l[r] = r < static_cast<int>(cs) ? ld_cluster_f32(cluster_addr(&S.red_l[tid], r)) : 0.f;
-    }
-    float M = -INFINITY;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) M = fmaxf(M, m[r]);
-    float Ls = 0.f;
-#pragma unroll
-    for (int r = 0; r < kMaxCluster; ++r) Ls += m[r] == -INFINITY ? 0.f : exp2f(m[r] - M) * l[r];
-    const float mine = S.red_m[tid];
-    S.wgt[tid] = mine == -INFINITY ? 0.f : exp2f(mine - M);
-    S.inv_l[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
-    S.lse[tid] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
-  }
-  __syncthreads();
-  // this CTA's O times its weight into obuf (the key tiles are free): warp w reads TMEM
-  // lanes of quadrant w % 4, columns 256 (w / 4) .. +255
+  const int lcs = __ffs(static_cast<int>(cs)) - 1;  // cs is a power of two
+  const int Dc = kD >> lcs, runs = Dc / 4, slab = kH * Dc;
+  // warp w reads TMEM lanes of quadrant w % 4, columns 256 (w / 4) .. +255
   if (warp < 8) {
     const int quad = warp & 3, h = quad * 16 + (lane & 15), col0 = (warp >> 2) * 256;
     const bool has = cr.lo < cr.hi && !S.abort_flag;
-    const float w = S.wgt[h];
 #pragma unroll 1
     for (int col = col0; col < col0 + 256; col += 64) {
       uint32_t o[2][32];
@@ -703,43 +718,77 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         for (int c = 0; c < 2; ++c)
 #pragma unroll
           for (int i = 0; i < 32; i += 4) {
-            const int run = (col + 32 * c + i) >> 2;
-            const float4 v = has ? make_float4(__uint_as_float(o[c][i]) * w, __uint_as_float(o[c][i + 1]) * w,
-                                               __uint_as_float(o[c][i + 2]) * w, __uint_as_float(o[c][i + 3]) * w)
+            const int d = col + 32 * c + i, q = d >> (9 - lcs);
+            const float4 v = has ? make_float4(__uint_as_float(o[c][i]), __uint_as_float(o[c][i + 1]),
+                                               __uint_as_float(o[c][i + 2]), __uint_as_float(o[c][i + 3]))
                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4 *>(&S.obuf[h][obuf_run(h, run) * 4]) = v;
+            *reinterpret_cast<float4 *>(&S.rbuf[q * slab + h * Dc + slab_run(h, (d & (Dc - 1)) >> 2) * 4]) = v;
           }
       }
     }
   }
+  float *const part_b = P.part + static_cast<size_t>(b) * cs * (cs - 1) * slab;
+  float *const red_b = P.red + static_cast<size_t>(b) * cs * 2 * kH;
+  if (tid < kH) {
+    red_b[(rank * 2) * kH + tid] = S.red_m[tid];
+    red_b[(rank * 2 + 1) * kH + tid] = S.red_l[tid];
+  }
   tc_fence_before();
+  fence_proxy_async_smem();  // the staged slabs are read by the bulk copies
   __syncthreads();
-  cluster_sync_all();
-  // CTA r finishes columns [r * Dc, (r + 1) * Dc): the sum over the cluster, / l, inverse
-  // RoPE, store
-  {
-    const int Dc = kD / static_cast<int>(cs), runs = Dc / 4, rope0 = kD - p.rope_dims;
-    for (int e = tid; e < kH * runs; e += kThreads) {
-      const int h = e / runs, d = static_cast<int>(rank) * Dc + (e % runs) * 4;
-      const uint32_t a = smem_u32(&S.obuf[h][obuf_run(h, d >> 2) * 4]);
-      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      float4 v[kMaxCluster];
-#pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) {
-        if (r < static_cast<int>(cs)) {
-          uint32_t ra;
-          asm("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(r));
-          v[r] = ld_cluster_v4(ra);
-        }
+  if (tid == 0 && cs > 1) {
+    float *dst = part_b + static_cast<size_t>(rank) * (cs - 1) * slab;
+    for (uint32_t q = 0; q < cs; ++q)
+      if (q != rank) {
+        bulk_store(dst, &S.rbuf[q * slab], static_cast<uint32_t>(slab * sizeof(float)));
+        dst += slab;
       }
-#pragma unroll
-      for (int r = 0; r < kMaxCluster; ++r) {
-        if (r < static_cast<int>(cs)) {
-          acc.x += v[r].x;
-          acc.y += v[r].y;
-          acc.z += v[r].z;
-          acc.w += v[r].w;
-        }
+    bulk_store_wait_all();  // (also frees the slots for the loads below)
+  }
+  cluster_sync_all();  // every CTA's slabs and (R, l) are in global memory
+  if (tid == 0 && cs > 1) {
+    fence_proxy_async_global();
+    mbar_arrive_expect_tx(&S.part_full, static_cast<uint32_t>((cs - 1) * slab * sizeof(float)));
+    for (uint32_t src = 0; src < cs; ++src)
+      if (src != rank)
+        bulk_load(&S.rbuf[src * slab],
+                  part_b + (static_cast<size_t>(src) * (cs - 1) + (rank < src ? rank : rank - 1)) * slab,
+                  static_cast<uint32_t>(slab * sizeof(float)), &S.part_full);
+  }
+  if (tid < kH) {  // the weights of head tid
+    float M = -INFINITY;
+    for (uint32_t r = 0; r < cs; ++r) M = fmaxf(M, __ldcg(&red_b[(r * 2) * kH + tid]));
+    float Ls = 0.f;
+    for (uint32_t r = 0; r < cs; ++r) {
+      const float m = __ldcg(&red_b[(r * 2) * kH + tid]), l = __ldcg(&red_b[(r * 2 + 1) * kH + tid]);
+      const float w = m == -INFINITY ? 0.f : exp2f(m - M);
+      S.wsrc[r][tid] = w;
+      Ls += w * l;
+    }
+    S.inv_l[tid] = Ls > 0.f ? 1.f / Ls : 0.f;
+    S.lse[tid] = Ls > 0.f ? (M + log2f(Ls)) * kLn2 : -INFINITY;
+  }
+  if (cs > 1) {
+    volatile int no_abort = 0;
+    if (!mbar_wait(&S.part_full, 0u, &no_abort) && tid == 0) S.abort_flag = 1;
+  }
+  __syncthreads();
+  // CTA rank finishes its columns: the weighted sum of the cs slabs, / l, inverse RoPE, store
+  {
+    const int rope0 = kD - p.rope_dims;
+    const int lruns = 7 - lcs;  // runs = 2^lruns
+    for (int e = tid; e < kH * runs; e += kThreads) {
+      const int h = e >> lruns, r4 = e & (runs - 1), d = static_cast<int>(rank) * Dc + r4 * 4;
+      const int at = h * Dc + slab_run(h, r4) * 4;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 4
+      for (uint32_t src = 0; src < cs; ++src) {
+        const float w = S.wsrc[src][h];
+        const float4 v = *reinterpret_cast<const float4 *>(&S.rbuf[src * slab + at]);
+        acc.x += w * v.x;
+        acc.y += w * v.y;
+        acc.z += w * v.z;
+        acc.w += w * v.w;
       }
       const float il = S.inv_l[h];
       float y[4] = {acc.x * il, acc.y * il, acc.z * il, acc.w * il};
@@ -764,7 +813,6 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     if (rank == 0 && p.lse && tid < kH) p.lse[static_cast<size_t>(b) * kH + tid] = S.lse[tid];
   }
   if (tid == 0 && S.abort_flag) report(p.d_status, DSV4_DEV_TIMEOUT);
-  cluster_sync_all();  // no CTA leaves while another may still read its shared memory
   if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc(tmem, 512);
@@ -888,17 +936,27 @@ bool mqa_uses_tensor_cores(const MqaLaunch &p) {
          p.rope_dims % 8 == 0 && p.B <= 1024;
 }
 
-size_t mqa_workspace_bytes(const MqaLaunch &p) {
-  if (!mqa_uses_tensor_cores(p)) return 0;
-  return align_up(static_cast<size_t>(p.B) * kH * kD * sizeof(uint16_t), 256) +
-         align_up(static_cast<size_t>(p.B) * kH * sizeof(float), 256);
-}
-
-// CTAs per sequence: as many as keep the batch within one wave of SMs (a power of two, at
-// most 16, and at most 8 where the device cannot co-schedule 16 of these CTAs)
-static int mqa_cluster(const MqaLaunch &p, size_t smem) {
+// CTAs per sequence by the batch alone: as many as keep the batch within one wave of SMs
+// (a power of two, at most 16). The launch may take fewer (below), never more.
+static int mqa_cluster_rule(const MqaLaunch &p) {
   int cs = 1;
   while (cs < kMaxCluster && static_cast<long long>(cs) * 2 * p.B <= sm_count()) cs <<= 1;
+  return cs;
+}
+
+size_t mqa_workspace_bytes(const MqaLaunch &p) {
+  if (!mqa_uses_tensor_cores(p)) return 0;
+  const size_t cs = static_cast<size_t>(mqa_cluster_rule(p));
+  return align_up(static_cast<size_t>(p.B) * kH * kD * sizeof(uint16_t), 256) +
+         align_up(static_cast<size_t>(p.B) * kH * sizeof(float), 256) +
+         align_up(static_cast<size_t>(p.B) * kMaxCluster * 2 * kH * sizeof(float), 256) +
+         align_up(static_cast<size_t>(p.B) * (cs - 1) * kH * kD * sizeof(float), 256);
+}
+
+// CTAs per sequence: the rule above, at most 8 where the device cannot co-schedule 16 of
+// these CTAs
+static int mqa_cluster(const MqaLaunch &p, size_t smem) {
+  int cs = mqa_cluster_rule(p);
   if (cs > 8) {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B));
@@ -930,6 +988,10 @@ static MqaTcParams tc_params(const MqaLaunch &p0, void *ws) {
   P.qp = reinterpret_cast<uint16_t *>(w);
   w += align_up(static_cast<size_t>(p0.B) * kH * kD * sizeof(uint16_t), 256);
   P.qinv = reinterpret_cast<float *>(w);
+  w += align_up(static_cast<size_t>(p0.B) * kH * sizeof(float), 256);
+  P.red = reinterpret_cast<float *>(w);
+  w += align_up(static_cast<size_t>(p0.B) * kMaxCluster * 2 * kH * sizeof(float), 256);
+  P.part = reinterpret_cast<float *>(w);
   return P;
 }
 

@@ -213,9 +213,12 @@ def test_indexer_cuda_core_path_fp32_with_query_rope():
 
 
 # ---------------------------------------------------------------------------- attention
-def _mqa_case(spec, B, pos, n_entries, idx=None, seed=41, value_std=1.0, out_dtype=None, garbage_ws=True):
-    la = W.make_layer(spec, B, max(n_entries) + 1, seed, value_std=value_std, outlier_frac=0.05)
-    st = W.make_step(spec, B, pos, seed + 1, q_std=value_std)
+def _mqa_case(spec, B, pos, n_entries, idx=None, seed=41, value_std=1.0, out_dtype=None, garbage_ws=True,
+              tweak=None, q_std=None, outlier_frac=0.05):
+    la = W.make_layer(spec, B, max(n_entries) + 1, seed, value_std=value_std, outlier_frac=outlier_frac)
+    if tweak is not None:
+        tweak(la)
+    st = W.make_step(spec, B, pos, seed + 1, q_std=value_std if q_std is None else q_std)
     dl = dsv4.DeviceLayer.from_arrays(la)
     q = dsv4.to_device_codes(st.q, spec.q_dtype, "cuda")
     status = torch.zeros(1, dtype=torch.int32, device="cuda")
@@ -277,6 +280,34 @@ def test_mqa_tensor_core_sparse_fp8_with_padding_and_bad_index():
             o, l = _ref_attention(ol, qd, st, s, sel, spec)
             check_output(out[s], o, "lowp", f"seq {s} out {out_dtype}", stored_bf16=out_dtype == "bf16")
             assert np.max(np.abs(lse[s] - l)) < 2e-2
+
+
+def test_mqa_tensor_core_rising_logits_rescale_the_output():
+    """Selected keys whose logits rise by about 10 (log2 units) from one 64-key chunk to the
+    next within each CTA's run: about half of the (head, chunk) steps raise the head's
+    reference max by more than the lazy threshold, so the partial output accumulated so far
+    is rescaled, chunk after chunk. 40 sequences run two CTAs each (chunks 0-4 and 5-9, the
+    first two being the window). The row gains per 64 selected keys keep the largest logit
+    near 55 and the outputs of order one, where fp16 operands still meet the tolerance."""
+    spec = W.C4_SPEC
+    B, n_c = 40, 3000
+    gains = [4, 7, 10, 0.3, 3, 6, 9, 1]
+    rng = np.random.default_rng(8)
+    idx = np.stack([rng.permutation(n_c)[:512] for _ in range(B)]).astype(np.int64)
+
+    def rising(la):
+        per_page = spec.per_page
+        for s in range(B):
+            for u, j in enumerate(idx[s]):
+                la.scales[la.block_table[s, j // per_page], j % per_page] *= np.float32(gains[u // 64])
+
+    out, lse, status, ol, qd, st = _mqa_case(spec, B, [131072] * B, [n_c] * B, idx=idx, out_dtype="f32",
+                                             tweak=rising, value_std=0.1, q_std=10.0, outlier_frac=0.0)
+    assert status == 0
+    for s in range(B):
+        o, l = _ref_attention(ol, qd, st, s, idx[s], spec)
+        check_output(out[s], o, "lowp", f"seq {s}")
+        assert np.max(np.abs(lse[s] - l)) < 2e-2
 
 
 def test_mqa_cuda_core_fp32():
