@@ -129,6 +129,7 @@ struct alignas(1024) MqaSmem {
   uint64_t k_full[2], k_empty[2], q_full, s_full[2], s_empty[2], p_full, o_full, mma_done, part_full;
   uint32_t tmem_base;
   int abort_flag;
+  int dry[kThreads / 32];  // per warp: 1 during its first, dry pass (see the kernel)
 };
 
 static_assert(sizeof(MqaSmem) + 1024 <= 227 * 1024, "attention shared memory exceeds one SM");
@@ -141,6 +142,12 @@ struct MqaTcParams {
   float *part;     // [B][cs][cs - 1] slabs [H][D / cs]: CTA src's O for owner dst != src
   float *red;      // [B][cs][2][H]: each CTA's reference max R and sum l per head
 };
+
+// The dry pass of this warp: read from shared memory at every use, so that the compiler
+// keeps one copy of the code for both passes.
+__device__ __forceinline__ bool dry_pass(const MqaSmem &S) {
+  return *reinterpret_cast<const volatile int *>(&S.dry[threadIdx.x >> 5]) != 0;
+}
 
 // Operands of the two MMAs. fp8 caches: fp16 (e4m3 -> fp16 is exact, and fp16 keeps 11
 // significand bits of the rotated query and of P); bf16 caches: bf16.
@@ -180,11 +187,17 @@ struct ChunkRange {
 // memory latencies are paid once per batch.
 __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const KeyList &L, const ChunkRange &cr) {
   const int lane = threadIdx.x & 31, b = cr.b;
-  const int per_page = DSV4_PAGE_POSITIONS / p.m;
+  // entries per page and the window's first ring slot (m and the page size are powers of two)
+  const int per_shift = __ffs(DSV4_PAGE_POSITIONS) - __ffs(p.m), per_mask = (1 << per_shift) - 1;
+  const int64_t w0 = L.nw > 0 ? (L.pos - L.nw + 1) % p.W : 0;
   const size_t esz = dtype_size(p.kv_dt);
   constexpr int kKeys = kMetaSlots * 2;  // keys per lane per batch
-  for (long long g0 = cr.lo; g0 < cr.hi; g0 += kMetaSlots) {
-    const int nb = static_cast<int>(cr.hi - g0 < kMetaSlots ? cr.hi - g0 : kMetaSlots);
+  // the dry pass goes once through one batch with no wait and no arrival, every key taken
+  // as "none" (so every load reads element 0 of its array)
+  const bool dry = dry_pass(S);
+  const long long hi = dry ? (cr.lo < cr.hi ? cr.lo + 1 : cr.lo) : cr.hi;
+  for (long long g0 = cr.lo; g0 < hi; g0 += kMetaSlots) {
+    const int nb = static_cast<int>(hi - g0 < kMetaSlots ? hi - g0 : kMetaSlots);
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
       const long long n = g0 + i - cr.lo;
@@ -205,7 +218,7 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const KeyList &L, cons
     for (int u = 0; u < kKeys; ++u) {
       const int i = u >> 1;
       t_u[u] = (g0 + i) * kCh + lane + 32 * (u & 1);
-      kind[u] = i >= nb ? 0 : (t_u[u] < L.nw ? 1 : (t_u[u] - L.nw < L.nsel ? 2 : 0));
+      kind[u] = (i >= nb || dry) ? 0 : (t_u[u] < L.nw ? 1 : (t_u[u] - L.nw < L.nsel ? 2 : 0));
     }
 #pragma unroll
     for (int u = 0; u < kKeys; ++u) {  // stage 1: list position -> entry index (idx load)
@@ -213,48 +226,60 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const KeyList &L, cons
       j[u] = uu;
       if (p.idx) j[u] = p.idx[static_cast<size_t>(b) * p.k + uu];
     }
+    // (every stage issues its loads first and reports bad values after them, so that no
+    // atomic sits between two loads)
+    bool bad_index = false, bad_page = false;
+#pragma unroll
+    for (int u = 0; u < kKeys; ++u) {  // entries out of range and padding: no key
+      if (kind[u] == 2 && j[u] >= L.n_entries) bad_index = true;
+      if (kind[u] == 2 && (j[u] < 0 || j[u] >= L.n_entries)) kind[u] = 0;
+    }
     int32_t page[kKeys];
 #pragma unroll
-    for (int u = 0; u < kKeys; ++u) {  // stage 2: entry -> physical page (block table load)
-      bool ok = kind[u] == 2 && j[u] >= 0;
-      if (ok && j[u] >= L.n_entries) {
-        report(p.d_status, DSV4_DEV_BAD_INDEX);
-        ok = false;
-      }
-      if (!ok && kind[u] == 2) kind[u] = 0;  // padding or a bad index: no key
-      page[u] = p.block_table[static_cast<size_t>(b) * p.max_blocks + (ok ? j[u] / per_page : 0)];
-    }
+    for (int u = 0; u < kKeys; ++u)  // stage 2: entry -> physical page (block table load)
+      page[u] = p.block_table[static_cast<size_t>(b) * p.max_blocks + (kind[u] == 2 ? j[u] >> per_shift : 0)];
+    size_t slot_or_row[kKeys];
 #pragma unroll
-    for (int u = 0; u < kKeys; ++u) {  // stage 3: row address and scale
-      const int i = u >> 1;
-      size_t slot_or_row = 0;
+    for (int u = 0; u < kKeys; ++u) {
+      slot_or_row[u] = 0;
       if (kind[u] == 1) {
-        const int64_t pw = L.pos - L.nw + 1 + t_u[u];
-        slot_or_row = static_cast<size_t>(b) * p.W + static_cast<size_t>(pw % p.W);
+        int64_t slot = w0 + t_u[u];  // t < nw <= W
+        if (slot >= p.W) slot -= p.W;
+        slot_or_row[u] = static_cast<size_t>(b) * p.W + static_cast<size_t>(slot);
       } else if (kind[u] == 2) {
         if (page[u] < 0 || page[u] >= p.num_pages) {
-          report(p.d_status, DSV4_DEV_BAD_PAGE);
+          bad_page = true;
           kind[u] = 0;
         } else {
-          slot_or_row = static_cast<size_t>(page[u]) * per_page + static_cast<size_t>(j[u] % per_page);
+          slot_or_row[u] = (static_cast<size_t>(page[u]) << per_shift) + static_cast<size_t>(j[u] & per_mask);
         }
       }
-      float sc = 1.0f;
-      if (p.kv_dt == DSV4_FP8E4M3) sc = (kind[u] == 1 ? p.ring_scales : p.scales)[kind[u] == 0 ? 0 : slot_or_row];
+    }
+    float sc[kKeys];
+#pragma unroll
+    for (int u = 0; u < kKeys; ++u) {  // stage 3: row scale
+      sc[u] = 1.0f;
+      if (p.kv_dt == DSV4_FP8E4M3) sc[u] = (kind[u] == 1 ? p.ring_scales : p.scales)[kind[u] == 0 ? 0 : slot_or_row[u]];
+    }
+#pragma unroll
+    for (int u = 0; u < kKeys; ++u) {
+      const int i = u >> 1;
       const uint8_t *rp = kind[u] == 0 ? nullptr
                                        : static_cast<const uint8_t *>(kind[u] == 1 ? p.ring_rows : p.pages) +
-                                             slot_or_row * p.D * esz;
+                                             slot_or_row[u] * p.D * esz;
       if (i < nb) {
         const int slot = static_cast<int>((g0 + i - cr.lo) % kMetaSlots);
         S.mrow[slot][lane + 32 * (u & 1)] = rp;
-        S.mscale[slot][lane + 32 * (u & 1)] = rp ? sc : 0.f;
+        S.mscale[slot][lane + 32 * (u & 1)] = rp ? sc[u] : 0.f;
         // the gather of this CTA's third and later chunks waits for a free tile stage: their
         // rows travel to L2 meanwhile
         if (rp && g0 + i - cr.lo >= 2) bulk_prefetch_l2(rp, static_cast<uint32_t>(p.D * esz));
       }
     }
+    if (bad_index) report(p.d_status, DSV4_DEV_BAD_INDEX);
+    if (bad_page) report(p.d_status, DSV4_DEV_BAD_PAGE);
     __syncwarp();
-    if (lane == 0)
+    if (lane == 0 && !dry)
       for (int i = 0; i < nb; ++i) mbar_arrive(&S.meta_full[(g0 + i - cr.lo) % kMetaSlots]);
   }
 }
@@ -364,20 +389,27 @@ __device__ __forceinline__ void gather_issue_bf16(const MqaSmem &S, uint8_t *kt,
   cp_async_commit();
 }
 
-__device__ __forceinline__ void gather_load_fp8(const MqaSmem &S, int ms, int gw, int lane, uint4 (&v)[16]) {
+__device__ __forceinline__ void gather_load_fp8(const MqaSmem &S, int ms, int gw, int lane, uint4 (&v)[16],
+                                                bool none) {
 #pragma unroll
   for (int rr = 0; rr < 16; ++rr) {
-    const uint8_t *rp = S.mrow[ms][gw * 16 + rr];
+    const uint8_t *rp = none ? nullptr : S.mrow[ms][gw * 16 + rr];
     v[rr] = rp ? __ldg(reinterpret_cast<const uint4 *>(rp + lane * 16)) : make_uint4(0, 0, 0, 0);
   }
 }
 
+// 2^e as a float (exact; e outside the normal range goes through ldexpf)
+__device__ __forceinline__ float pow2f(int e) {
+  return (e >= -126 && e <= 127) ? __int_as_float((127 + e) << 23) : ldexpf(1.0f, e);
+}
+
 __device__ __forceinline__ void gather_store_fp8(MqaSmem &S, uint8_t *kt, int ms, int ec, int gw, int lane, const uint4 (&v)[16]) {
   const int atom = lane >> 2, c0 = (lane & 3) * 2;
+  const float f = pow2f(-ec);  // row scale * 2^-ec: exact (a power-of-two factor)
 #pragma unroll
   for (int rr = 0; rr < 16; ++rr) {
     const int row = gw * 16 + rr;
-    const __half2 sc2 = __float2half2_rn(ldexpf(S.mscale[ms][row], -ec));
+    const __half2 sc2 = __float2half2_rn(S.mscale[ms][row] * f);
     const uint32_t w[4] = {v[rr].x, v[rr].y, v[rr].z, v[rr].w};
     uint32_t o[8];
 #pragma unroll
@@ -395,16 +427,43 @@ __device__ __forceinline__ void gather_store_fp8(MqaSmem &S, uint8_t *kt, int ms
   }
 }
 
+// fp8 rows are software-pipelined: the rows of chunk n + 1 are loaded into registers before
+// chunk n is converted and before the tile stage of chunk n + 1 is free, so their memory
+// latency overlaps the conversion and the wait. The metadata of chunk n + 1 is awaited in
+// iteration n: early, or, when chunk n + 1 opens a new metadata batch (which the metadata
+// warp resolves only once every slot of the batch before is released, this chunk's
+// included), after chunk n released its slot.
 __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &cr) {
   const MqaLaunch &p = P.a;
   const int lane = threadIdx.x & 31, gw = (threadIdx.x >> 5) - kGatherWarp0;
   const bool fp8 = p.kv_dt == DSV4_FP8E4M3;
-  if (cr.lo < cr.hi) query_issue(P, S, cr.b, gw, lane);
-  for (long long g = cr.lo; g < cr.hi; ++g) {
-    const long long n = g - cr.lo;
+  // the dry pass goes once through the loop with no wait, no arrival and no row read
+  const bool dry = dry_pass(S);
+  const long long nc = dry ? (cr.lo < cr.hi ? 1 : 0) : cr.hi - cr.lo;
+  if (nc > 0 && !dry) query_issue(P, S, cr.b, gw, lane);
+  uint4 nxt[16];  // rows of the next chunk (fp8)
+  if (nc > 0) {
+    const bool ok = dry || mbar_wait(&S.meta_full[0], 0u, &S.abort_flag);
+    if (!__all_sync(0xFFFFFFFFu, ok)) {
+      if (lane == 0) S.abort_flag = 1;
+      return;
+    }
+    if (fp8) gather_load_fp8(S, 0, gw, lane, nxt, dry);
+  }
+  for (long long n = 0; n < nc; ++n) {
     const int s = static_cast<int>(n & 1), ms = static_cast<int>(n % kMetaSlots);
-    bool ok = mbar_wait(&S.meta_full[ms], static_cast<uint32_t>((n / kMetaSlots) & 1), &S.abort_flag);
+    uint4 v[16];
+#pragma unroll
+    for (int rr = 0; rr < 16; ++rr) v[rr] = nxt[rr];
+    bool ok = true;
+    const bool ahead = n + 1 < nc && (n + 1) % kMetaSlots != 0;
+    if (ahead) {
+      ok = mbar_wait(&S.meta_full[(n + 1) % kMetaSlots], static_cast<uint32_t>(((n + 1) / kMetaSlots) & 1),
+                     &S.abort_flag);
+      if (ok && fp8) gather_load_fp8(S, static_cast<int>((n + 1) % kMetaSlots), gw, lane, nxt, false);
+    }
     if (ok && n >= 2) ok = mbar_wait(&S.k_empty[s], static_cast<uint32_t>((n / 2 - 1) & 1), &S.abort_flag);
+    // (the dry pass reads placeholder metadata below and converts zero rows)
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) S.abort_flag = 1;
       break;
@@ -417,26 +476,33 @@ __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &
     int ec = 0;
     if (fp8) frexpf(smax, &ec);  // largest scale = f * 2^ec, f in [0.5, 1)
     if (lane < 16) S.rscale[s][gw * 16 + lane] = S.mscale[ms][gw * 16 + lane];
-    if (gw == 0 && lane == 0) S.ec[s] = ec;
+    if (gw == 0 && lane == 0 && !dry) S.ec[s] = ec;
     if (fp8) {
-      uint4 v[16];
-      gather_load_fp8(S, ms, gw, lane, v);
       gather_store_fp8(S, kt, ms, ec, gw, lane, v);
-    } else {
+    } else if (!dry) {
       gather_issue_bf16(S, kt, ms, gw, lane);
       cp_async_wait_all();
     }
     fence_proxy_async_smem();
     __syncwarp();
-    if (lane == 0) {
+    if (lane == 0 && !dry) {
       mbar_arrive(&S.k_full[s]);
       mbar_arrive(&S.meta_empty[ms]);
     }
-    if (n == 0) {
+    if (n == 0 && !dry) {
       query_finish(P, S, cr.b, gw, lane);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&S.q_full);
+    }
+    if (n + 1 < nc && !ahead) {
+      ok = mbar_wait(&S.meta_full[(n + 1) % kMetaSlots], static_cast<uint32_t>(((n + 1) / kMetaSlots) & 1),
+                     &S.abort_flag);
+      if (!__all_sync(0xFFFFFFFFu, ok)) {
+        if (lane == 0) S.abort_flag = 1;
+        break;
+      }
+      if (fp8) gather_load_fp8(S, static_cast<int>((n + 1) % kMetaSlots), gw, lane, nxt, false);
     }
   }
   cp_async_wait_all();
@@ -454,10 +520,15 @@ __device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const ChunkRange &cr, u
   const uint32_t s_tmem = tmem + (16u << 16);
   const uint64_t qd = sw128_desc(smem_u32(&S.q[0][0]), 16, 1024);
   const uint64_t pd = sw128_desc(smem_u32(S.p), 16, 1024);
-  const long long nc = cr.hi - cr.lo;
+  // the dry pass goes once through the loop below without waiting and with every MMA and
+  // commit predicated off
+  const bool dry = dry_pass(S);
+  const uint32_t en = dry ? 0u : 1u;
+  const long long nc = dry ? (cr.lo < cr.hi ? 1 : 0) : cr.hi - cr.lo;
   // chunk m may take MMA1 once the query (chunk 0) and its tile are staged and the softmax
   // has read S of chunk m - 2
   auto s_ready = [&](long long m) {
+    if (dry) return true;
     return (m > 0 || mbar_try_wait(&S.q_full, 0u)) &&
            mbar_try_wait(&S.k_full[m & 1], static_cast<uint32_t>((m >> 1) & 1)) &&
            (m < 2 || mbar_try_wait(&S.s_empty[m & 1], static_cast<uint32_t>(((m - 2) >> 1) & 1)));
@@ -470,9 +541,9 @@ __device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const ChunkRange &cr, u
     for (int kk = 0; kk < kD / 16; ++kk) {  // descriptor start advances in 16-byte units
       const uint32_t off = ((kk >> 2) * (kH * 128) + (kk & 3) * 32) >> 4;
       const uint32_t offk = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
-      mma_bf16(dt, qd + off, kd + offk, idesc1, kk > 0 ? 1u : 0u);
+      mma_bf16_if(en, dt, qd + off, kd + offk, idesc1, kk > 0 ? 1u : 0u);
     }
-    mma_commit(&S.s_full[m & 1]);
+    mma_commit_if(en, &S.s_full[m & 1]);
   };
   long long next = 0;  // the next chunk to take MMA1
   bool ok = true;
@@ -486,7 +557,7 @@ __device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const ChunkRange &cr, u
         issue_s(next++);
         continue;
       }
-      if (mbar_try_wait(&S.p_full, static_cast<uint32_t>(n & 1))) break;
+      if (dry || mbar_try_wait(&S.p_full, static_cast<uint32_t>(n & 1))) break;
       __nanosleep(ns);
       if (ns < 128) ns <<= 1;
       if ((i & 15) == 0 && (S.abort_flag || globaltimer() - t0 > kWaitLimitNs)) {
@@ -502,13 +573,13 @@ __device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const ChunkRange &cr, u
     for (int nh = 0; nh < 2; ++nh)
 #pragma unroll
       for (int ks = 0; ks < kCh / 16; ++ks)
-        mma_bf16(tmem + nh * 256, pd + ks * 2, sw128_desc(ka + nh * 4 * kAtom + ks * 2048, kAtom, 1024), idesc2,
-                 (n > 0 || ks > 0) ? 1u : 0u);
-    mma_commit(&S.k_empty[n & 1]);
-    mma_commit(&S.o_full);
+        mma_bf16_if(en, tmem + nh * 256, pd + ks * 2, sw128_desc(ka + nh * 4 * kAtom + ks * 2048, kAtom, 1024),
+                    idesc2, (n > 0 || ks > 0) ? 1u : 0u);
+    mma_commit_if(en, &S.k_empty[n & 1]);
+    mma_commit_if(en, &S.o_full);
   }
   // let every MMA issued here finish (also after an abort) before anyone reads or frees the TMEM
-  if (next > 0) {
+  if (next > 0 && !dry) {
     mma_commit(&S.mma_done);
     volatile int dummy = 0;
     mbar_wait(&S.mma_done, 0u, &dummy);
@@ -537,8 +608,11 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange 
   bool done = true;
   for (long long g = cr.lo; g < cr.hi; ++g, ++n) {
     const int s = static_cast<int>(n & 1);
-    bool ok = mbar_wait(&S.k_full[s], static_cast<uint32_t>((n / 2) & 1), &S.abort_flag);
-    ok = ok && mbar_wait(&S.s_full[s], static_cast<uint32_t>((n >> 1) & 1), &S.abort_flag);
+    bool ok = true;
+    if (!dry_pass(S)) {
+      ok = mbar_wait(&S.k_full[s], static_cast<uint32_t>((n / 2) & 1), &S.abort_flag);
+      ok = ok && mbar_wait(&S.s_full[s], static_cast<uint32_t>((n >> 1) & 1), &S.abort_flag);
+    }
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) S.abort_flag = 1;
       done = false;
@@ -555,7 +629,7 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange 
     tmem_ld_wait();
     tc_fence_before();
     __syncwarp();
-    if (lane == 0) mbar_arrive(&S.s_empty[s]);
+    if (lane == 0 && !dry_pass(S)) mbar_arrive(&S.s_empty[s]);
     const float *rs = S.rscale[s] + key0;
     float z[32];
     float mz = -INFINITY;
@@ -593,6 +667,7 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange 
       }
       lsum += a0 + a1;  // the denominator uses the rounded P, like the numerator
     }
+    if (dry_pass(S)) break;  // the dry pass stops here, having changed nothing
     l_half = l_half * alpha + lsum * lsc;
     R = Rn;
     // P and O are free once MMA2 of the previous chunk completed
@@ -627,6 +702,7 @@ __device__ void softmax_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange 
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.p_full);
   }
+  if (dry_pass(S)) return;
   const float l = l_half + __shfl_xor_sync(0xFFFFFFFFu, l_half, 16);
   if (hi) {
     S.red_m[head] = done ? R : -INFINITY;
@@ -662,6 +738,7 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     mbar_init(&S.mma_done, 1);
     mbar_init(&S.part_full, 1);
     S.abort_flag = 0;
+    for (int w = 0; w < kThreads / 32; ++w) S.dry[w] = w == kMetaWarp ? 0 : 1;
     fence_mbar_init();
   }
   if (warp == kMmaWarp) {
@@ -683,11 +760,27 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
   tc_fence_after();
   const uint32_t tmem = S.tmem_base;
 
-  if (warp == kMetaWarp) meta_role(p, S, L, cr);
-  else if (warp >= kGatherWarp0 && warp < kGatherWarp0 + 4) gather_role(P, S, cr);
-  else if (warp == kMmaWarp) {
-    if (lane == 0) mma_role(p, S, cr, tmem);
-  } else softmax_role(P, S, cr, tmem);
+  // Two passes over the roles. Code that runs once per launch is fetched at the pace of a
+  // cold instruction cache, several times slower than it executes. So the gather, MMA and
+  // softmax warps, which would only wait while the metadata warp resolves the first chunks,
+  // first go once through their long unrolled stretches over placeholder values, with no
+  // waits and no effect (their S.dry flag set), then do the real pass. The metadata warp,
+  // first in the chain, runs the real pass only.
+#pragma unroll 1
+  for (int pass = 0; pass < 2; ++pass) {
+    if (warp == kMetaWarp) {
+      if (pass == 1) meta_role(p, S, L, cr);
+    } else if (warp >= kGatherWarp0 && warp < kGatherWarp0 + 4) {
+      gather_role(P, S, cr);
+    } else if (warp == kMmaWarp) {
+      if (lane == 0) mma_role(p, S, cr, tmem);
+    } else {
+      softmax_role(P, S, cr, tmem);
+    }
+    __syncwarp();
+    if (pass == 0 && lane == 0) S.dry[warp] = 0;
+    __syncwarp();
+  }
 
   // ---- merge of the cluster's partials. CTA q owns output columns [q Dc, (q + 1) Dc). As
   // soon as its own chunks are done, each CTA stages its O (in units of its 2^R) in rbuf as
