@@ -187,17 +187,20 @@ struct ChunkRange {
 // memory latencies are paid once per batch.
 __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const KeyList &L, const ChunkRange &cr) {
   const int lane = threadIdx.x & 31, b = cr.b;
-  // entries per page and the window's first ring slot (m and the page size are powers of two)
+  // 32-bit arithmetic throughout (this code runs once per launch, so its length is its cost):
+  // entries per page (m and the page size are powers of two), the window's first ring slot
   const int per_shift = __ffs(DSV4_PAGE_POSITIONS) - __ffs(p.m), per_mask = (1 << per_shift) - 1;
-  const int64_t w0 = L.nw > 0 ? (L.pos - L.nw + 1) % p.W : 0;
-  const size_t esz = dtype_size(p.kv_dt);
+  const int nw = static_cast<int>(L.nw), W = p.W;
+  const int w0 = nw > 0 ? static_cast<int>((L.pos - L.nw + 1) % p.W) : 0;
+  const size_t row_bytes = static_cast<size_t>(p.D) * dtype_size(p.kv_dt);
+  const bool fp8 = p.kv_dt == DSV4_FP8E4M3;
+  const int32_t *idx_b = p.idx ? p.idx + static_cast<size_t>(b) * p.k : nullptr;
+  const int32_t *bt_b = p.block_table + static_cast<size_t>(b) * p.max_blocks;
+  const uint8_t *ring_b = static_cast<const uint8_t *>(p.ring_rows) + static_cast<size_t>(b) * W * row_bytes;
+  const float *ring_sc_b = fp8 ? p.ring_scales + static_cast<size_t>(b) * W : nullptr;
   constexpr int kKeys = kMetaSlots * 2;  // keys per lane per batch
-  // the dry pass goes once through one batch with no wait and no arrival, every key taken
-  // as "none" (so every load reads element 0 of its array)
-  const bool dry = dry_pass(S);
-  const long long hi = dry ? (cr.lo < cr.hi ? cr.lo + 1 : cr.lo) : cr.hi;
-  for (long long g0 = cr.lo; g0 < hi; g0 += kMetaSlots) {
-    const int nb = static_cast<int>(hi - g0 < kMetaSlots ? hi - g0 : kMetaSlots);
+  for (long long g0 = cr.lo; g0 < cr.hi; g0 += kMetaSlots) {
+    const int nb = static_cast<int>(cr.hi - g0 < kMetaSlots ? cr.hi - g0 : kMetaSlots);
     bool ok = true;
     for (int i = 0; i < nb; ++i) {
       const long long n = g0 + i - cr.lo;
@@ -211,75 +214,70 @@ __device__ void meta_role(const MqaLaunch &p, MqaSmem &S, const KeyList &L, cons
     }
     // Three stages, each with the loads of all kKeys keys issued together: every load reads
     // a clamped, always-valid address and the result is selected afterwards, so no branch
-    // separates them. kind: 0 none, 1 window row, 2 selected entry.
-    int kind[kKeys];
-    int64_t t_u[kKeys], j[kKeys];
+    // separates them; bad indices and pages are reported after the loads, so no atomic sits
+    // between two loads. kind: 0 none, 1 window row, 2 selected entry.
+    int kind[kKeys], t[kKeys], j[kKeys];
 #pragma unroll
     for (int u = 0; u < kKeys; ++u) {
       const int i = u >> 1;
-      t_u[u] = (g0 + i) * kCh + lane + 32 * (u & 1);
-      kind[u] = (i >= nb || dry) ? 0 : (t_u[u] < L.nw ? 1 : (t_u[u] - L.nw < L.nsel ? 2 : 0));
+      t[u] = static_cast<int>(g0 + i) * kCh + lane + 32 * (u & 1);
+      kind[u] = i >= nb ? 0 : (t[u] < nw ? 1 : (t[u] - nw < L.nsel ? 2 : 0));
     }
 #pragma unroll
     for (int u = 0; u < kKeys; ++u) {  // stage 1: list position -> entry index (idx load)
-      const int64_t uu = kind[u] == 2 ? t_u[u] - L.nw : 0;
-      j[u] = uu;
-      if (p.idx) j[u] = p.idx[static_cast<size_t>(b) * p.k + uu];
+      j[u] = kind[u] == 2 ? t[u] - nw : 0;
+      if (idx_b) j[u] = idx_b[j[u]];
     }
-    // (every stage issues its loads first and reports bad values after them, so that no
-    // atomic sits between two loads)
     bool bad_index = false, bad_page = false;
 #pragma unroll
     for (int u = 0; u < kKeys; ++u) {  // entries out of range and padding: no key
       if (kind[u] == 2 && j[u] >= L.n_entries) bad_index = true;
       if (kind[u] == 2 && (j[u] < 0 || j[u] >= L.n_entries)) kind[u] = 0;
     }
-    int32_t page[kKeys];
+    int page[kKeys];
 #pragma unroll
     for (int u = 0; u < kKeys; ++u)  // stage 2: entry -> physical page (block table load)
-      page[u] = p.block_table[static_cast<size_t>(b) * p.max_blocks + (kind[u] == 2 ? j[u] >> per_shift : 0)];
-    size_t slot_or_row[kKeys];
+      page[u] = bt_b[kind[u] == 2 ? j[u] >> per_shift : 0];
+    size_t row[kKeys];  // window: ring slot of the sequence; entry: row of the page pool
 #pragma unroll
     for (int u = 0; u < kKeys; ++u) {
-      slot_or_row[u] = 0;
+      row[u] = 0;
       if (kind[u] == 1) {
-        int64_t slot = w0 + t_u[u];  // t < nw <= W
-        if (slot >= p.W) slot -= p.W;
-        slot_or_row[u] = static_cast<size_t>(b) * p.W + static_cast<size_t>(slot);
+        int slot = w0 + t[u];  // t < nw <= W
+        if (slot >= W) slot -= W;
+        row[u] = static_cast<size_t>(slot);
       } else if (kind[u] == 2) {
         if (page[u] < 0 || page[u] >= p.num_pages) {
           bad_page = true;
           kind[u] = 0;
         } else {
-          slot_or_row[u] = (static_cast<size_t>(page[u]) << per_shift) + static_cast<size_t>(j[u] & per_mask);
+          row[u] = (static_cast<size_t>(page[u]) << per_shift) | static_cast<size_t>(j[u] & per_mask);
         }
       }
     }
     float sc[kKeys];
 #pragma unroll
-    for (int u = 0; u < kKeys; ++u) {  // stage 3: row scale
-      sc[u] = 1.0f;
-      if (p.kv_dt == DSV4_FP8E4M3) sc[u] = (kind[u] == 1 ? p.ring_scales : p.scales)[kind[u] == 0 ? 0 : slot_or_row[u]];
-    }
+    for (int u = 0; u < kKeys; ++u)  // stage 3: row scale
+      sc[u] = fp8 ? (kind[u] == 1 ? ring_sc_b : p.scales)[row[u]] : 1.0f;
 #pragma unroll
     for (int u = 0; u < kKeys; ++u) {
       const int i = u >> 1;
       const uint8_t *rp = kind[u] == 0 ? nullptr
-                                       : static_cast<const uint8_t *>(kind[u] == 1 ? p.ring_rows : p.pages) +
-                                             slot_or_row[u] * p.D * esz;
+                                       : (kind[u] == 1 ? ring_b : static_cast<const uint8_t *>(p.pages)) +
+                                             row[u] * row_bytes;
       if (i < nb) {
         const int slot = static_cast<int>((g0 + i - cr.lo) % kMetaSlots);
         S.mrow[slot][lane + 32 * (u & 1)] = rp;
         S.mscale[slot][lane + 32 * (u & 1)] = rp ? sc[u] : 0.f;
         // the gather of this CTA's third and later chunks waits for a free tile stage: their
         // rows travel to L2 meanwhile
-        if (rp && g0 + i - cr.lo >= 2) bulk_prefetch_l2(rp, static_cast<uint32_t>(p.D * esz));
+        if (rp && g0 + i - cr.lo >= 2) bulk_prefetch_l2(rp, static_cast<uint32_t>(row_bytes));
       }
     }
     if (bad_index) report(p.d_status, DSV4_DEV_BAD_INDEX);
     if (bad_page) report(p.d_status, DSV4_DEV_BAD_PAGE);
     __syncwarp();
-    if (lane == 0 && !dry)
+    if (lane == 0)
       for (int i = 0; i < nb; ++i) mbar_arrive(&S.meta_full[(g0 + i - cr.lo) % kMetaSlots]);
   }
 }
@@ -403,7 +401,11 @@ __device__ __forceinline__ float pow2f(int e) {
   return (e >= -126 && e <= 127) ? __int_as_float((127 + e) << 23) : ldexpf(1.0f, e);
 }
 
-__device__ __forceinline__ void gather_store_fp8(MqaSmem &S, uint8_t *kt, int ms, int ec, int gw, int lane, const uint4 (&v)[16]) {
+// Converts and stores the rows in v (chunk of metadata slot ms); with next >= 0, each row's
+// registers are refilled at once with the same row of the chunk in slot next, so those loads
+// are in flight while the rest converts.
+__device__ __forceinline__ void gather_store_fp8(MqaSmem &S, uint8_t *kt, int ms, int ec, int gw, int lane, uint4 (&v)[16],
+                                                 int next) {
   const int atom = lane >> 2, c0 = (lane & 3) * 2;
   const float f = pow2f(-ec);  // row scale * 2^-ec: exact (a power-of-two factor)
 #pragma unroll
@@ -424,15 +426,19 @@ __device__ __forceinline__ void gather_store_fp8(MqaSmem &S, uint8_t *kt, int ms
     uint8_t *base = kt + atom * kAtom;
     *reinterpret_cast<uint4 *>(base + sw128_offset(row, c0)) = make_uint4(o[0], o[1], o[2], o[3]);
     *reinterpret_cast<uint4 *>(base + sw128_offset(row, c0 + 1)) = make_uint4(o[4], o[5], o[6], o[7]);
+    if (next >= 0) {
+      const uint8_t *rp = S.mrow[next][row];
+      v[rr] = rp ? __ldg(reinterpret_cast<const uint4 *>(rp + lane * 16)) : make_uint4(0, 0, 0, 0);
+    }
   }
 }
 
-// fp8 rows are software-pipelined: the rows of chunk n + 1 are loaded into registers before
-// chunk n is converted and before the tile stage of chunk n + 1 is free, so their memory
-// latency overlaps the conversion and the wait. The metadata of chunk n + 1 is awaited in
+// fp8 rows are software-pipelined: while chunk n is converted, the registers of each row are
+// refilled with the same row of chunk n + 1, so the memory latency of chunk n + 1 overlaps the
+// conversion and the wait for its tile stage. The metadata of chunk n + 1 is awaited in
 // iteration n: early, or, when chunk n + 1 opens a new metadata batch (which the metadata
 // warp resolves only once every slot of the batch before is released, this chunk's
-// included), after chunk n released its slot.
+// included), after chunk n released its slot (and its rows are loaded then).
 __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &cr) {
   const MqaLaunch &p = P.a;
   const int lane = threadIdx.x & 31, gw = (threadIdx.x >> 5) - kGatherWarp0;
@@ -441,27 +447,22 @@ __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &
   const bool dry = dry_pass(S);
   const long long nc = dry ? (cr.lo < cr.hi ? 1 : 0) : cr.hi - cr.lo;
   if (nc > 0 && !dry) query_issue(P, S, cr.b, gw, lane);
-  uint4 nxt[16];  // rows of the next chunk (fp8)
+  uint4 v[16];  // rows of the chunk at hand (fp8)
   if (nc > 0) {
     const bool ok = dry || mbar_wait(&S.meta_full[0], 0u, &S.abort_flag);
     if (!__all_sync(0xFFFFFFFFu, ok)) {
       if (lane == 0) S.abort_flag = 1;
       return;
     }
-    if (fp8) gather_load_fp8(S, 0, gw, lane, nxt, dry);
+    if (fp8) gather_load_fp8(S, 0, gw, lane, v, dry);
   }
   for (long long n = 0; n < nc; ++n) {
     const int s = static_cast<int>(n & 1), ms = static_cast<int>(n % kMetaSlots);
-    uint4 v[16];
-#pragma unroll
-    for (int rr = 0; rr < 16; ++rr) v[rr] = nxt[rr];
     bool ok = true;
     const bool ahead = n + 1 < nc && (n + 1) % kMetaSlots != 0;
-    if (ahead) {
+    if (ahead)
       ok = mbar_wait(&S.meta_full[(n + 1) % kMetaSlots], static_cast<uint32_t>(((n + 1) / kMetaSlots) & 1),
                      &S.abort_flag);
-      if (ok && fp8) gather_load_fp8(S, static_cast<int>((n + 1) % kMetaSlots), gw, lane, nxt, false);
-    }
     if (ok && n >= 2) ok = mbar_wait(&S.k_empty[s], static_cast<uint32_t>((n / 2 - 1) & 1), &S.abort_flag);
     // (the dry pass reads placeholder metadata below and converts zero rows)
     if (!__all_sync(0xFFFFFFFFu, ok)) {
@@ -478,7 +479,7 @@ __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &
     if (lane < 16) S.rscale[s][gw * 16 + lane] = S.mscale[ms][gw * 16 + lane];
     if (gw == 0 && lane == 0 && !dry) S.ec[s] = ec;
     if (fp8) {
-      gather_store_fp8(S, kt, ms, ec, gw, lane, v);
+      gather_store_fp8(S, kt, ms, ec, gw, lane, v, ahead ? static_cast<int>((n + 1) % kMetaSlots) : -1);
     } else if (!dry) {
       gather_issue_bf16(S, kt, ms, gw, lane);
       cp_async_wait_all();
@@ -502,7 +503,7 @@ __device__ void gather_role(const MqaTcParams &P, MqaSmem &S, const ChunkRange &
         if (lane == 0) S.abort_flag = 1;
         break;
       }
-      if (fp8) gather_load_fp8(S, static_cast<int>((n + 1) % kMetaSlots), gw, lane, nxt, false);
+      if (fp8) gather_load_fp8(S, static_cast<int>((n + 1) % kMetaSlots), gw, lane, v, false);
     }
   }
   cp_async_wait_all();
@@ -794,29 +795,25 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
   tc_fence_after();
   const int lcs = __ffs(static_cast<int>(cs)) - 1;  // cs is a power of two
   const int Dc = kD >> lcs, runs = Dc / 4, slab = kH * Dc;
-  // warp w reads TMEM lanes of quadrant w % 4, columns 256 (w / 4) .. +255
+  // warp w reads the O rows (TMEM lanes 0..15) of quadrant w % 4, columns 256 (w / 4) ..
+  // +255, 64 at a time: thread t takes head 16 (w % 4) + t % 16, columns col + 32 (t / 16) .. +31
   if (warp < 8) {
-    const int quad = warp & 3, h = quad * 16 + (lane & 15), col0 = (warp >> 2) * 256;
+    const int quad = warp & 3, h = quad * 16 + (lane & 15), col0 = (warp >> 2) * 256 + 32 * (lane >> 4);
     const bool has = cr.lo < cr.hi && !S.abort_flag;
 #pragma unroll 1
-    for (int col = col0; col < col0 + 256; col += 64) {
-      uint32_t o[2][32];
+    for (int c64 = 0; c64 < 256; c64 += 64) {
+      uint32_t o[32];
       if (has) {
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + col, o[0]);
-        tmem_ld32(tmem + (static_cast<uint32_t>(quad * 32) << 16) + col + 32, o[1]);
+        tmem_ld16x2(tmem + (static_cast<uint32_t>(quad * 32) << 16) + (warp >> 2) * 256 + c64, o);
         tmem_ld_wait();
       }
-      if (lane < 16) {
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int i = 0; i < 32; i += 4) {
-            const int d = col + 32 * c + i, q = d >> (9 - lcs);
-            const float4 v = has ? make_float4(__uint_as_float(o[c][i]), __uint_as_float(o[c][i + 1]),
-                                               __uint_as_float(o[c][i + 2]), __uint_as_float(o[c][i + 3]))
-                                 : make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4 *>(&S.rbuf[q * slab + h * Dc + slab_run(h, (d & (Dc - 1)) >> 2) * 4]) = v;
-          }
+      for (int i = 0; i < 32; i += 4) {
+        const int d = col0 + c64 + i, q = d >> (9 - lcs);
+        const float4 v = has ? make_float4(__uint_as_float(o[i]), __uint_as_float(o[i + 1]), __uint_as_float(o[i + 2]),
+                                           __uint_as_float(o[i + 3]))
+                             : make_float4(0.f, 0.f, 0.f, 0.f);
+        *reinterpret_cast<float4 *>(&S.rbuf[q * slab + h * Dc + slab_run(h, (d & (Dc - 1)) >> 2) * 4]) = v;
       }
     }
   }
