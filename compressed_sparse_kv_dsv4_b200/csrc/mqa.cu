@@ -538,7 +538,9 @@ __device__ void mma_role(const MqaLaunch &p, MqaSmem &S, const ChunkRange &cr, u
     tc_fence_after();
     const uint64_t kd = sw128_desc(smem_u32(&S.k[m & 1][0][0]), 16, 1024);
     const uint32_t dt = s_tmem + 64u * static_cast<uint32_t>(m & 1);
-#pragma unroll
+    // (rolled by four: this loop's issue time is the tensor pipe's, and its code is fetched
+    // cold once per launch)
+#pragma unroll 4
     for (int kk = 0; kk < kD / 16; ++kk) {  // descriptor start advances in 16-byte units
       const uint32_t off = ((kk >> 2) * (kH * 128) + (kk & 3) * 32) >> 4;
       const uint32_t offk = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
