@@ -261,8 +261,12 @@ dsv4_status dsv4_indexer_topk_noalloc(const dsv4_indexer_args *args, dsv4_stream
  *   (natural log of the softmax denominator, optional).
  *   softmax_scale <= 0 means 1/sqrt(dim).
  * cache and ring share dim and dtype (F32, BF16 or FP8E4M3). BF16/FP8 caches with dim 512
- * and heads 64 run on the tensor cores (tcgen05, bf16 operands, fp32 accumulation); other
- * shapes run on a CUDA-core kernel. A sequence with no key gets a zero output.
+ * and heads 64 run on the tensor cores (tcgen05; bf16 operands for BF16 caches, fp16
+ * operands holding the exact e4m3 codes with their row scales for FP8 caches; fp32
+ * accumulation); other shapes run on a CUDA-core kernel. A sequence with no key gets a zero
+ * output. The tensor-core path's workspace holds the prepared query and the partial outputs
+ * its thread-block clusters exchange (batch * (cs - 1) * 128 KiB, cs <= 16 the CTAs per
+ * sequence); nothing in it outlives the call.
  */
 typedef struct {
   int32_t batch;
