@@ -626,28 +626,29 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
     }
     __syncthreads();
   };
-  // first pass: also counts the valid keys of the whole sequence
-  pass(24, 0);
-  pick(1 << 30);  // the total, in bcast; the digit is chosen below once k is known
-  total_valid = bcast;
-  kk = total_valid < k ? total_valid : k;
-  need = kk;
-  const bool partial = kk < total_valid;
-  if (partial) {
+  // The radix passes, each lambda called from one place (this code runs once per launch and
+  // is fetched cold, so its length is its cost). The first pass also counts the valid keys
+  // of the whole sequence (bcast): with fewer than k of them every valid key is kept;
+  // otherwise its pick already found the digit of the k-th.
+  bool partial = false;
+  need = k;
+#pragma unroll 1
+  for (int shift = 24, par = 0;; shift -= 8, par ^= 1) {
+    pass(shift, par);
     pick(need);
-    int par = 0;
-    for (int shift = 24;; shift -= 8) {
-      prefix |= static_cast<uint32_t>(sel_digit) << shift;
-      mask |= 0xFFu << shift;
-      need -= sel_above;
-      const int cntd = sel_count;
-      __syncthreads();
-      whole_class = cntd == need;
-      if (whole_class || shift == 0) break;  // the whole class is taken, or the key is exact
-      par ^= 1;
-      pass(shift - 8, par);
-      pick(need);
+    if (shift == 24) {
+      total_valid = bcast;
+      kk = total_valid < k ? total_valid : k;
+      partial = kk < total_valid;
+      if (!partial) break;
     }
+    prefix |= static_cast<uint32_t>(sel_digit) << shift;
+    mask |= 0xFFu << shift;
+    need -= sel_above;
+    const int cntd = sel_count;
+    __syncthreads();
+    whole_class = cntd == need;
+    if (whole_class || shift == 0) break;  // the whole class is taken, or the key is exact
   }
   auto above = [&](uint32_t kv) { return kv != 0u && (!partial || (kv & mask) > prefix); };
   auto in_class = [&](uint32_t kv) { return partial && kv != 0u && (kv & mask) == prefix; };
@@ -698,25 +699,31 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
     }
     return kept;
   };
-  const int kept = walk(false, 0);
-  if (lane == 0) warp_cnt[warp] = kept;
-  __syncthreads();
-  if (tid == 0) {
-    int run = 0;
-    for (int w = 0; w < (NT / 32); ++w) { warp_base[w] = run; run += warp_cnt[w]; }
-    xch[1] = run;
-  }
-  cluster_sync_all();
-  if (warp == 0) {  // lane r reads CTA r
-    const int v = lane < static_cast<int>(cs) ? ld_cluster(&xch[1], lane) : 0;
-    const int before = warp_sum_int(lane < static_cast<int>(rank) ? v : 0), all = warp_sum_int(v);
-    if (lane == 0) {
-      sel_above = before;
-      sel_count = all;
+  // the walk, from one place: counted (pass 0), then, with the counts of the warps before
+  // and of the CTAs before exchanged, written (pass 1)
+#pragma unroll 1
+  for (int wp = 0, at = 0; wp < 2; ++wp) {
+    const int kept = walk(wp == 1, at);
+    if (wp == 1) break;
+    if (lane == 0) warp_cnt[warp] = kept;
+    __syncthreads();
+    if (tid == 0) {
+      int run = 0;
+      for (int w = 0; w < (NT / 32); ++w) { warp_base[w] = run; run += warp_cnt[w]; }
+      xch[1] = run;
     }
+    cluster_sync_all();
+    if (warp == 0) {  // lane r reads CTA r
+      const int v = lane < static_cast<int>(cs) ? ld_cluster(&xch[1], lane) : 0;
+      const int before = warp_sum_int(lane < static_cast<int>(rank) ? v : 0), all = warp_sum_int(v);
+      if (lane == 0) {
+        sel_above = before;
+        sel_count = all;
+      }
+    }
+    __syncthreads();
+    at = sel_above + warp_base[warp];
   }
-  __syncthreads();
-  walk(true, sel_above + warp_base[warp]);
   if (rank == 0) {
     for (int i = sel_count + tid; i < k; i += NT) {
       idx[static_cast<size_t>(b) * k + i] = -1;
