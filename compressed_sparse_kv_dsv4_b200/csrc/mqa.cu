@@ -99,7 +99,7 @@ __device__ __forceinline__ const uint8_t *key_row(const MqaLaunch &p, int b, con
 // ------------------------------------------------------------------------------------
 // tensor-core kernel: one thread-block cluster of cs CTAs per sequence; CTA r takes a
 // contiguous run of the sequence's 64-key chunks, and the cluster merges the CTAs' partial
-// results in distributed shared memory.
+// results through L2 (the workspace) at the end.
 
 constexpr int kH = 64, kD = 512, kCh = 64;
 constexpr int kAtom = kCh * 128;  // one 64-dim column block of a 64-row tile: 8 KB

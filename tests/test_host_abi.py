@@ -82,6 +82,21 @@ def _indexer(**kw):
     return a
 
 
+def test_attention_workspace_covers_the_cluster_exchange(lib):
+    """The tensor-core attention splits each sequence over a cluster of cs CTAs (a power of
+    two up to 16 that keeps the batch within one wave of the 148 SMs) whose partial outputs,
+    (cs - 1) slabs of [64 heads][512 / cs] fp32 per CTA, pass through the workspace; the
+    prepared query (bf16/fp16, [B][64][512]) sits there too. No GPU here: 148 SMs assumed."""
+    for batch, cs in ((1, 16), (2, 16), (9, 16), (10, 8), (32, 4), (37, 4), (40, 2), (74, 2), (75, 1)):
+        a = _mqa(batch=batch)
+        need = lib.dsv4_mqa_workspace_size(C.byref(a))
+        partials = batch * (cs - 1) * 64 * 512 * 4
+        query = batch * 64 * 512 * 2
+        assert need >= partials + query, (batch, need)
+        # nothing else of size: per-sequence scales and (max, sum) pairs, and alignment
+        assert need - partials - query <= batch * (64 * 4 + 16 * 2 * 64 * 4) + 3 * 256, (batch, need)
+
+
 def test_validation_rejects_bad_calls(lib):
     # null argument structs
     assert lib.dsv4_compress(None, None) == A.ERR_INVALID_ARG
