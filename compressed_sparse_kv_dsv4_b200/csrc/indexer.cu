@@ -700,17 +700,33 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
     return kept;
   };
   // the walk, from one place: counted (pass 0), then, with the counts of the warps before
-  // and of the CTAs before exchanged, written (pass 1)
+  // and of the CTAs before exchanged, written (pass 1). When the whole class is kept (the
+  // usual case) a warp's count needs no ranks: it is the number of its keys kept.
 #pragma unroll 1
   for (int wp = 0, at = 0; wp < 2; ++wp) {
-    const int kept = walk(wp == 1, at);
+    int kept;
+    if (wp == 0 && whole_class) {
+      int c = 0;
+#pragma unroll
+      for (int r = 0; r < KPT; ++r) c += (above(key[r]) || in_class(key[r])) ? 1 : 0;
+      kept = warp_sum_int(c);
+    } else {
+      kept = walk(wp == 1, at);
+    }
     if (wp == 1) break;
     if (lane == 0) warp_cnt[warp] = kept;
     __syncthreads();
-    if (tid == 0) {
-      int run = 0;
-      for (int w = 0; w < (NT / 32); ++w) { warp_base[w] = run; run += warp_cnt[w]; }
-      xch[1] = run;
+    if (warp == 0) {  // exclusive scan of the warps' counts, lane w for warp w
+      static_assert(NT / 32 <= 32, "one lane per warp");
+      const int v = lane < NT / 32 ? warp_cnt[lane] : 0;
+      int incl = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += u;
+      }
+      if (lane < NT / 32) warp_base[lane] = incl - v;
+      if (lane == 31) xch[1] = incl;
     }
     cluster_sync_all();
     if (warp == 0) {  // lane r reads CTA r
