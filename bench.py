@@ -213,6 +213,31 @@ def indexer_traffic():
     return rec.get("dram_bytes_per_launch")
 
 
+STEP_INPUTS = ("kv", "gate", "idx_kv", "idx_gate", "q", "q_idx", "q_idx_scale", "w")
+
+
+def pack_step_inputs(ds, dev):
+    """A copy of step ds whose input tensors are views into one device buffer (each at a
+    256-byte offset), with a pinned host mirror of that buffer: (host, device, step)."""
+    import dataclasses
+
+    import torch
+
+    offs, size = [], 0
+    for n in STEP_INPUTS:
+        t = getattr(ds, n)
+        offs.append(size)
+        size += (t.numel() * t.element_size() + 255) // 256 * 256
+    dbuf = torch.zeros(size, dtype=torch.uint8, device=dev)
+    views = {}
+    for n, off in zip(STEP_INPUTS, offs):
+        t = getattr(ds, n)
+        v = dbuf[off:off + t.numel() * t.element_size()].view(t.dtype).view(t.shape)
+        v.copy_(t)
+        views[n] = v
+    return dbuf.cpu().pin_memory() if dbuf.is_cuda else dbuf.clone(), dbuf, dataclasses.replace(ds, **views)
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_ours(args):
     import torch
@@ -293,32 +318,34 @@ def run_ours(args):
     torch.cuda.synchronize()
     ix_ms = float(np.mean([e0[j].elapsed_time(e1[j]) for j in range(k_iters)]))
 
-    # ---- end to end through the public API: inputs from pinned host memory, output back
-    host_in = []
-    for ds in dsteps:
-        tensors = [ds.kv, ds.gate, ds.idx_kv, ds.idx_gate, ds.q, ds.q_idx, ds.q_idx_scale, ds.w]
-        host_in.append([t.cpu().pin_memory() for t in tensors])
-    out_host = torch.empty(dsteps[0].out.shape, dtype=dsteps[0].out.dtype).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host_in[0]) + B_PER_GPU * 4
-    d2h = out_host.numel() * out_host.element_size()
+    # ---- end to end through the public API: inputs from pinned host memory, output back.
+    # A step's eight input tensors live in one device buffer (views at 256-byte offsets) with
+    # a pinned host mirror of the same layout, so they cross in one copy; the positions in a
+    # second one.
     pos_host = pos_table.cpu().pin_memory()
     pos_dev = torch.empty(B_PER_GPU, dtype=torch.int32, device=dev)
+    packed = [pack_step_inputs(ds, dev) for ds in dsteps]  # (host mirror, device buffer, step)
+    e2e_structs = []
+    for hbuf, dbuf, ds_e in packed:
+        S = ds_e.struct()
+        S.pos = pos_dev.data_ptr()
+        e2e_structs.append(S)
+    out_host = torch.empty(dsteps[0].out.shape, dtype=dsteps[0].out.dtype).pin_memory()
+    h2d = packed[0][0].numel() + B_PER_GPU * 4
+    d2h = out_host.numel() * out_host.element_size()
     e2e_steps = min(args.steps, 200)
     f0 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     f1 = [torch.cuda.Event(enable_timing=True) for _ in range(e2e_steps)]
     for j in range(e2e_steps):
         i = args.warmup + j
-        ds = dsteps[i % N_INPUT_SETS]
-        S = structs[i]
-        S.pos = pos_dev.data_ptr()
+        hbuf, dbuf, ds_e = packed[i % N_INPUT_SETS]
         flush.fill_(j & 0xFF)
         f0[j].record(stream)
-        for dst, src in zip([ds.kv, ds.gate, ds.idx_kv, ds.idx_gate, ds.q, ds.q_idx, ds.q_idx_scale, ds.w],
-                            host_in[i % N_INPUT_SETS]):
-            dst.copy_(src, non_blocking=True)
+        dbuf.copy_(hbuf, non_blocking=True)
         pos_dev.copy_(pos_host[i], non_blocking=True)
-        step(i)
-        out_host.copy_(ds.out, non_blocking=True)
+        A.check("dsv4_hybrid_decode", lib.dsv4_hybrid_decode(C.byref(L), C.byref(e2e_structs[i % N_INPUT_SETS]),
+                                                              C.c_void_p(ws.data_ptr()), ws.numel(), sh))
+        out_host.copy_(ds_e.out, non_blocking=True)
         f1[j].record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(float(np.mean([f0[j].elapsed_time(f1[j]) for j in range(e2e_steps)])), world)
