@@ -147,7 +147,7 @@ struct TcParams {
 constexpr int kPerPage = 64;
 constexpr int kStageTiles = 2;
 constexpr int kStagePages = kStageTiles * kTile / kPerPage;  // 4
-constexpr int kSlots = 8;        // key-scale ring, one slot per stage
+constexpr int kSlots = 8;        // ring of the stages' page rows, one slot per stage
 constexpr int kBatchStages = 32 / kStagePages;  // stages whose page ids one warp load covers (8)
 constexpr int kGroups = 2;       // epilogue warp groups, alternating stages
 constexpr int kGroupThreads = 128;
@@ -157,7 +157,7 @@ template <int H, int kStages>  // H in {32, 64}; kStages key stages of 32 KB in 
 struct alignas(1024) TcSmem {
   uint8_t stage[kStages][kStageTiles][kTile * kRowBytes];  // key tiles (rows = entries)
   uint8_t q[2][H * kRowBytes];
-  float sig[kSlots][kStageTiles * kTile];  // key scales of each stage (0: no key)
+  int spage[kSlots][kStagePages];          // first key-scale row of each page of a stage (or past the pool: none)
   float coef[kGroups * 4][H];              // per epilogue warp: w_h * scale_q[h] of its sequence
   uint64_t full[kStages], empty[kStages], sfull[kSlots], sempty[kSlots];
   uint64_t tfull[kGroups], tempty[kGroups], qfull[2], qempty[2];
@@ -327,22 +327,11 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
         if (p.after_append && seg_end && lt0 + nt == prefix[sb + 1] - prefix[sb]) pdl_wait();
         if (k >= kSlots && !mbar_wait(&S.sempty[slot], static_cast<uint32_t>((k / kSlots - 1) & 1), &S.abort_flag))
           ok = 0;
-        if (ok) {  // key scales: one 256-byte bulk copy per valid page, zeros for the others
-          uint32_t bytes = 0;
+        if (ok) {  // the pages' rows; the epilogue threads load their keys' scales themselves
+          // (as four 256-byte bulk copies per stage they held up the producer's issue)
 #pragma unroll
-          for (int i = 0; i < kStagePages; ++i) bytes += rows[i] != oob_row ? kPerPage * 4 : 0;
-          float4 *z = reinterpret_cast<float4 *>(S.sig[slot]);
-#pragma unroll
-          for (int i = 0; i < kStagePages; ++i)
-            if (rows[i] == oob_row)
-              for (int u = 0; u < kPerPage / 4; ++u) z[i * kPerPage / 4 + u] = make_float4(0.f, 0.f, 0.f, 0.f);
-          fence_proxy_async_smem();  // the slot is written by bulk copies too
-          mbar_arrive_expect_tx(&S.sfull[slot], bytes);
-#pragma unroll
-          for (int i = 0; i < kStagePages; ++i)
-            if (rows[i] != oob_row)
-              bulk_load(&S.sig[slot][i * kPerPage], p.k_scales + static_cast<size_t>(rows[i]), kPerPage * 4,
-                        &S.sfull[slot]);
+          for (int i = 0; i < kStagePages; ++i) S.spage[slot][i] = rows[i];
+          mbar_arrive(&S.sfull[slot]);
         }
         if (ok && new_seg) {
           ++seg;
@@ -415,6 +404,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
     const int gi = (warp - 2) / 4;
     const int quad = warp & 3;
     const int row = quad * 32 + lane;
+    const int oob_row = p.num_pages * kPerPage;  // (a page past the pool: no key)
     float *coef = S.coef[warp - 2];
     StageIter it;
     it.init(prefix, p.B, t0, t1);
@@ -435,6 +425,13 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
       }
       const int slot = static_cast<int>(kk % kSlots);
       bool ok = mbar_wait(&S.sfull[slot], static_cast<uint32_t>((kk / kSlots) & 1), &S.abort_flag);
+      // this thread's key scales (0: no key), in flight while the MMA finishes
+      float scl[kStageTiles];
+#pragma unroll
+      for (int t = 0; t < kStageTiles; ++t) {
+        const int base = ok ? S.spage[slot][t * (kTile / kPerPage) + row / kPerPage] : oob_row;
+        scl[t] = (t < nt && base != oob_row) ? __ldg(p.k_scales + static_cast<size_t>(base) + row % kPerPage) : 0.f;
+      }
       ok = mbar_wait(&S.tfull[gi], static_cast<uint32_t>((kk / kGroups) & 1), &S.abort_flag) && ok;
       if (!__all_sync(0xFFFFFFFFu, ok)) {
         if (lane == 0) S.abort_flag = 1;
@@ -451,7 +448,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
           const uint32_t ta = tmem + (static_cast<uint32_t>(quad * 32) << 16) + (gi * kStageTiles + t) * H;
           tmem_ld32(ta, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
           if (H > 32) tmem_ld32(ta + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32 % H]));
-          const float sc = S.sig[slot][t * kTile + row];
+          const float sc = scl[t];
           tmem_ld_wait();
           float part[4] = {0.f, 0.f, 0.f, 0.f};  // 4 short chains, not one of H
 #pragma unroll
