@@ -56,6 +56,26 @@ def algorithmic_bytes_per_seq(n_c: int, out_bytes: int = 2) -> dict:
     return dict(indexer=idx + qidx, attention=attn, updates=upd, total=idx + qidx + attn + upd)
 
 
+def c128_bytes_per_seq(n_c: int, D: int = 512, H: int = 64, W: int = 128) -> int:
+    """Bytes one sequence's dense C128 layer step must move (bf16 caches): every visible entry
+    and the W window rows (2D bytes each), the bf16 query and output, and the updates (the new
+    token's kv and gate read, the state slot (float32 kv + gate) and the window row written)."""
+    return (n_c + W) * 2 * D + 2 * H * D * 2 + (2 * D * 2 + 2 * D * 4 + 2 * D)
+
+
+def c4_step_bytes_per_seq(n_c: int) -> int:
+    return algorithmic_bytes_per_seq(n_c)["total"]
+
+
+def prefill_bytes(T: int, B: int, m: int, D: int = 512, cache_bytes_per_row: int = 1024) -> int:
+    """Bytes one compressor must move for a prefill of T bf16 tokens over B sequences of T/B
+    tokens each (starting at position 0): the kv and gate rows read (2D bf16 each), one
+    cache row per completed block written, and the ring state of each sequence's last m
+    tokens written (float32 kv + gate)."""
+    per = T // B
+    return T * 2 * D * 2 + B * (per // m) * cache_bytes_per_row + B * min(m, per) * 2 * D * 4
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     def __init__(self, gpu_id: str):
@@ -238,6 +258,118 @@ def pack_step_inputs(ds, dev):
     return dbuf.cpu().pin_memory() if dbuf.is_cuda else dbuf.clone(), dbuf, dataclasses.replace(ds, **views)
 
 
+# ----------------------------------------------------------------------------- extra legs
+def event_mean_ms(stream, fn, iters: int, flush, warm: int = 3) -> float:
+    """Mean duration of fn() over `iters` runs, CUDA events on `stream`, L2 flushed before each."""
+    import torch
+
+    for j in range(warm):
+        flush.fill_(j & 0xFF)
+        fn(j)
+    torch.cuda.synchronize()
+    e0 = [torch.cuda.Event(enable_timing=True) for _ in range(iters)]
+    e1 = [torch.cuda.Event(enable_timing=True) for _ in range(iters)]
+    for j in range(iters):
+        flush.fill_(j & 0xFF)
+        e0[j].record(stream)
+        fn(warm + j)
+        e1[j].record(stream)
+    torch.cuda.synchronize()
+    return float(np.mean([e0[j].elapsed_time(e1[j]) for j in range(iters)]))
+
+
+def leg_compress_prefill(lib, dev, stream, flush, hbm_peak: float, iters: int = 20) -> dict:
+    """The compressor prefill workload: 8 x 4096 bf16 tokens (D = 512) into a C4 and a C128
+    compressor (pool + RMSNorm + RoPE + bf16 insert + ring state), each dsv4_compress call
+    timed alone and both together."""
+    import torch
+
+    import compressed_sparse_kv_dsv4_b200 as dsv4
+    from compressed_sparse_kv_dsv4_b200 import _abi as A
+    import synthetic as W
+
+    wl = W.compressor_prefill()
+    B, T = wl.start_pos.shape[0], int(wl.cu_seqlens[-1])
+    cu = torch.from_numpy(wl.cu_seqlens).to(dev)
+    sp = torch.from_numpy(wl.start_pos).to(dev)
+    calls = []
+    for la, kv, gate in ((wl.layer4, wl.kv4, wl.gate4), (wl.layer128, wl.kv128, wl.gate128)):
+        spec = la.spec
+        dl = dsv4.DeviceLayer.from_arrays(la, dev)
+        kvd, gd = dsv4.to_device_codes(kv, "bf16", dev), dsv4.to_device_codes(gate, "bf16", dev)
+        a = A.CompressArgs(batch=B, total_tokens=T, kv=kvd.data_ptr(), gate=gd.data_ptr(), kv_dtype=A.BF16,
+                           cu_seqlens=cu.data_ptr(), start_pos=sp.data_ptr(), gamma=dl.gamma.data_ptr(), eps=spec.eps,
+                           rope=A.Rope(spec.rope_dims, spec.rope_base), state=dl.state.struct(),
+                           cache=dl.cache.struct(), d_status=None)
+        calls.append((spec.m, a, (dl, kvd, gd)))
+    sh = C.c_void_p(stream.cuda_stream)
+    out = {"workload": "compressor_prefill_8x4096", "tokens": T, "kv_dim": 512, "cache": "bf16",
+           "input": "bf16 kv + per-channel gate"}
+    total_bytes, total_ms = 0, 0.0
+    for m, a, _keep in calls:
+        ms = event_mean_ms(stream, lambda j, a=a: A.check("dsv4_compress", lib.dsv4_compress(C.byref(a), sh)),
+                           iters, flush)
+        byts = prefill_bytes(T, B, m)
+        out[f"c{m}"] = {"ms": round(ms, 5), "algorithmic_bytes": byts, "gbs": round(byts / ms / 1e6, 1),
+                        "frac": round(byts / ms / 1e6 / hbm_peak, 4)}
+        total_bytes += byts
+        total_ms += ms
+    both = event_mean_ms(stream, lambda j: [A.check("dsv4_compress", lib.dsv4_compress(C.byref(a), sh))
+                                            for _m, a, _k in calls], iters, flush)
+    out["both"] = {"ms": round(both, 5), "algorithmic_bytes": total_bytes, "gbs": round(total_bytes / both / 1e6, 1),
+                   "frac": round(total_bytes / both / 1e6 / hbm_peak, 4), "tokens_per_s": round(T / (both * 1e-3), 1)}
+    return out
+
+
+def leg_stack_1m(lib, dev, stream, flush, hbm_peak: float, steps: int = 16) -> dict:
+    """The 1M-context mixed stack: two C4 layers (262144 fp8 entries, top-512) and two C128
+    layers (8192 bf16 entries), 4 sequences; one step = the four layers' dsv4_hybrid_decode
+    calls, each sequence appending one token per layer. `steps` consecutive steps after three
+    warm-up steps, the L2 flushed before each."""
+    import torch
+
+    import compressed_sparse_kv_dsv4_b200 as dsv4
+    from compressed_sparse_kv_dsv4_b200 import _abi as A
+    import synthetic as W
+
+    B, ctx = 4, 1 << 20
+    layers, step_sets = W.stack_1m(B=B, context=ctx, steps=1)
+    dls = [dsv4.DeviceLayer.from_arrays(la, dev) for la in layers]
+    dss = [dsv4.DeviceStep.from_arrays(la.spec, ss[0], dev) for la, ss in zip(layers, step_sets)]
+    total = steps + 3
+    pos = torch.tensor([[ctx + i] * B for i in range(total)], dtype=torch.int32, device=dev)
+    wss = [dl.workspace(B) for dl in dls]
+    Ls = [dl.struct() for dl in dls]
+    Ss = []
+    for ds in dss:
+        row = []
+        for i in range(total):
+            S = ds.struct()
+            S.pos = pos[i].data_ptr()
+            row.append(S)
+        Ss.append(row)
+    sh = C.c_void_p(stream.cuda_stream)
+
+    def step(i):
+        for li in range(4):
+            A.check("dsv4_hybrid_decode", lib.dsv4_hybrid_decode(C.byref(Ls[li]), C.byref(Ss[li][i]),
+                                                                  C.c_void_p(wss[li].data_ptr()), wss[li].numel(), sh))
+
+    n0 = lib.dsv4_launch_count()
+    ms = event_mean_ms(stream, step, steps, flush, warm=3)
+    launches = (lib.dsv4_launch_count() - n0) // total
+    status = [int(ds.d_status.item()) for ds in dss]
+    byts = B * (2 * c4_step_bytes_per_seq(ctx // 4) + 2 * c128_bytes_per_seq(ctx // 128))
+    res = {"workload": "stack_1m", "batch": B, "context": ctx, "layers": "C4, C128, C4, C128", "steps": steps,
+           "ms_per_step": round(ms, 5), "tokens_per_s": round(B / (ms * 1e-3), 1), "algorithmic_bytes": byts,
+           "gbs": round(byts / ms / 1e6, 1), "pct_of_8tbs": round(100 * byts / ms / 1e6 / 8000.0, 1),
+           "frac": round(byts / ms / 1e6 / hbm_peak, 4), "launches_per_step": launches, "device_status": status,
+           "l2": "flushed between steps (256 MiB write)"}
+    del dls, dss, wss
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_ours(args):
     import torch
@@ -283,11 +415,13 @@ def run_ours(args):
         barrier(world)
         torch.cuda.synchronize()
         t_a = time.time()
+        launches0 = lib.dsv4_launch_count()
         for j in range(args.steps):
             flush.fill_(j & 0xFF)
             ev0[j].record(stream)
             step(args.warmup + j)
             ev1[j].record(stream)
+        launches = lib.dsv4_launch_count() - launches0
         torch.cuda.synchronize()
         barrier(world)
         t_b = time.time()
@@ -384,15 +518,19 @@ def run_ours(args):
         "hbm": {"step_algorithmic_bytes": step_bytes, "achieved_gbs": round(step_gbs, 1),
                 "pct_of_8tbs": round(100 * step_gbs / 8000.0, 1),
                 "pct_of_measured_copy": round(100 * step_gbs / hbm_peak, 1)},
-        "roofline": {"kernel": "indexer_tc_kernel (+ top-k select)", "bound": "hbm", "achieved": round(ix_gbs, 1),
+        "roofline": {"kernel": "dsv4_indexer_topk call: indexer_tc_kernel + topk_scores_kernel", "bound": "hbm",
+                     "achieved": round(ix_gbs, 1),
                      "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s", "frac": round(ix_gbs / hbm_peak, 4),
                      "traffic": traffic, "algorithmic_bytes_per_launch": ix_bytes, "launch_ms": round(ix_ms, 5)},
         "e2e": {"value": round(job_tokens_per_s(world, e2e_ms), 1), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": round(e2e_ms, 5)},
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": int(launches),
         "clocks": clk.summary(t_a, t_b),
         "device_status": status,
     }
+    if world == 1 and not args.no_extra:
+        line["compress_prefill"] = leg_compress_prefill(lib, dev, stream, flush, hbm_peak)
+        line["stack_1m"] = leg_stack_1m(lib, dev, stream, flush, hbm_peak)
     if world == 1 and not args.no_cpu_baseline:
         seqs, dt = oracle_sample(la, sets, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(seqs / dt, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
@@ -438,6 +576,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the compressor-prefill and 1M-stack legs")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -90,6 +90,7 @@ EXPORTS = {
     "dsv4_hybrid_decode": (C.c_int, [C.POINTER(Layer), C.POINTER(Step), p, C.c_size_t, p]),
     "dsv4_status_string": (C.c_char_p, [C.c_int]),
     "dsv4_abi_version": (i32, []),
+    "dsv4_launch_count": (C.c_uint64, []),
     "dsv4_layer_state_bytes": (C.c_uint64, [C.c_uint64, i32, i32, i32, i32, i32]),
 }
 

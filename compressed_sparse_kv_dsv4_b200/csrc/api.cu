@@ -4,6 +4,7 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 #include <vector>
 
@@ -25,6 +26,12 @@ int sm_count() {
   }
   return cache[dev];
 }
+
+namespace {
+std::atomic<uint64_t> g_launches{0};
+}
+
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 }  // namespace dsv4
 
@@ -86,6 +93,8 @@ const char *dsv4_status_string(dsv4_status s) {
 }
 
 int32_t dsv4_abi_version(void) { return DSV4_ABI_VERSION; }
+
+uint64_t dsv4_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 uint64_t dsv4_layer_state_bytes(uint64_t context, int32_t m, int32_t entry_width, int32_t window, int32_t window_width,
                                 int32_t bytes_per_value) {

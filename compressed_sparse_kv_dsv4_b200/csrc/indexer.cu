@@ -6,14 +6,15 @@
 //
 // Tensor-core path (fp8 keys, 128-dim, the C4 layers): a persistent kernel, one CTA per
 // SM, over the flattened (sequence, 128-entry tile) space, in stages of up to two tiles of
-// one sequence. Warp 0 streams key pages with TMA (8 KB boxes, 128B swizzle) into a
-// 5-stage ring, with the block-table entries fetched a batch of 8 stages ahead and the key
-// scales copied by cp.async; warp 1 issues tcgen05.mma kind::f8f6f4 (M = 128 entries,
-// N = H heads, K = 128) into two TMEM accumulator sets; two groups of four warps take
-// alternate stages, read their accumulators back (tcgen05.ld), apply ReLU, the per-head
-// weights w_h * scale_q[h] and the per-entry key scale, and store every score (4 bytes per
-// entry, coalesced). A second kernel selects the top k of each sequence from the scores
-// in shared memory (radix select), writing them in ascending entry order.
+// one sequence. Warp 0 streams key pages with TMA (8 KB boxes, 128B swizzle) into a ring of
+// 5 or 6 stages, with the block-table entries fetched a batch of 8 stages ahead, and hands
+// each stage's page rows to the epilogue; warp 1 issues tcgen05.mma kind::f8f6f4 (M = 128
+// entries, N = H heads, K = 128) into two TMEM accumulator sets; two groups of four warps
+// take alternate stages, load their keys' scales, read their accumulators back
+// (tcgen05.ld), apply ReLU, the per-head weights w_h * scale_q[h] and the per-entry key
+// scale, and store every score (4 bytes per entry, coalesced). A second kernel selects the
+// top k of each sequence from the scores (a cluster radix select over registers), writing
+// them in ascending entry order.
 //
 // The scale handling relies on ReLU(a * x) = a * ReLU(x) for a > 0:
 //   s_j = scale_k[j] * sum_h (w_h * scale_q[h]) * ReLU(q8_h . k8_j).
@@ -285,9 +286,9 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
 
   if (warp == 0) {
     // ---------------- producer. Lane 0 issues the key TMA of stage k (one box per 64-row
-    // page; an invalid page, or one past the visible entries, takes a zero-filled
-    // out-of-range box) and one bulk copy of the key scales per page, both completing as
-    // transaction bytes on their barriers.
+    // page, completing as transaction bytes on the stage's barrier; an invalid page, or one
+    // past the visible entries, takes a zero-filled out-of-range box) and stores the stage's
+    // page rows in a small ring for the epilogue, which loads the keys' scales itself.
     const int oob_row = p.num_pages * kPerPage;
     StageIter it, ahead;
     it.init(prefix, p.B, t0, t1);
@@ -430,7 +431,9 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
 #pragma unroll
       for (int t = 0; t < kStageTiles; ++t) {
         const int base = ok ? S.spage[slot][t * (kTile / kPerPage) + row / kPerPage] : oob_row;
-        scl[t] = (t < nt && base != oob_row) ? __ldg(p.k_scales + static_cast<size_t>(base) + row % kPerPage) : 0.f;
+        // (a coherent L2 load, not the read-only path: after a decode-step append the last
+        // stage's scale was written by the kernel this one overlaps)
+        scl[t] = (t < nt && base != oob_row) ? __ldcg(p.k_scales + static_cast<size_t>(base) + row % kPerPage) : 0.f;
       }
       ok = mbar_wait(&S.tfull[gi], static_cast<uint32_t>((kk / kGroups) & 1), &S.abort_flag) && ok;
       if (!__all_sync(0xFFFFFFFFu, ok)) {
@@ -479,6 +482,11 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   }
 
   if (tid == 0 && S.abort_flag) report(p.d_status, DSV4_DEV_TIMEOUT);
+  // After an append only the producers of stages holding a sequence's last tile waited for
+  // the kernel before; a CTA with no such stage (or a step where no sequence has a tile at
+  // all) waits here, so that this grid completes only after its predecessor: the kernels
+  // after it rely on that chain for the prologue's window and cache writes.
+  if (p.after_append && tid == 0) pdl_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {

@@ -174,6 +174,9 @@ cudaError_t launch_mqa_attention(const MqaLaunch &p, void *ws, cudaStream_t st);
 
 inline size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
+// Kernels this library has launched in the process (every launch goes through launch_pdl).
+void count_launch();
+
 // Launch with programmatic stream serialization (the kernel's pdl_wait() orders it after
 // its predecessor), optionally as clusters of `cluster` CTAs along x.
 template <typename... KArgs, typename... Args>
@@ -197,7 +200,9 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
   }
   cfg.attrs = attr;
   cfg.numAttrs = n;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+  if (e == cudaSuccess) count_launch();
+  return e;
 }
 
 }  // namespace dsv4

@@ -358,6 +358,11 @@ const char *dsv4_status_string(dsv4_status status);
 /* DSV4_ABI_VERSION of the loaded library. */
 int32_t dsv4_abi_version(void);
 
+/* Number of kernels this library has launched in the calling process so far (every device
+ * launch of every entry point, counted on the host when the launch is accepted). The
+ * difference of two readings is the number of kernels a stretch of calls launched. */
+uint64_t dsv4_launch_count(void);
+
 /* Bytes of cache state one layer keeps for one sequence of `context` tokens (vLLM
  * "four moves" sizing: compressed entries of entry_width values at rate m plus `window`
  * raw rows of window_width values), at bytes_per_value bytes per value. */

@@ -13,7 +13,7 @@ import compressed_sparse_kv_dsv4_b200 as dsv4
 import oracle.dsv4_oracle as O
 import synthetic as W
 from oracle import adapters as OA
-from tests.parity import check_output, check_topk, decode_out, input_class, require_gpu
+from tests.parity import check_output, check_topk, codes_close, decode_out, input_class, require_gpu
 
 pytestmark = pytest.mark.gpu
 
@@ -21,30 +21,6 @@ pytestmark = pytest.mark.gpu
 @pytest.fixture(scope="module", autouse=True)
 def _gpu():
     require_gpu()
-
-
-def _codes_close(gpu_codes, ref_codes, gpu_scales, ref_scales, dtype, ctx):
-    """Rows rounded into a cache dtype by the two sides from slightly different
-    float32 values: equal, or one rounding step apart."""
-    if dtype == "f32":
-        g = np.asarray(gpu_codes, np.float64)
-        r = np.asarray(ref_codes, np.float64)
-        assert np.max(np.abs(g - r)) <= 2e-5 * max(1.0, np.max(np.abs(r))), ctx
-        return
-    if dtype == "bf16":
-        g, r = O.bf16_decode(gpu_codes), O.bf16_decode(ref_codes)
-        assert np.all(np.abs(g - r) <= 2.0 ** -7 * np.abs(r) + 1e-30), ctx
-        return
-    gs, rs = np.asarray(gpu_scales, np.float64), np.asarray(ref_scales, np.float64)
-    assert np.all(np.abs(gs - rs) <= 1e-6 * rs), f"{ctx}: scales"
-    g = np.asarray(gpu_codes).astype(np.int32)
-    r = np.asarray(ref_codes).astype(np.int32)
-    same_sign = (g & 0x80) == (r & 0x80)
-    step = np.abs((g & 0x7F) - (r & 0x7F))
-    zero = ((g & 0x7F) == 0) & ((r & 0x7F) <= 1) | ((r & 0x7F) == 0) & ((g & 0x7F) <= 1)
-    ok = (same_sign & (step <= 1)) | zero
-    assert np.all(ok), f"{ctx}: fp8 codes more than one step apart"
-    assert np.mean(g != r) < 0.01, f"{ctx}: too many fp8 rounding differences"
 
 
 # ---------------------------------------------------------------------------- compressor
@@ -82,7 +58,7 @@ def test_compress_prefill_matches_oracle(m, cache_dtype, D):
     for s in range(B):
         for b in range(start[s] // m, (start[s] + lens[s]) // m):
             pg, sl = ol.main_cache.locate(s, b)
-            _codes_close(pages[pg, sl], ol.main_cache.pages[pg, sl], scales[pg, sl], ol.main_cache.scales[pg, sl],
+            codes_close(pages[pg, sl], ol.main_cache.pages[pg, sl], scales[pg, sl], ol.main_cache.scales[pg, sl],
                          cache_dtype, f"seq {s} block {b}")
     # rows that no block wrote keep their bytes
     untouched = np.ones(pages.shape[:2], bool)
@@ -117,6 +93,58 @@ def test_compress_prefill_equals_token_by_token():
             assert np.array_equal(a, b)
 
 
+@pytest.mark.slow
+@pytest.mark.parametrize("cache_dtype", ["bf16", "fp8"])
+def test_compressor_prefill_full_size(cache_dtype):
+    """The compressor prefill workload at full size: 8 sequences of 4096 bf16 tokens (D = 512)
+    into a C4 and a C128 compressor. Checked against the oracle: every C128 entry (256), a
+    seeded sample of 320 C4 entries (every sequence's first and last among them), and both
+    state rings, which end holding each sequence's last block of inputs."""
+    wl = W.compressor_prefill(cache_dtype=cache_dtype)
+    B = wl.start_pos.shape[0]
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    cu = torch.from_numpy(wl.cu_seqlens).cuda()
+    sp = torch.from_numpy(wl.start_pos).cuda()
+    rng = np.random.default_rng(71)
+    for la, kv, gate in ((wl.layer4, wl.kv4, wl.gate4), (wl.layer128, wl.kv128, wl.gate128)):
+        spec = la.spec
+        m = spec.m
+        dl = dsv4.DeviceLayer.from_arrays(la)
+        dsv4.compress(dsv4.to_device_codes(kv, "bf16", "cuda"), dsv4.to_device_codes(gate, "bf16", "cuda"), cu, sp,
+                      dl.state, dl.cache, dl.gamma, kv_dtype="bf16", eps=spec.eps, rope_dims=spec.rope_dims,
+                      rope_base=spec.rope_base, d_status=status)
+        torch.cuda.synchronize()
+        assert status.item() == 0
+        ol = OA.layer_state(la)
+        pages = dsv4.to_numpy_codes(dl.cache.pages, cache_dtype)
+        scales = dl.cache.scales.cpu().numpy()
+        n_blocks = [(int(wl.cu_seqlens[s + 1] - wl.cu_seqlens[s]) + int(wl.start_pos[s])) // m for s in range(B)]
+        if m == 128:
+            pairs = [(s, b) for s in range(B) for b in range(n_blocks[s])]
+        else:
+            pairs = {(s, b) for s in range(B) for b in (0, n_blocks[s] - 1)}
+            while len(pairs) < 320:
+                s = int(rng.integers(B))
+                pairs.add((s, int(rng.integers(n_blocks[s]))))
+            pairs = sorted(pairs)
+        for s, b in pairs:
+            t0 = int(wl.cu_seqlens[s]) + b * m - int(wl.start_pos[s])
+            e = O.compress_block(OA.decode_input(kv[t0:t0 + m], "bf16"), OA.decode_input(gate[t0:t0 + m], "bf16"),
+                                 b, m, ol.gamma, spec.eps, spec.rope_dims, spec.rope_base)
+            codes, scale, _ = O.store(e, cache_dtype)
+            pg, sl = ol.main_cache.locate(s, b)
+            codes_close(pages[pg, sl], codes, scales[pg, sl], scale, cache_dtype, f"m={m} seq {s} entry {b}",
+                        max_frac=0.05)
+        ring = dl.state.buf.cpu().numpy()
+        for s in range(B):
+            t_end = int(wl.cu_seqlens[s + 1])
+            for i in range(m):  # the ring slot of each of the last m positions holds its inputs
+                t = t_end - m + i
+                p = t - int(wl.cu_seqlens[s]) + int(wl.start_pos[s])
+                want = np.concatenate([OA.decode_input(kv[t], "bf16"), OA.decode_input(gate[t], "bf16")])
+                assert np.array_equal(ring[s, p % m], want.astype(np.float32)), f"m={m} seq {s} ring slot {p % m}"
+
+
 @pytest.mark.parametrize("dtype,D", [("fp8", 512), ("bf16", 512), ("f32", 128)])
 def test_swa_insert_matches_oracle(dtype, D):
     rng = W.rng_for(13)
@@ -143,7 +171,7 @@ def test_swa_insert_matches_oracle(dtype, D):
     sc = dl.ring.scales.cpu().numpy()
     for s in range(3):
         for i in range(128):
-            _codes_close(rows[s, i], ol.window.rows[s, i], sc[s, i], ol.window.scales[s, i], dtype, f"seq {s} slot {i}")
+            codes_close(rows[s, i], ol.window.rows[s, i], sc[s, i], ol.window.scales[s, i], dtype, f"seq {s} slot {i}")
 
 
 # ---------------------------------------------------------------------------- indexer
@@ -253,15 +281,17 @@ def _ref_attention(ol, qd, st, s, sel, spec):
     return o, lse
 
 
-def test_mqa_tensor_core_dense_bf16():
+@pytest.mark.parametrize("out_dtype", ["f32", "bf16"])
+def test_mqa_tensor_core_dense_bf16(out_dtype):
     spec = W.C128_SPEC
     pos = [3, 70000, 65536]           # a truncated window, then full ones
     n_entries = [0, 300, 513]          # n_c = 0, then ragged chunk tails
-    out, lse, status, ol, qd, st = _mqa_case(spec, 3, pos, n_entries, value_std=1 / np.sqrt(512))
+    out, lse, status, ol, qd, st = _mqa_case(spec, 3, pos, n_entries, value_std=1 / np.sqrt(512),
+                                             out_dtype=out_dtype)
     assert status == 0
     for s in range(3):
         o, l = _ref_attention(ol, qd, st, s, np.arange(n_entries[s]), spec)
-        check_output(out[s], o, "lowp", f"seq {s}", stored_bf16=True)
+        check_output(out[s], o, "lowp", f"seq {s}", out_dtype=out_dtype)
         assert np.max(np.abs(lse[s] - l)) < 2e-2
 
 
@@ -278,7 +308,7 @@ def test_mqa_tensor_core_sparse_fp8_with_padding_and_bad_index():
         for s in range(B):
             sel = [j for j in idx[s] if 0 <= j < n_c]
             o, l = _ref_attention(ol, qd, st, s, sel, spec)
-            check_output(out[s], o, "lowp", f"seq {s} out {out_dtype}", stored_bf16=out_dtype == "bf16")
+            check_output(out[s], o, "lowp", f"seq {s} out {out_dtype}", out_dtype=out_dtype)
             assert np.max(np.abs(lse[s] - l)) < 2e-2
 
 
