@@ -295,7 +295,7 @@ struct HybridPlan {
   IndexerLaunch ix;
   MqaLaunch mq;
   bool c4;
-  size_t idx_bytes, ix_bytes, mq_bytes;
+  size_t idx_bytes, ix_bytes, mq_bytes;  // workspace: selected entries, indexer, attention
 };
 
 dsv4_status hybrid_plan(const dsv4_layer *L, const dsv4_step *S, int32_t batch, HybridPlan *hp) {
@@ -466,21 +466,37 @@ dsv4_status dsv4_hybrid_decode(const dsv4_layer *layer, const dsv4_step *step, v
   if (need > 0 && (!ws || ws_bytes < need || (reinterpret_cast<uintptr_t>(ws) & 255u))) return DSV4_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   char *w = static_cast<char *>(ws);
-  // prologue -> query preparation -> (C4: indexer -> top-k) -> attention; the query kernel
-  // depends on no kernel of the step, so it runs beside the prologue and the indexer
   void *mq_ws = w + hp.idx_bytes + hp.ix_bytes;
-  cudaError_t e = launch_decode_prologue(hp.pro, st);
-  if (e != cudaSuccess) return to_status(e);
-  e = launch_mqa_query(hp.mq, mq_ws, st);
-  if (e != cudaSuccess) return to_status(e);
+  void *ix_ws = w + hp.idx_bytes;
+  cudaError_t e = cudaSuccess;
   if (hp.c4) {
     int32_t *idx = step->topk_idx ? step->topk_idx : reinterpret_cast<int32_t *>(w);
     hp.ix.idx = idx;
-    hp.ix.after_append = true;  // the prologue appended at most each sequence's last entry
     hp.ix.release_next = true;  // the attention follows in this call
-    e = launch_indexer_topk(hp.ix, w + hp.idx_bytes, st);
-    if (e != cudaSuccess) return to_status(e);
     hp.mq.idx = idx;
+  }
+  if (hp.c4 && indexer_uses_tensor_cores(hp.ix)) {
+    // indexer (the entries before this step's append) -> prologue and query preparation,
+    // beside it -> top-k (which scores the appended entry) -> attention
+    hp.ix.before_append = true;
+    e = launch_indexer_part(hp.ix, ix_ws, st, 1);
+    if (e != cudaSuccess) return to_status(e);
+    e = launch_decode_prologue(hp.pro, st);
+    if (e != cudaSuccess) return to_status(e);
+    e = launch_mqa_query(hp.mq, mq_ws, st);
+    if (e != cudaSuccess) return to_status(e);
+    e = launch_indexer_part(hp.ix, ix_ws, st, 2);
+    if (e != cudaSuccess) return to_status(e);
+  } else {
+    // prologue -> query preparation (beside it) -> (C4: indexer -> top-k) -> attention
+    e = launch_decode_prologue(hp.pro, st);
+    if (e != cudaSuccess) return to_status(e);
+    e = launch_mqa_query(hp.mq, mq_ws, st);
+    if (e != cudaSuccess) return to_status(e);
+    if (hp.c4) {
+      e = launch_indexer_topk(hp.ix, ix_ws, st);
+      if (e != cudaSuccess) return to_status(e);
+    }
   }
   e = launch_mqa_attention(hp.mq, mq_ws, st);
   return to_status(e);

@@ -52,14 +52,14 @@ __device__ void finish_and_store(float *e, int D, const float *gamma, float eps,
                                  double rope_theta1, dsv4_dtype dt, void *row, float *scale_out, float *red) {
   const int tid = threadIdx.x;
   float ss = 0.f;
-  for (int c = tid; c < D; c += kThreads) ss += e[c] * e[c];
+  for (int c = tid; c < D; c += static_cast<int>(blockDim.x)) ss += e[c] * e[c];
   ss = block_sum(ss, red);
   const float rs = 1.0f / sqrtf(ss / static_cast<float>(D) + eps);
   __syncthreads();
-  for (int c = tid; c < D; c += kThreads) e[c] = e[c] * rs * gamma[c];
+  for (int c = tid; c < D; c += static_cast<int>(blockDim.x)) e[c] = e[c] * rs * gamma[c];
   __syncthreads();
   const int half = rope_dims / 2;
-  for (int i = tid; i < half; i += kThreads) {
+  for (int i = tid; i < half; i += static_cast<int>(blockDim.x)) {
     float cs, sn;
     rope_cos_sin(rope_pos, i, rope_theta1, &cs, &sn);
     const int c0 = D - rope_dims + 2 * i;
@@ -70,18 +70,18 @@ __device__ void finish_and_store(float *e, int D, const float *gamma, float eps,
   __syncthreads();
   if (dt == DSV4_F32) {
     float *o = static_cast<float *>(row);
-    for (int c = tid; c < D; c += kThreads) o[c] = e[c];
+    for (int c = tid; c < D; c += static_cast<int>(blockDim.x)) o[c] = e[c];
   } else if (dt == DSV4_BF16) {
     uint16_t *o = static_cast<uint16_t *>(row);
-    for (int c = tid; c < D; c += kThreads) o[c] = float_to_bf16_bits(e[c]);
+    for (int c = tid; c < D; c += static_cast<int>(blockDim.x)) o[c] = float_to_bf16_bits(e[c]);
   } else {
     float am = 0.f;
-    for (int c = tid; c < D; c += kThreads) am = fmaxf(am, fabsf(e[c]));
+    for (int c = tid; c < D; c += static_cast<int>(blockDim.x)) am = fmaxf(am, fabsf(e[c]));
     am = block_max(am, red);
     const float scale = am > 0.f ? __fdiv_rn(am, 448.0f) : 1.0f;
     const float inv = am > 0.f ? __fdiv_rn(448.0f, am) : 1.0f;
     uint8_t *o = static_cast<uint8_t *>(row);
-    for (int c2 = tid; c2 < D / 2; c2 += kThreads) {
+    for (int c2 = tid; c2 < D / 2; c2 += static_cast<int>(blockDim.x)) {
       const uint16_t pr = float2_to_e4m3x2(__fmul_rn(e[2 * c2], inv), __fmul_rn(e[2 * c2 + 1], inv));
       *reinterpret_cast<uint16_t *>(o + 2 * c2) = pr;
     }
@@ -128,10 +128,10 @@ struct PrefillShape {
   int R, NG, S, BPC;  // threads per row, row groups per CTA, groups per block, blocks per CTA
 };
 
-__host__ __device__ inline PrefillShape prefill_shape(int D, int m) {
+__host__ __device__ inline PrefillShape prefill_shape(int D, int m, int threads = kThreads) {
   PrefillShape sh;
   sh.R = D / 8;
-  sh.NG = kThreads / sh.R;
+  sh.NG = threads / sh.R > 0 ? threads / sh.R : 1;
   int s = m / 8 > 1 ? m / 8 : 1;
   sh.S = s < sh.NG ? s : sh.NG;
   sh.BPC = sh.NG / sh.S;
@@ -295,7 +295,7 @@ struct CompressView {
 // gives an item's sequence, its index among the sequence's items and the sequence's range.
 // The arithmetic of a block does not depend on where its tokens come from (input rows or the
 // ring), so a prefill in one call and the same tokens fed one by one store the same bytes.
-template <class Map>
+template <bool kEagerLoads, class Map>
 __device__ void compress_chunk(const CompressView &p, const PrefillShape &sh, float *part, float *red, long long chunk,
                                long long total, const Map &map) {
   const int tid = threadIdx.x;
@@ -371,6 +371,14 @@ __device__ void compress_chunk(const CompressView &p, const PrefillShape &sh, fl
             for (int c = 0; c < 8; ++c) g[k][c] = 0.f;
           }
         }
+        // (kEagerLoads: every token's kv is loaded before the arithmetic, for the latency-bound
+        // decode step; the arithmetic is the same either way)
+        float ve[kEagerLoads ? kTokUnroll : 1][8];
+        if (kEagerLoads) {
+#pragma unroll
+          for (int k = 0; k < (kEagerLoads ? kTokUnroll : 1); ++k)
+            if (k < nv) load_kv8(src, b * p.m + u + k, cg, ve[k]);
+        }
         float bm[8], sa[8], sw[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
@@ -387,7 +395,12 @@ __device__ void compress_chunk(const CompressView &p, const PrefillShape &sh, fl
           if (k < nv) {
             const int64_t t = b * p.m + u + k;
             float v[8];
-            load_kv8(src, t, cg, v);
+            if (kEagerLoads) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c) v[c] = ve[kEagerLoads ? k : 0][c];
+            } else {
+              load_kv8(src, t, cg, v);
+            }
             if (t >= tail_lo && ring_slot_safe(r, p.m, t))
               store_token8(st + static_cast<size_t>(t % p.m) * (p.D + p.G), p.D, p.G, cg, v, g[k][0], g[k]);
 #pragma unroll
@@ -514,14 +527,15 @@ __device__ void compress_chunk(const CompressView &p, const PrefillShape &sh, fl
     const int n = static_cast<int>(rr.p1 - t0);
     // thread -> (token, 8-channel chunk); two tokens' loads in flight before their stores
     constexpr int kTail = 2;
-    for (int base = 0; base < n * sh.R; base += kThreads * kTail) {
+    const int nt = static_cast<int>(blockDim.x);
+    for (int base = 0; base < n * sh.R; base += nt * kTail) {
       float v[kTail][8], g[kTail][8];
       int64_t tt[kTail];
       int cc[kTail];
       bool want[kTail];
 #pragma unroll
       for (int k2 = 0; k2 < kTail; ++k2) {
-        const int e8 = base + k2 * kThreads + tid;
+        const int e8 = base + k2 * nt + tid;
         tt[k2] = t0 + e8 / sh.R;
         cc[k2] = e8 % sh.R;
         want[k2] = e8 < n * sh.R && (tt[k2] >= done_end || !ring_slot_safe(rr, p.m, tt[k2]));
@@ -597,7 +611,8 @@ __global__ void __launch_bounds__(kThreads, 2) compress_kernel(const CompressLau
   const CompressView v{p.kv, p.gate, p.kv_dt, p.gamma, p.eps, p.rope_dims, p.rope_theta1, p.state, p.m, p.D, p.G,
                        p.pages, p.scales, p.block_table, p.num_pages, p.max_blocks, p.cache_dt, p.d_status};
   const PrefillMap map{prefix, p.cu_seqlens, p.start_pos, p.B};
-  for (long long chunk = blockIdx.x; chunk < chunks; chunk += gridDim.x) compress_chunk(v, sh, part, red, chunk, total, map);
+  for (long long chunk = blockIdx.x; chunk < chunks; chunk += gridDim.x)
+    compress_chunk<false>(v, sh, part, red, chunk, total, map);
 }
 
 __global__ void __launch_bounds__(kThreads) swa_insert_kernel(const SwaLaunch p) {
@@ -634,13 +649,25 @@ struct DecodeMap {
 
 // One decode step's updates. blockIdx.y: 0 = window insert, 1 = main compressor append,
 // 2 = indexer-key compressor append.
-__global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const PrologueLaunch p) {
-  pdl_wait();
+// Launched with as few threads as its roles need (a row group per slice of a block: 64 threads
+// for D = 512 and m = 4) and little shared memory, so that its CTAs share SMs with the
+// indexer's persistent CTAs. In a C4 step it runs beside the indexer, which scores only the
+// entries visible before this step's append: it touches nothing the indexer reads, and
+// nothing any kernel before it in the call writes. So it releases its dependents at its start
+// and waits for its predecessor only at its end (its completion still implies the
+// predecessor's: the chain of waits stays unbroken).
+__device__ __forceinline__ void decode_prologue_body(const PrologueLaunch &p);
+
+__global__ void __launch_bounds__(kThreads, 2) decode_prologue_kernel(const PrologueLaunch p) {
   pdl_launch_dependents();
-  extern __shared__ __align__(16) float smem[];
-  float *scratch = smem;
-  float *e = smem + 3 * kMaxD;
-  float *red = e + kMaxD;
+  decode_prologue_body(p);
+  pdl_wait();
+}
+
+__device__ __forceinline__ void decode_prologue_body(const PrologueLaunch &p) {
+  extern __shared__ __align__(16) float smem[];  // window role: e[D], red[32]
+  float *e = smem;
+  float *red = smem + p.D;
   const int s = blockIdx.x, role = blockIdx.y;
   const int tid = threadIdx.x;
   const int64_t pos = p.pos[s];
@@ -649,7 +676,8 @@ __global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const Prologu
     return;
   }
   if (role == 0) {
-    for (int c = tid; c < p.D; c += kThreads) e[c] = load_one_f(p.kv, p.kv_dt, static_cast<size_t>(s) * p.D + c);
+    for (int c = tid; c < p.D; c += static_cast<int>(blockDim.x))
+      e[c] = load_one_f(p.kv, p.kv_dt, static_cast<size_t>(s) * p.D + c);
     __syncthreads();
     const size_t slot = static_cast<size_t>(s) * p.W + static_cast<size_t>(pos % p.W);
     void *row = static_cast<char *>(p.ring_rows) + slot * p.D * dtype_size(p.ring_dt);
@@ -666,12 +694,12 @@ __global__ void __launch_bounds__(kThreads) decode_prologue_kernel(const Prologu
                        idx ? p.idx_pages : p.pages, idx ? p.idx_scales : p.scales,
                        idx ? p.idx_block_table : p.block_table, idx ? p.idx_num_pages : p.num_pages,
                        idx ? p.idx_max_blocks : p.max_blocks, idx ? p.idx_dt : p.cache_dt, p.d_status};
-  const PrefillShape sh = prefill_shape(v.D, v.m);
+  const PrefillShape sh = prefill_shape(v.D, v.m, static_cast<int>(blockDim.x));
   const DecodeMap map{s, pos};
-  compress_chunk(v, sh, smem, smem + 3 * sh.NG * v.D, 0, 1, map);
+  // (part, the slices' merge buffer, is only used when a block is split over row groups)
+  compress_chunk<true>(v, sh, smem, smem + (sh.S > 1 ? 3 * sh.NG * v.D : 0), 0, 1, map);
 }
 
-constexpr size_t kPoolSmem = (4 * kMaxD + 32) * sizeof(float);
 
 }  // namespace
 
@@ -703,11 +731,27 @@ cudaError_t launch_decode_prologue(const PrologueLaunch &p0, cudaStream_t st) {
   PrologueLaunch p = p0;
   p.rope_theta1 = rope_theta1(p.rope_base, p.rope_dims);
   p.idx_rope_theta1 = rope_theta1(p.rope_base, p.idx_rope_dims);
-  cudaError_t e =
-      cudaFuncSetAttribute(decode_prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kPoolSmem);
+  // threads: the row groups of one block (each compressor role pools one block); shared
+  // memory: the window role's row and reduction slots, or the slices' merge buffer
+  int threads = 32;
+  size_t floats = static_cast<size_t>(p.D) + 32;
+  for (int role = 0; role < (p.idx_D > 0 ? 2 : 1); ++role) {
+    const int D = role ? p.idx_D : p.D;
+    const PrefillShape sh = prefill_shape(D, p.m);
+    const int t = (sh.S * sh.R + 31) / 32 * 32;
+    threads = t > threads ? t : threads;
+  }
+  for (int role = 0; role < (p.idx_D > 0 ? 2 : 1); ++role) {
+    const int D = role ? p.idx_D : p.D;
+    const PrefillShape sh = prefill_shape(D, p.m, threads);
+    const size_t need = (sh.S > 1 ? 3 * static_cast<size_t>(sh.NG) * D : 0) + 32;
+    floats = need > floats ? need : floats;
+  }
+  const size_t smem = floats * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(decode_prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid(p.B, p.idx_D > 0 ? 3 : 2);
-  return launch_pdl(decode_prologue_kernel, grid, dim3(kThreads), kPoolSmem, st, 1, p);
+  return launch_pdl(decode_prologue_kernel, grid, dim3(threads), smem, st, 1, p);
 }
 
 }  // namespace dsv4

@@ -53,9 +53,13 @@ __device__ __forceinline__ void hist_add_warp(int *hist, const unsigned long lon
   }
 }
 
+// Entries of sequence b the selection sees: n_entries[b], or (without it) the complete blocks
+// once the token at pos[b] is in, floor((pos + 1) / m); `appended` = 0 counts them before that
+// token's append, floor(pos / m).
 __device__ __forceinline__ int64_t visible_entries(const int32_t *n_entries, const int32_t *pos, int m, int b,
-                                                   int64_t capacity, uint32_t *d_status, bool report_it) {
-  int64_t n = n_entries ? static_cast<int64_t>(n_entries[b]) : (static_cast<int64_t>(pos[b]) + 1) / m;
+                                                   int64_t capacity, uint32_t *d_status, bool report_it,
+                                                   int appended = 1) {
+  int64_t n = n_entries ? static_cast<int64_t>(n_entries[b]) : (static_cast<int64_t>(pos[b]) + appended) / m;
   if (n < 0) n = 0;
   if (n > capacity) {
     if (report_it) report(d_status, DSV4_DEV_BAD_LENGTH);
@@ -140,7 +144,8 @@ struct TcParams {
   float *scores;  // [B][ld]; -inf where the entry has no valid page
   int64_t ld;
   uint32_t *d_status;
-  int after_append;  // wait for the kernel before only ahead of each sequence's last tile
+  int before_append;  // score only the entries visible before this step's append (floor(pos / m))
+  int release;  // release the next kernel early (always: the top-k kernel follows)
 };
 
 // The tensor-core path serves C4 layers: 64 entries per page, a 128-entry tile = 2 pages,
@@ -253,7 +258,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
     tmem_relinquish();
   }
   for (int b = tid; b < p.B; b += kIxThreads)
-    nvis[b] = visible_entries(p.n_entries, p.pos, p.m, b, capacity, p.d_status, blockIdx.x == 0);
+    nvis[b] = visible_entries(p.n_entries, p.pos, p.m, b, capacity, p.d_status, blockIdx.x == 0,
+                              p.before_append ? 0 : 1);
   __syncthreads();
   if (warp == 0) {  // tiles per sequence, scanned by one warp
     long long carry = 0;
@@ -271,11 +277,11 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
     }
     if (lane == 0) prefix[p.B] = carry;
   }
-  // Keys and scales may be written by the kernel before. In general every read waits for
-  // it; after a decode-step append (which touches only each sequence's last entry) only
-  // the stages holding a sequence's last tile do (the producer waits ahead of them).
-  if (!p.after_append) pdl_wait();
-  pdl_launch_dependents();
+  // Keys and scales may be written by the kernel before: every read waits for it. (In a
+  // decode step this kernel runs first, beside the step's own updates, which touch no entry it
+  // scores.)
+  pdl_wait();
+  if (p.release) pdl_launch_dependents();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -323,9 +329,6 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
       }
       int ok = 1;
       if (lane == 0) {
-        // the stage holding a sequence's last tile waits for the kernel before (it may have
-        // just written that entry's key and scale)
-        if (p.after_append && seg_end && lt0 + nt == prefix[sb + 1] - prefix[sb]) pdl_wait();
         if (k >= kSlots && !mbar_wait(&S.sempty[slot], static_cast<uint32_t>((k / kSlots - 1) & 1), &S.abort_flag))
           ok = 0;
         if (ok) {  // the pages' rows; the epilogue threads load their keys' scales themselves
@@ -482,11 +485,6 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   }
 
   if (tid == 0 && S.abort_flag) report(p.d_status, DSV4_DEV_TIMEOUT);
-  // After an append only the producers of stages holding a sequence's last tile waited for
-  // the kernel before; a CTA with no such stage (or a step where no sequence has a tile at
-  // all) waits here, so that this grid completes only after its predecessor: the kernels
-  // after it rely on that chain for the prologue's window and cache writes.
-  if (p.after_append && tid == 0) pdl_wait();
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
@@ -538,12 +536,90 @@ __device__ __forceinline__ int warp_sum_int(int v) {
   return v;
 }
 
+// Where the top-k kernels write: the selected entry indices (and scores).
+struct TopkOut {
+  int32_t *idx;        // [B][k]
+  float *scores;       // [B][k] or null
+  int k;
+  uint32_t *d_status;
+
+  __device__ __forceinline__ void put(int b, int o, int32_t j, float score) const {
+    const size_t at = static_cast<size_t>(b) * k + o;
+    idx[at] = j;
+    if (scores) scores[at] = score;
+  }
+};
+
+// The entry a decode step appends (entry floor((pos + 1) / m) - 1, when the step completes a
+// block), scored by the top-k kernel from the cache row the step's prologue wrote, after the
+// scoring kernel (which ran beside the prologue) scored the entries before it. The arithmetic
+// follows the scoring kernel's epilogue: c_h = w_h * scale_q[h], four chains of
+// c_h * ReLU(q_h . k) over the heads, their sum times the key's scale.
+struct AppendedKey {
+  int enabled;
+  const uint8_t *q;      // [B][H][128] e4m3 codes
+  const float *q_scale;  // [B][H] or null (1)
+  const void *w;         // [B][H]
+  dsv4_dtype w_dt;
+  const uint8_t *k_pages;
+  const float *k_scales;
+  const int32_t *block_table;
+  int num_pages, max_blocks, H;
+};
+
+// Score of sequence b's appended entry j by the CTA's threads (thread t: head t / 16, dims
+// 8 (t % 16) .. +7); -inf where the entry has no valid page. Every thread of the CTA calls it.
+__device__ float appended_score(const AppendedKey &ap, int b, int64_t j, float *part /* [64] */) {
+  const int tid = threadIdx.x, h = tid >> 4, sub = tid & 15;
+  const int64_t lb = j / kPerPage;
+  const int page = lb < ap.max_blocks ? ap.block_table[static_cast<size_t>(b) * ap.max_blocks + lb] : -1;
+  const bool valid = page >= 0 && page < ap.num_pages;
+  const size_t row = valid ? static_cast<size_t>(page) * kPerPage + static_cast<size_t>(j % kPerPage) : 0;
+  float acc = 0.f;
+  if (h < ap.H && valid) {
+    const uint2 kq = *reinterpret_cast<const uint2 *>(ap.k_pages + row * kRowBytes + 8 * sub);
+    const uint2 qq = *reinterpret_cast<const uint2 *>(ap.q + (static_cast<size_t>(b) * ap.H + h) * kRowBytes + 8 * sub);
+    const uint32_t kw[2] = {kq.x, kq.y}, qw[2] = {qq.x, qq.y};
+#pragma unroll
+    for (int u = 0; u < 2; ++u) {
+      const float2 k0 = e4m3x2_to_float2(static_cast<uint16_t>(kw[u] & 0xFFFF));
+      const float2 k1 = e4m3x2_to_float2(static_cast<uint16_t>(kw[u] >> 16));
+      const float2 q0 = e4m3x2_to_float2(static_cast<uint16_t>(qw[u] & 0xFFFF));
+      const float2 q1 = e4m3x2_to_float2(static_cast<uint16_t>(qw[u] >> 16));
+      acc = fmaf(q0.x, k0.x, acc);
+      acc = fmaf(q0.y, k0.y, acc);
+      acc = fmaf(q1.x, k1.x, acc);
+      acc = fmaf(q1.y, k1.y, acc);
+    }
+  }
+#pragma unroll
+  for (int o = 8; o > 0; o >>= 1) acc += __shfl_xor_sync(0xFFFFFFFFu, acc, o);
+  if (sub == 0 && h < ap.H) part[h] = fmaxf(acc, 0.f);
+  __syncthreads();
+  float score = -INFINITY;
+  if (tid == 0 && valid) {
+    float c4[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int hh = 0; hh < ap.H; ++hh) {
+      const float qs = ap.q_scale ? ap.q_scale[static_cast<size_t>(b) * ap.H + hh] : 1.0f;
+      const float c = load_one_f(ap.w, ap.w_dt, static_cast<size_t>(b) * ap.H + hh) * qs;
+      c4[hh & 3] = fmaf(c, part[hh], c4[hh & 3]);
+    }
+    const float sc = ap.k_scales[row];
+    if (sc > 0.f) score = ((c4[0] + c4[1]) + (c4[2] + c4[3])) * sc;
+  }
+  return score;  // (thread 0's value)
+}
+
 template <int KPT, int NT>  // NT threads of KPT keys each: a CTA holds up to NT * KPT keys, all in registers
 __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores, int64_t ld,
                                                                    const int32_t *n_entries, const int32_t *pos,
-                                                                   int m, int64_t capacity, int k, int slice,
-                                                                   int32_t *idx, float *out_scores, uint32_t *d_status,
+                                                                   int m, int64_t capacity, int slice,
+                                                                   const TopkOut out, const AppendedKey ap,
                                                                    int release) {
+  const int k = out.k;
+  uint32_t *d_status = out.d_status;
+  __shared__ float app_part[64];
+  __shared__ float app_score;
   __shared__ int hist[2][256];  // this CTA's histogram of the current pass (double buffered)
   __shared__ int whist[NT / 32][256];  // first pass: one histogram per warp (no collisions between warps)
   __shared__ int ghist[256];    // the cluster's
@@ -557,6 +633,17 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
   const int cnt = static_cast<int>(n > lo ? (n - lo < slice ? n - lo : slice) : 0);
   pdl_wait();  // the scores come from the kernel before
   if (release) pdl_launch_dependents();  // only when a kernel of the same call follows
+  // this step's appended entry, when it falls in this CTA's slice: scored here
+  int app_i = -1;
+  if (ap.enabled) {
+    const int64_t p0 = pos[b], jn = (p0 + 1) / m - 1;
+    if ((p0 + 1) % m == 0 && jn >= lo && jn < lo + cnt) app_i = static_cast<int>(jn - lo);
+  }
+  if (app_i >= 0) {  // uniform over the CTA
+    const float sc = appended_score(ap, b, lo + app_i, app_part);
+    if (tid == 0) app_score = sc;
+    __syncthreads();
+  }
   // warp w owns the contiguous run [w * 32 * KPT, (w + 1) * 32 * KPT) of the slice; its
   // lane l holds key r at position w * 32 * KPT + 32 r + l (coalesced loads, and the rounds
   // of the index-order walks below are the register index r)
@@ -566,7 +653,8 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
 #pragma unroll
   for (int r = 0; r < KPT; ++r) {
     const int i = wbase + 32 * r + lane;
-    const float v = i < cnt ? __ldcs(src + i) : -INFINITY;
+    float v = i < cnt ? __ldcs(src + i) : -INFINITY;
+    if (i == app_i) v = app_score;
     key[r] = isfinite(v) ? float_order_key(v) : 0u;
   }
   uint32_t prefix = 0, mask = 0;
@@ -695,10 +783,7 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
       const unsigned kb = __ballot_sync(0xFFFFFFFFu, keep);
       if (write && keep) {
         const int o = at + kept + __popc(kb & ((1u << lane) - 1u));
-        if (o < k) {
-          idx[static_cast<size_t>(b) * k + o] = static_cast<int32_t>(lo + wbase + 32 * r + lane);
-          if (out_scores) out_scores[static_cast<size_t>(b) * k + o] = order_key_to_float(key[r]);
-        }
+        if (o < k) out.put(b, o, static_cast<int32_t>(lo + wbase + 32 * r + lane), order_key_to_float(key[r]));
       }
       kept += __popc(kb);
     }
@@ -746,10 +831,7 @@ __global__ void __launch_bounds__(NT, 1) topk_scores_kernel(const float *scores,
     at = sel_above + warp_base[warp];
   }
   if (rank == 0) {
-    for (int i = sel_count + tid; i < k; i += NT) {
-      idx[static_cast<size_t>(b) * k + i] = -1;
-      if (out_scores) out_scores[static_cast<size_t>(b) * k + i] = -INFINITY;
-    }
+    for (int i = sel_count + tid; i < k; i += NT) out.put(b, i, -1, -INFINITY);
   }
   cluster_sync_all();  // no CTA leaves while another may still read its shared memory
 }
@@ -908,9 +990,17 @@ int64_t cand_stride(const IndexerLaunch &p) {
   return capacity > 0 ? capacity : 1;
 }
 
+// shared memory of the scoring kernel: TcSmem plus the tile prefix and visible counts
+size_t tc_tail_bytes(int B) { return 1024 + (2 * static_cast<size_t>(B) + 1) * 8; }
+
+template <int H>
+int tc_stages(int B) {
+  return sizeof(TcSmem<H, 6>) + tc_tail_bytes(B) <= 227 * 1024 ? 6 : 5;
+}
+
 template <int H>
 cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st) {
-  TcParams tp;
+  TcParams tp{};
   if (!make_rows_map(&tp.tmap_k, p.k_pages, static_cast<uint64_t>(p.num_pages) * kPerPage, kPerPage))
     return cudaErrorInvalidValue;
   if (!make_rows_map(&tp.tmap_q, p.q, static_cast<uint64_t>(p.B) * H, H)) return cudaErrorInvalidValue;
@@ -928,10 +1018,11 @@ cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st) {
   tp.scores = scores;
   tp.ld = score_ld(p);
   tp.d_status = p.d_status;
-  tp.after_append = p.after_append ? 1 : 0;
+  tp.before_append = p.before_append ? 1 : 0;
+  tp.release = 1;
   // six stages in flight where shared memory allows, else five
-  const size_t tail = 1024 + (2 * static_cast<size_t>(p.B) + 1) * 8;
-  if (sizeof(TcSmem<H, 6>) + tail <= 227 * 1024) {
+  const size_t tail = tc_tail_bytes(p.B);
+  if (tc_stages<H>(p.B) == 6) {
     const size_t smem = sizeof(TcSmem<H, 6>) + tail;
     cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -958,7 +1049,12 @@ size_t indexer_workspace_bytes(const IndexerLaunch &p) {
   return bytes;
 }
 
+
 cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t st) {
+  return launch_indexer_part(p0, ws, st, 0);
+}
+
+cudaError_t launch_indexer_part(const IndexerLaunch &p0, void *ws, cudaStream_t st, int part) {
   IndexerLaunch p = p0;
   p.rope_theta1 = rope_theta1(p.rope_base, p.q_rope_dims);
   char *w = static_cast<char *>(ws);
@@ -970,8 +1066,30 @@ cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t 
   cudaError_t e = cudaSuccess;
   if (indexer_uses_tensor_cores(p)) {
     float *scores = reinterpret_cast<float *>(w);
-    e = p.H == 32 ? launch_tc<32>(p, scores, st) : launch_tc<64>(p, scores, st);
-    if (e != cudaSuccess) return e;
+    if (part != 2) {
+      e = p.H == 32 ? launch_tc<32>(p, scores, st) : launch_tc<64>(p, scores, st);
+      if (e != cudaSuccess || part == 1) return e;
+    }
+    AppendedKey ap{};
+    if (p.before_append && !p.n_entries) {
+      ap.enabled = 1;
+      ap.q = static_cast<const uint8_t *>(p.q);
+      ap.q_scale = p.q_scale;
+      ap.w = p.w;
+      ap.w_dt = p.w_dt;
+      ap.k_pages = static_cast<const uint8_t *>(p.k_pages);
+      ap.k_scales = p.k_scales;
+      ap.block_table = p.block_table;
+      ap.num_pages = p.num_pages;
+      ap.max_blocks = p.max_blocks;
+      ap.H = p.H;
+    }
+    TopkOut out{};
+    out.idx = p.idx;
+    out.scores = p.scores;
+    out.k = p.k;
+    out.d_status = p.d_status;
+    const int rel = p.release_next ? 1 : 0;
     const int cs = tk_cluster(p), slice = tk_slice(p);
     auto launch_k = [&](auto kern, int nt) -> cudaError_t {
       if (cs > 8) {
@@ -979,8 +1097,8 @@ cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t 
         if (a != cudaSuccess) return a;
       }
       return launch_pdl(kern, dim3(static_cast<unsigned>(cs), static_cast<unsigned>(p.B)), dim3(nt), 0, st, cs,
-                        static_cast<const float *>(scores), score_ld(p), p.n_entries, p.pos, p.m, capacity_of(p), p.k,
-                        slice, p.idx, p.scores, p.d_status, p.release_next ? 1 : 0);
+                        static_cast<const float *>(scores), score_ld(p), p.n_entries, p.pos, p.m, capacity_of(p),
+                        slice, out, ap, rel);
     };
     if (slice <= 8 * kTkThreads) return launch_k(topk_scores_kernel<8, kTkThreads>, kTkThreads);
     if (slice <= 16 * kTkThreads) return launch_k(topk_scores_kernel<16, kTkThreads>, kTkThreads);

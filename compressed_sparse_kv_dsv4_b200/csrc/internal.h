@@ -125,10 +125,12 @@ struct IndexerLaunch {
   int32_t *idx;
   float *scores;
   uint32_t *d_status;
-  // The kernel before it on the stream wrote at most the last visible entry of each
-  // sequence (the decode step's prologue): the other keys may be read before that kernel
-  // has finished.
-  bool after_append = false;
+  // Decode step order (n_entries NULL): the scoring kernel runs before the step's prologue
+  // and scores the entries visible before the step's append, floor(pos / m); the top-k
+  // kernel, which runs after the prologue, scores the appended entry (floor((pos + 1) / m) - 1,
+  // when the step completes a block) from the cache row the prologue wrote, and selects over
+  // floor((pos + 1) / m) entries. Tensor-core path only.
+  bool before_append = false;
   // Another kernel of the same call follows: the last kernel releases it early. When the
   // indexer ends its call, its last kernel does not (the next call's kernels might read
   // what it writes).
@@ -137,6 +139,8 @@ struct IndexerLaunch {
 bool indexer_uses_tensor_cores(const IndexerLaunch &p);
 size_t indexer_workspace_bytes(const IndexerLaunch &p);
 cudaError_t launch_indexer_topk(const IndexerLaunch &p, void *ws, cudaStream_t st);
+// part 1: the scoring kernel only (tensor-core path); part 2: the top-k only; 0: both
+cudaError_t launch_indexer_part(const IndexerLaunch &p, void *ws, cudaStream_t st, int part);
 
 // ---------------------------------------------------------------- sparse / dense MQA
 struct MqaLaunch {

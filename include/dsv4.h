@@ -195,7 +195,9 @@ dsv4_status dsv4_swa_insert(const dsv4_swa_insert_args *args, dsv4_stream stream
  *   pos [batch] device int32 (used only when q_rope_dims > 0).
  * fp8 queries and keys with dim 128, heads 32 or 64, m == 4, no query RoPE and batch <= 512
  * run on the tensor cores (tcgen05, fed by TMA); other shapes run on a CUDA-core kernel.
- * Both give the same entries.
+ * Both give the same entries. On the tensor-core path a second kernel selects each
+ * sequence's top k from the streamed scores (one thread-block cluster per sequence) and writes
+ * idx in ascending entry order.
  */
 typedef struct {
   int32_t batch;
@@ -240,8 +242,9 @@ dsv4_status dsv4_indexer_topk(const dsv4_indexer_args *args, void *workspace,
  * DSV4_ERR_SCRATCH_LIMIT and launches nothing (use dsv4_indexer_topk with a caller
  * workspace instead). The tensor-core path needs about 4 bytes per cache entry of every
  * sequence: 16 MiB admits about 127 sequences of 32768 entries (a 131072-token context).
- * Zero state: nothing has to start at zero; the per-sequence candidate counts at the head
- * of the scratch are zeroed by the call itself, on `stream`, before its kernels run.
+ * Zero state: nothing has to start at zero; on the CUDA-core path the per-sequence candidate
+ * counts at the head of the scratch are zeroed by the call itself, on `stream`, before its
+ * kernels run.
  * Concurrency: the scratch is shared by every call on a device. Calls ordered on one
  * stream are safe; calls that can overlap (different streams, or several host threads
  * without ordering) race on the scratch and give wrong results: serialize them.
@@ -300,6 +303,9 @@ dsv4_status dsv4_sparse_mqa_decode(const dsv4_mqa_args *args, void *workspace,
  *   append; query RoPE; for C4 layers the indexer + top-k over floor((pos+1)/m) entries;
  *   the shared-K/V attention over the window united with the selected (C4) or all
  *   (C128) entries; inverse RoPE; the output store.
+ *   (On the tensor-core path of a C4 layer the indexer's scoring kernel runs first, beside the
+ *   state updates, over the entries visible before the append; the top-k kernel scores the
+ *   appended entry itself. The results are those of the order above.)
  * The caches, the ring and the compressor states are updated in place. n_c is derived
  * from pos; the caller keeps pos < capacity.
  */

@@ -213,6 +213,32 @@ def test_indexer_tensor_core_topk_matches_oracle(k):
         assert np.all(np.abs(got - want) <= 1e-5 * np.abs(want).max()), f"seq {s}: scores"
 
 
+def test_indexer_tensor_core_long_sequences_topk_matches_oracle():
+    """Sequences of 46K-70K entries: top-k clusters of more CTAs, slices of 24 keys per
+    thread, an empty sequence beside them."""
+    n_list = [50000, 46100, 0, 70001]
+    idx, scores, ol, qd, wd = _indexer_case(n_list, 512, seed=23)
+    for s, n in enumerate(n_list):
+        if n == 0:
+            assert np.all(idx[s] == -1)
+            continue
+        ref = O.indexer_scores(qd[s], wd[s], ol.idx_cache.read(s, np.arange(n)))
+        check_topk(idx[s], ref, 512, n, f"seq {s}")
+
+
+def test_indexer_many_short_sequences_topk_in_entry_order():
+    """48 sequences of 0 to 5000 entries (several per CTA of the scoring kernel), many with
+    fewer entries than k: the selection pads with -1 and writes the kept entries in ascending
+    entry order."""
+    n_list = [3, 700, 64, 5000, 1, 130, 0, 257] * 6
+    idx, scores, ol, qd, wd = _indexer_case(n_list, 64, seed=25)
+    for s, n in enumerate(n_list):
+        ref = O.indexer_scores(qd[s], wd[s], ol.idx_cache.read(s, np.arange(n))) if n else np.zeros(0)
+        check_topk(idx[s], ref, 64, n, f"seq {s}")
+        v = idx[s] >= 0
+        assert np.all(np.diff(idx[s][v]) > 0), f"seq {s}: output not in ascending entry order"
+
+
 def test_indexer_full_tie_takes_lowest_indices():
     idx, scores, ol, qd, wd = _indexer_case([3000, 700], 512, all_negative=True)
     for s in range(2):
