@@ -64,6 +64,14 @@ Readings taken where both are silent (the plainest one the text supports):
   R14 top-k ties go to the lower entry index; with n_c <= k every entry is
       taken and the rest of the k slots hold -1.
   R15 with no visible key at all the output is zero.
+  R21 query norm ([vLLM] "vLLM side": the fused "Q-norm + KV RoPE + K insert"
+      kernel): when a layer has a query norm weight, each query head is
+      RMS-normed over its D dims with that weight and the layer's eps before its
+      RoPE, like the window key of R4.
+  R22 fp8 output ([vLLM] "vLLM side": the fused "inverse RoPE + fp8 quant"
+      kernel): the output of each head, after its inverse RoPE, is stored as
+      e4m3 codes in blocks of 128 channels, each block with one float32 scale
+      amax/448 (the rule of R12 applied to every 128-value block).
 """
 
 from __future__ import annotations
@@ -389,6 +397,37 @@ def shared_kv_attention(q, pos: int, keys, softmax_scale: float, rope_dims: int,
     return apply_rope(p @ keys, pos, rope_dims, rope_base, inverse=True)
 
 
+def query_norm(q, gamma_q, eps: float) -> np.ndarray:
+    """R21: each head of q [H, D] RMS-normed over its D dims, times gamma_q [D]."""
+    return rms_norm(q, gamma_q, eps)
+
+
+OUT_BLOCK = 128  # channels per fp8 output block (R22)
+
+
+def store_output(o, dtype: str):
+    """Round an attention output [H, D] into its stored form (R22 for fp8).
+
+    Returns (codes, scales, decoded float64): f32 / bf16 rows as `store` gives
+    them (scales [H, 1] of ones); fp8: codes [H, D] and scales [H, D/128], each
+    128-channel block rounded by `store` on its own.
+    """
+    o = np.asarray(o, dtype=np.float64)
+    h, d = o.shape
+    if dtype != "fp8":
+        codes, _, dec = store(o, dtype)
+        return codes, np.ones((h, 1), np.float32), dec
+    nb = d // OUT_BLOCK
+    codes = np.zeros((h, d), np.uint8)
+    scales = np.zeros((h, nb), np.float32)
+    dec = np.zeros((h, d))
+    for i in range(h):
+        for j in range(nb):
+            sl = slice(j * OUT_BLOCK, (j + 1) * OUT_BLOCK)
+            codes[i, sl], scales[i, j], dec[i, sl] = store(o[i, sl], "fp8")
+    return codes, scales, dec
+
+
 def window_positions(pos: int, W: int) -> np.ndarray:
     """Positions max(0, p-W+1) .. p (reading R9)."""
     return np.arange(max(0, pos - W + 1), pos + 1, dtype=np.int64)
@@ -435,6 +474,7 @@ class LayerState:
     gamma_idx: np.ndarray | None = None
     idx_state: CompressorState | None = None
     idx_cache: PagedCache | None = None
+    gamma_q: np.ndarray | None = None  # query norm weight (R21); None: no query norm
 
 
 @dataclass
@@ -496,7 +536,10 @@ def decode_attend(layer: LayerState, step: StepInputs, seqs=None):
         if sel.shape[0]:
             parts.append(layer.main_cache.read(s, sel))
         keys = np.concatenate(parts, axis=0)
-        o = shared_kv_attention(step.q[s], p, keys, c.tau, c.rope_dims, c.rope_base)
+        q = step.q[s]
+        if layer.gamma_q is not None:
+            q = query_norm(q, layer.gamma_q, c.eps)
+        o = shared_kv_attention(q, p, keys, c.tau, c.rope_dims, c.rope_base)
         out[s] = (o, sel, scores)
     return out
 

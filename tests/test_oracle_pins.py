@@ -343,3 +343,42 @@ def test_kv_state_sizing_reproduces_the_page(golden_dir):
     assert round(v32, 1) == g["v32_gib"]
     assert round(v4, 2) == g["v4_gib"]
     assert round(v32 / v4, 1) == g["ratio"]
+
+
+# ----------------------------------------------------------------- query norm, fp8 output
+def test_query_norm_closed_form_and_scale_invariance():
+    """R21: with gamma = 1 every normed head has RMS 1 (up to eps); the attention then does not
+    depend on a positive per-head scale of the query."""
+    H, D, N = 4, 64, 23
+    q = RNG.standard_normal((H, D)) * np.array([[0.5], [3.0], [10.0], [0.1]])
+    qn = O.query_norm(q, np.ones(D), 1e-6)
+    ms = np.mean(q * q, axis=1)
+    assert np.allclose(np.sqrt(np.mean(qn * qn, axis=1)), np.sqrt(ms / (ms + 1e-6)), rtol=1e-12)
+    keys = RNG.standard_normal((N, D))
+    scale = np.array([[7.0], [0.25], [1.0], [40.0]])
+    a = O.shared_kv_attention(O.query_norm(q, np.ones(D), 0.0), 99, keys, 0.125, 16, 1e4)
+    b = O.shared_kv_attention(O.query_norm(q * scale, np.ones(D), 0.0), 99, keys, 0.125, 16, 1e4)
+    assert np.allclose(a, b, atol=1e-12)
+
+
+def test_fp8_output_blocks_hand_example():
+    """R22: every 128-channel block gets its own scale amax/448; a block's largest value maps
+    to code 448 (0x7E), and the blocks do not see each other."""
+    o = np.zeros((2, 256))
+    o[0, :128] = np.linspace(-1.0, 1.0, 128)       # amax 1
+    o[0, 128:] = 1e-3 * np.linspace(0.0, 2.0, 128)  # amax 2e-3
+    o[1, :] = 448.0 * 4                             # amax 1792, constant
+    codes, scales, dec = O.store_output(o, "fp8")
+    assert scales.shape == (2, 2)
+    assert scales[0, 0] == np.float32(np.float32(1.0) / np.float32(448.0))
+    assert scales[0, 1] == np.float32(np.float32(2e-3) / np.float32(448.0))
+    assert scales[1, 0] == scales[1, 1] == np.float32(4.0)
+    assert codes[0, 127] == 0x7E and codes[0, 0] == 0xFE and codes[0, 255] == 0x7E
+    assert np.all(codes[1] == 0x7E) and np.all(dec[1] == 1792.0)
+    # the small block keeps its relative precision (its own scale), e4m3: 2^-4 relative
+    big = np.abs(o[0, 128:]) > 2.0 ** -6 * float(scales[0, 1])
+    assert np.all(np.abs(dec[0, 128:][big] - o[0, 128:][big]) <= 2.0 ** -4 * np.abs(o[0, 128:][big]))
+    # against the library cast of the scaled block
+    inv = np.float32(np.float32(448.0) / np.float32(1.0))
+    lib = torch.from_numpy(np.float32(o[0, :128]).astype(np.float32) * inv).to(torch.float8_e4m3fn)
+    assert np.array_equal(codes[0, :128], lib.view(torch.uint8).numpy())
