@@ -530,7 +530,8 @@ def run_ours(args):
     }
     if world == 1 and not args.no_extra:
         line["compress_prefill"] = leg_compress_prefill(lib, dev, stream, flush, hbm_peak)
-        line["stack_1m"] = leg_stack_1m(lib, dev, stream, flush, hbm_peak)
+        if not args.skip_1m:
+            line["stack_1m"] = leg_stack_1m(lib, dev, stream, flush, hbm_peak)
     if world == 1 and not args.no_cpu_baseline:
         seqs, dt = oracle_sample(la, sets, budget_s=args.cpu_budget)
         line["cpu_baseline"] = {"value": round(seqs / dt, 3), "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
@@ -577,6 +578,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the compressor-prefill and 1M-stack legs")
+    ap.add_argument("--skip-1m", action="store_true", help="skip the 1M-stack leg")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle time for cpu_baseline")
     args = ap.parse_args()
     if args.warmup < 3:

@@ -13,6 +13,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SCRATCH_LIMIT = 0, 1, 2, 3, 
 NOALLOC_SCRATCH_BYTES = 16 << 20
 DEV_BAD_INDEX, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
 PAGE_POSITIONS = 256
+OUT_BLOCK = 128  # channels per fp8 output block
 
 DTYPE_CODE = {"f32": F32, "bf16": BF16, "fp8": FP8}
 
@@ -60,7 +61,7 @@ class MqaArgs(C.Structure):
     _fields_ = [("batch", i32), ("heads", i32), ("dim", i32), ("q", p), ("q_dtype", C.c_int), ("pos", p),
                 ("cache", PagedCache), ("n_entries", p), ("idx", p), ("k", i32), ("ring", WindowRing),
                 ("softmax_scale", C.c_float), ("rope", Rope), ("out", p), ("out_dtype", C.c_int), ("lse", p),
-                ("d_status", p)]
+                ("d_status", p), ("q_norm_gamma", p), ("q_norm_eps", C.c_float), ("out_scales", p)]
 
 
 class Layer(C.Structure):
@@ -68,14 +69,14 @@ class Layer(C.Structure):
                 ("idx_dim", i32), ("rope", Rope), ("idx_rope_dims", i32), ("q_idx_rope", i32),
                 ("eps", C.c_float), ("softmax_scale", C.c_float), ("gamma", p), ("gamma_idx", p),
                 ("state", CompressorState), ("cache", PagedCache), ("ring", WindowRing),
-                ("idx_state", CompressorState), ("idx_cache", PagedCache)]
+                ("idx_state", CompressorState), ("idx_cache", PagedCache), ("gamma_q", p)]
 
 
 class Step(C.Structure):
     _fields_ = [("batch", i32), ("pos", p), ("kv", p), ("gate", p), ("idx_kv", p), ("idx_gate", p),
                 ("kv_dtype", C.c_int), ("q", p), ("q_dtype", C.c_int), ("q_idx", p), ("q_idx_dtype", C.c_int),
                 ("q_idx_scale", p), ("w", p), ("w_dtype", C.c_int), ("out", p), ("out_dtype", C.c_int),
-                ("topk_idx", p), ("d_status", p)]
+                ("topk_idx", p), ("d_status", p), ("out_scales", p)]
 
 
 EXPORTS = {

@@ -106,6 +106,7 @@ class DeviceLayer:
     gamma_idx: torch.Tensor | None = None
     idx_state: DeviceState | None = None
     idx_cache: DeviceCache | None = None
+    gamma_q: torch.Tensor | None = None
     _ws: torch.Tensor | None = field(default=None, repr=False)
 
     def struct(self) -> A.Layer:
@@ -122,6 +123,7 @@ class DeviceLayer:
         L.state = self.state.struct()
         L.cache = self.cache.struct()
         L.ring = self.ring.struct()
+        L.gamma_q = _ptr(self.gamma_q)
         if self.kind == "c4":
             L.idx_state = self.idx_state.struct()
             L.idx_cache = self.idx_cache.struct()
@@ -140,6 +142,8 @@ class DeviceLayer:
                     ring=DeviceRing(to_device_codes(la.swa_rows, s.swa_dtype, dev), f(la.swa_scales), s.swa_dtype),
                     topk=s.k, H_I=s.H_I, d_I=s.d_I, rope_dims=s.rope_dims, rope_base=s.rope_base,
                     idx_rope_dims=s.idx_rope_dims, q_idx_rope=s.q_idx_rope, eps=s.eps)
+        if getattr(la, "gamma_q", None) is not None:
+            layer.gamma_q = f(la.gamma_q.astype(np.float32))
         if s.kind == "c4":
             layer.gamma_idx = f(la.gamma_idx.astype(np.float32))
             layer.idx_state = DeviceState(f(la.idx_state.astype(np.float32)), s.d_I)
@@ -176,6 +180,7 @@ class DeviceStep:
     w_dtype: str = "bf16"
     topk_idx: torch.Tensor | None = None
     d_status: torch.Tensor | None = None
+    out_scales: torch.Tensor | None = None  # [B, H, D/128] float32 for fp8 outputs
 
     def struct(self) -> A.Step:
         S = A.Step()
@@ -190,6 +195,7 @@ class DeviceStep:
         S.out, S.out_dtype = _ptr(self.out), DT[self.out_dtype]
         S.topk_idx = _ptr(self.topk_idx)
         S.d_status = _ptr(self.d_status)
+        S.out_scales = _ptr(self.out_scales)
         return S
 
     @classmethod
@@ -203,6 +209,8 @@ class DeviceStep:
                    out=torch.empty((B, spec.H, spec.D), dtype=TORCH_CODE_DTYPE[spec.out_dtype], device=dev),
                    kv_dtype=spec.kv_dtype, q_dtype=spec.q_dtype, out_dtype=spec.out_dtype,
                    d_status=torch.zeros(1, dtype=torch.int32, device=dev))
+        if spec.out_dtype == "fp8":
+            step.out_scales = torch.empty((B, spec.H, spec.D // A.OUT_BLOCK), dtype=torch.float32, device=dev)
         if spec.kind == "c4":
             step.idx_kv, step.idx_gate = c(st.idx_kv, spec.kv_dtype), c(st.idx_gate, spec.kv_dtype)
             step.q_idx, step.q_idx_dtype = c(st.q_idx, spec.q_idx_dtype), spec.q_idx_dtype
@@ -287,12 +295,13 @@ def indexer_topk_noalloc(q_idx, w, keys: DeviceCache, n_entries, k: int, *, idx,
 
 def mqa_args(q, pos, cache: DeviceCache, ring: DeviceRing, *, q_dtype: str, out, out_dtype: str, idx=None,
              n_entries=None, softmax_scale: float = 0.0, rope_dims: int = 64, rope_base: float = 10000.0, lse=None,
-             d_status=None) -> A.MqaArgs:
+             d_status=None, q_norm_gamma=None, q_norm_eps: float = 1e-6, out_scales=None) -> A.MqaArgs:
     B, H, D = q.shape
     return A.MqaArgs(batch=B, heads=H, dim=D, q=_ptr(q), q_dtype=DT[q_dtype], pos=_ptr(pos), cache=cache.struct(),
                      n_entries=_ptr(n_entries), idx=_ptr(idx), k=0 if idx is None else idx.shape[1],
                      ring=ring.struct(), softmax_scale=softmax_scale, rope=A.Rope(rope_dims, rope_base),
-                     out=_ptr(out), out_dtype=DT[out_dtype], lse=_ptr(lse), d_status=_ptr(d_status))
+                     out=_ptr(out), out_dtype=DT[out_dtype], lse=_ptr(lse), d_status=_ptr(d_status),
+                     q_norm_gamma=_ptr(q_norm_gamma), q_norm_eps=q_norm_eps, out_scales=_ptr(out_scales))
 
 
 def mqa_workspace_size(args: A.MqaArgs) -> int:
@@ -302,17 +311,23 @@ def mqa_workspace_size(args: A.MqaArgs) -> int:
 
 def sparse_mqa_decode(q, pos, cache: DeviceCache, ring: DeviceRing, *, q_dtype: str, out_dtype: str, idx=None,
                       n_entries=None, softmax_scale: float = 0.0, rope_dims: int = 64, rope_base: float = 10000.0,
-                      with_lse: bool = False, d_status=None, workspace=None, stream=None):
+                      with_lse: bool = False, d_status=None, workspace=None, stream=None, q_norm_gamma=None,
+                      q_norm_eps: float = 1e-6):
+    """Returns out (and lse); for fp8 outputs, out is (codes, scales [B, H, D/128])."""
     lib = A.load()
     B, H, D = q.shape
     out = torch.empty((B, H, D), dtype=TORCH_CODE_DTYPE[out_dtype], device=q.device)
+    out_scales = (torch.empty((B, H, D // A.OUT_BLOCK), dtype=torch.float32, device=q.device)
+                  if out_dtype == "fp8" else None)
     lse = torch.empty((B, H), dtype=torch.float32, device=q.device) if with_lse else None
     a = mqa_args(q, pos, cache, ring, q_dtype=q_dtype, out=out, out_dtype=out_dtype, idx=idx, n_entries=n_entries,
-                 softmax_scale=softmax_scale, rope_dims=rope_dims, rope_base=rope_base, lse=lse, d_status=d_status)
+                 softmax_scale=softmax_scale, rope_dims=rope_dims, rope_base=rope_base, lse=lse, d_status=d_status,
+                 q_norm_gamma=q_norm_gamma, q_norm_eps=q_norm_eps, out_scales=out_scales)
     need = lib.dsv4_mqa_workspace_size(C.byref(a))
     ws = workspace if workspace is not None else torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
     A.check("dsv4_sparse_mqa_decode", lib.dsv4_sparse_mqa_decode(C.byref(a), _ptr(ws), ws.numel(), _stream(stream)))
-    return (out, lse) if with_lse else out
+    res = (out, out_scales) if out_dtype == "fp8" else out
+    return (res, lse) if with_lse else res
 
 
 def layer_state_bytes(context: int, m: int, entry_width: int, window: int, window_width: int,

@@ -239,7 +239,9 @@ static dsv4_status mqa_launch_args(const dsv4_mqa_args *a, MqaLaunch *p) {
   if (!a->idx && !a->n_entries) return DSV4_ERR_INVALID_ARG;
   if (!valid_rope(a->rope, a->dim)) return DSV4_ERR_INVALID_ARG;
   if (a->q_dtype != DSV4_F32 && a->q_dtype != DSV4_BF16) return DSV4_ERR_UNSUPPORTED;
-  if (a->out_dtype != DSV4_F32 && a->out_dtype != DSV4_BF16) return DSV4_ERR_UNSUPPORTED;
+  if (!valid_dtype(a->out_dtype)) return DSV4_ERR_UNSUPPORTED;
+  if (a->out_dtype == DSV4_FP8E4M3 && (!a->out_scales || a->dim % kOutBlock != 0)) return DSV4_ERR_INVALID_ARG;
+  if (a->q_norm_gamma && !(a->q_norm_eps >= 0.f)) return DSV4_ERR_INVALID_ARG;
   if (a->dim > 1024 || a->dim % 32 != 0) return DSV4_ERR_UNSUPPORTED;
   if (!aligned16(a->q) || !aligned16(a->out)) return DSV4_ERR_INVALID_ARG;
   *p = MqaLaunch{};
@@ -269,6 +271,9 @@ static dsv4_status mqa_launch_args(const dsv4_mqa_args *a, MqaLaunch *p) {
   p->out_dt = a->out_dtype;
   p->lse = a->lse;
   p->d_status = a->d_status;
+  p->q_norm_gamma = a->q_norm_gamma;
+  p->q_norm_eps = a->q_norm_eps;
+  p->out_scales = a->out_scales;
   return DSV4_OK;
 }
 
@@ -389,12 +394,15 @@ dsv4_status hybrid_plan(const dsv4_layer *L, const dsv4_step *S, int32_t batch, 
   mq.softmax_scale = L->softmax_scale;
   mq.rope_dims = L->rope.rope_dims;
   mq.rope_base = L->rope.rope_base;
+  mq.q_norm_gamma = L->gamma_q;
+  mq.q_norm_eps = L->eps;
   if (mq.D > 1024 || mq.D % 32 != 0) return DSV4_ERR_UNSUPPORTED;
   if (S) {
     if (S->batch != batch || !S->pos || !S->kv || !S->gate || !S->q || !S->out) return DSV4_ERR_INVALID_ARG;
     if (S->kv_dtype != DSV4_F32 && S->kv_dtype != DSV4_BF16) return DSV4_ERR_UNSUPPORTED;
     if (S->q_dtype != DSV4_F32 && S->q_dtype != DSV4_BF16) return DSV4_ERR_UNSUPPORTED;
-    if (S->out_dtype != DSV4_F32 && S->out_dtype != DSV4_BF16) return DSV4_ERR_UNSUPPORTED;
+    if (!valid_dtype(S->out_dtype)) return DSV4_ERR_UNSUPPORTED;
+    if (S->out_dtype == DSV4_FP8E4M3 && (!S->out_scales || L->dim % kOutBlock != 0)) return DSV4_ERR_INVALID_ARG;
     if (!aligned16(S->q) || !aligned16(S->out)) return DSV4_ERR_INVALID_ARG;
     pr.pos = S->pos;
     pr.kv_dt = S->kv_dtype;
@@ -425,6 +433,7 @@ dsv4_status hybrid_plan(const dsv4_layer *L, const dsv4_step *S, int32_t batch, 
     mq.n_entries = nullptr;
     mq.out = S->out;
     mq.out_dt = S->out_dtype;
+    mq.out_scales = S->out_scales;
     mq.lse = nullptr;
     mq.d_status = S->d_status;
   } else {

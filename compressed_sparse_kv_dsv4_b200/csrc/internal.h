@@ -167,7 +167,11 @@ struct MqaLaunch {
   dsv4_dtype out_dt;
   float *lse;
   uint32_t *d_status;
+  const float *q_norm_gamma = nullptr;  // [D]: RMS-norm each query head before RoPE (null: no)
+  float q_norm_eps = 0.f;
+  float *out_scales = nullptr;          // [B][H][D / 128] for fp8 output
 };
+constexpr int kOutBlock = 128;  // channels per fp8 output block (one scale each)
 bool mqa_uses_tensor_cores(const MqaLaunch &p);
 size_t mqa_workspace_bytes(const MqaLaunch &p);
 cudaError_t launch_mqa(const MqaLaunch &p, void *ws, cudaStream_t st);

@@ -305,12 +305,32 @@ __global__ void __launch_bounds__(128) mqa_query_kernel(const MqaTcParams P) {
   __syncthreads();
   float x[4][8];
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {  // the 8 values of run i, rotated where they are rope dims
+  for (int i = 0; i < 4; ++i) {
     const uint32_t v[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       x[i][2 * u] = __uint_as_float(v[u] << 16);
       x[i][2 * u + 1] = __uint_as_float(v[u] & 0xFFFF0000u);
+    }
+  }
+  if (p.q_norm_gamma) {  // RMSNorm of the head (its 16 threads are consecutive lanes), times gamma
+    float ss = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int u = 0; u < 8; ++u) ss += x[i][u] * x[i][u];
+#pragma unroll
+    for (int o = 8; o > 0; o >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, o);
+    const float rs = 1.0f / sqrtf(ss / static_cast<float>(kD) + p.q_norm_eps);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[i][u] = x[i][u] * rs * __ldg(p.q_norm_gamma + d0 + i * 8 + u);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {  // the 8 values of run i, rotated where they are rope dims
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
       const int d = d0 + i * 8 + 2 * u;
       if (d >= rope0) {
         const float c = cs[(d - rope0) >> 1], sv = sn[(d - rope0) >> 1];
@@ -865,12 +885,20 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
     if (!mbar_wait(&S.part_full, 0u, &no_abort) && tid == 0) S.abort_flag = 1;
   }
   __syncthreads();
-  // CTA rank finishes its columns: the weighted sum of the cs slabs, / l, inverse RoPE, store
-  {
+  // CTA rank finishes its columns: the weighted sum of the cs slabs, / l, inverse RoPE, store.
+  // fp8 outputs go through the freed query buffer 128 columns at a time (one [64][128] float
+  // stage), each head's 128-column block quantized by one warp with its own scale.
+  const bool out_fp8 = p.out_dt == DSV4_FP8E4M3;
+  const int pieces = out_fp8 ? Dc / kOutBlock : 1;
+  float *stage = reinterpret_cast<float *>(&S.q[0][0]);
+#pragma unroll 1
+  for (int pc = 0; pc < pieces; ++pc) {
     const int rope0 = kD - p.rope_dims;
-    const int lruns = 7 - lcs;  // runs = 2^lruns
-    for (int e = tid; e < kH * runs; e += kThreads) {
-      const int h = e >> lruns, r4 = e & (runs - 1), d = static_cast<int>(rank) * Dc + r4 * 4;
+    const int lruns = out_fp8 ? 5 : 7 - lcs;  // runs of 4 columns: 2^lruns (a piece of 128 for fp8)
+    const int runs_here = 1 << lruns;
+    for (int e = tid; e < kH * runs_here; e += kThreads) {
+      const int h = e >> lruns, r4 = (e & (runs_here - 1)) + (out_fp8 ? pc * 32 : 0),
+                d = static_cast<int>(rank) * Dc + r4 * 4;
       const int at = h * Dc + slab_run(h, r4) * 4;
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll 4
@@ -895,15 +923,33 @@ __global__ void __launch_bounds__(kThreads, 1) mqa_tc_kernel(const __grid_consta
         }
       }
       const size_t off = (static_cast<size_t>(b) * kH + h) * kD + d;
-      if (p.out_dt == DSV4_F32) {
+      if (out_fp8) {
+        *reinterpret_cast<float4 *>(stage + h * kOutBlock + (r4 - pc * 32) * 4) = make_float4(y[0], y[1], y[2], y[3]);
+      } else if (p.out_dt == DSV4_F32) {
         *reinterpret_cast<float4 *>(static_cast<float *>(p.out) + off) = make_float4(y[0], y[1], y[2], y[3]);
       } else {
         *reinterpret_cast<uint2 *>(static_cast<uint16_t *>(p.out) + off) =
             make_uint2(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]));
       }
     }
-    if (rank == 0 && p.lse && tid < kH) p.lse[static_cast<size_t>(b) * kH + tid] = S.lse[tid];
+    if (out_fp8) {
+      __syncthreads();
+      const int col0 = static_cast<int>(rank) * Dc + pc * kOutBlock;  // the block's first column
+      for (int h = warp; h < kH; h += kThreads / 32) {
+        const float4 v = *reinterpret_cast<const float4 *>(stage + h * kOutBlock + lane * 4);
+        const float am = warp_max(fmaxf(fmaxf(fabsf(v.x), fabsf(v.y)), fmaxf(fabsf(v.z), fabsf(v.w))));
+        const float scale = am > 0.f ? __fdiv_rn(am, 448.0f) : 1.0f;
+        const float inv = am > 0.f ? __fdiv_rn(448.0f, am) : 1.0f;
+        const uint32_t w = static_cast<uint32_t>(float2_to_e4m3x2(__fmul_rn(v.x, inv), __fmul_rn(v.y, inv))) |
+                           (static_cast<uint32_t>(float2_to_e4m3x2(__fmul_rn(v.z, inv), __fmul_rn(v.w, inv))) << 16);
+        *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(p.out) + (static_cast<size_t>(b) * kH + h) * kD + col0 +
+                                      lane * 4) = w;
+        if (lane == 0) p.out_scales[(static_cast<size_t>(b) * kH + h) * (kD / kOutBlock) + col0 / kOutBlock] = scale;
+      }
+      __syncthreads();  // the stage is rewritten by the next piece
+    }
   }
+  if (rank == 0 && p.lse && tid < kH) p.lse[static_cast<size_t>(b) * kH + tid] = S.lse[tid];
   if (tid == 0 && S.abort_flag) report(p.d_status, DSV4_DEV_TIMEOUT);
   if (warp == kMmaWarp) {
     tc_fence_after();
@@ -931,6 +977,15 @@ __global__ void __launch_bounds__(256) mqa_simt_kernel(const MqaLaunch p, float 
   const int D = p.D, half = p.rope_dims / 2, rope0 = D - p.rope_dims;
   for (int d = tid; d < D; d += 256) qr[d] = load_one_f(p.q, p.q_dt, (static_cast<size_t>(b) * p.H + h) * D + d);
   __syncthreads();
+  if (p.q_norm_gamma) {  // RMSNorm of the head, times gamma
+    float ss = 0.f;
+    for (int d = tid; d < D; d += 256) ss += qr[d] * qr[d];
+    ss = block_sum(ss, red);
+    const float rs = 1.0f / sqrtf(ss / static_cast<float>(D) + p.q_norm_eps);
+    __syncthreads();
+    for (int d = tid; d < D; d += 256) qr[d] = qr[d] * rs * p.q_norm_gamma[d];
+    __syncthreads();
+  }
   for (int i = tid; i < half; i += 256) {
     float c, s;
     rope_cos_sin(L.pos, i, p.rope_theta1, &c, &s);
@@ -1007,10 +1062,28 @@ __global__ void __launch_bounds__(256) mqa_simt_kernel(const MqaLaunch p, float 
     ob[rope0 + 2 * i + 1] = -x0 * s + x1 * c;
   }
   __syncthreads();
-  for (int d = tid; d < D; d += 256) {
-    const size_t off = (static_cast<size_t>(b) * p.H + h) * D + d;
-    if (p.out_dt == DSV4_F32) static_cast<float *>(p.out)[off] = ob[d];
-    else static_cast<uint16_t *>(p.out)[off] = float_to_bf16_bits(ob[d]);
+  if (p.out_dt == DSV4_FP8E4M3) {  // 128-channel blocks, one scale each: a warp per block
+    const int lane = tid & 31, warp = tid >> 5;
+    for (int blk = warp; blk < D / kOutBlock; blk += 8) {
+      float am = 0.f;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) am = fmaxf(am, fabsf(ob[blk * kOutBlock + lane * 4 + u]));
+      am = warp_max(am);
+      const float scale = am > 0.f ? __fdiv_rn(am, 448.0f) : 1.0f;
+      const float inv = am > 0.f ? __fdiv_rn(448.0f, am) : 1.0f;
+      const float *v = ob + blk * kOutBlock + lane * 4;
+      const uint32_t w = static_cast<uint32_t>(float2_to_e4m3x2(__fmul_rn(v[0], inv), __fmul_rn(v[1], inv))) |
+                         (static_cast<uint32_t>(float2_to_e4m3x2(__fmul_rn(v[2], inv), __fmul_rn(v[3], inv))) << 16);
+      *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(p.out) + (static_cast<size_t>(b) * p.H + h) * D +
+                                    blk * kOutBlock + lane * 4) = w;
+      if (lane == 0) p.out_scales[(static_cast<size_t>(b) * p.H + h) * (D / kOutBlock) + blk] = scale;
+    }
+  } else {
+    for (int d = tid; d < D; d += 256) {
+      const size_t off = (static_cast<size_t>(b) * p.H + h) * D + d;
+      if (p.out_dt == DSV4_F32) static_cast<float *>(p.out)[off] = ob[d];
+      else static_cast<uint16_t *>(p.out)[off] = float_to_bf16_bits(ob[d]);
+    }
   }
   if (p.lse && tid == 0)
     p.lse[static_cast<size_t>(b) * p.H + h] = l_run > 0.f ? (m_run + log2f(l_run)) * kLn2 : -INFINITY;
@@ -1031,8 +1104,10 @@ bool mqa_uses_tensor_cores(const MqaLaunch &p) {
 // CTAs per sequence by the batch alone: as many as keep the batch within one wave of SMs
 // (a power of two, at most 16). The launch may take fewer (below), never more.
 static int mqa_cluster_rule(const MqaLaunch &p) {
+  // (fp8 output: at most 4 CTAs, so that each owns whole 128-column blocks of the output)
+  const int cap = p.out_dt == DSV4_FP8E4M3 ? kD / kOutBlock : kMaxCluster;
   int cs = 1;
-  while (cs < kMaxCluster && static_cast<long long>(cs) * 2 * p.B <= sm_count()) cs <<= 1;
+  while (cs < cap && static_cast<long long>(cs) * 2 * p.B <= sm_count()) cs <<= 1;
   return cs;
 }
 

@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define DSV4_ABI_VERSION 1
+#define DSV4_ABI_VERSION 2
 
 typedef void *dsv4_stream; /* a cudaStream_t; NULL = the legacy default stream */
 
@@ -260,9 +260,16 @@ dsv4_status dsv4_indexer_topk_noalloc(const dsv4_indexer_args *args, dsv4_stream
  * every entry 0..n_entries[s)-1 (dense). V = K.
  *   o_h = RoPE_{-pos}( sum_j softmax_j( softmax_scale * RoPE_pos(q_h) . k_j ) * k_j )
  *   q [batch][heads][dim] in q_dtype (F32 or BF16), un-rotated; pos [batch] int32;
- *   out [batch][heads][dim] in out_dtype (F32 or BF16); lse [batch][heads] float32
+ *   out [batch][heads][dim] in out_dtype (F32, BF16 or FP8E4M3); lse [batch][heads] float32
  *   (natural log of the softmax denominator, optional).
  *   softmax_scale <= 0 means 1/sqrt(dim).
+ *   q_norm_gamma [dim] float32, optional ("vLLM side": the fused "Q-norm + KV RoPE + K
+ *   insert" kernel): each query head is first RMS-normed over its dim values with this
+ *   weight and q_norm_eps, before RoPE; NULL: no query norm.
+ *   FP8E4M3 output ("vLLM side": the fused "inverse RoPE + fp8 quant" kernel): each head's
+ *   output, after its inverse RoPE, is stored in blocks of 128 channels as e4m3 codes with one
+ *   float32 scale amax/448 per block (1 if the block is all zero) in out_scales
+ *   [batch][heads][dim/128] (value = code * scale); dim must be a multiple of 128.
  * cache and ring share dim and dtype (F32, BF16 or FP8E4M3). BF16/FP8 caches with dim 512
  * and heads 64 run on the tensor cores (tcgen05; bf16 operands for BF16 caches, fp16
  * operands holding the exact e4m3 codes with their row scales for FP8 caches; fp32
@@ -289,6 +296,9 @@ typedef struct {
   dsv4_dtype out_dtype;
   float *lse;
   uint32_t *d_status;
+  const float *q_norm_gamma; /* [dim] or NULL */
+  float q_norm_eps;
+  float *out_scales;         /* [batch][heads][dim/128] for FP8E4M3 output */
 } dsv4_mqa_args;
 
 size_t dsv4_mqa_workspace_size(const dsv4_mqa_args *args);
@@ -328,6 +338,7 @@ typedef struct {
   dsv4_window_ring ring;            /* raw window keys */
   dsv4_compressor_state idx_state;  /* C4 only */
   dsv4_paged_cache idx_cache;       /* C4 only */
+  const float *gamma_q;             /* [dim]: query norm weight (eps as above); NULL: none */
 } dsv4_layer;
 
 typedef struct {
@@ -346,9 +357,10 @@ typedef struct {
   const void *w;          /* [batch][idx_heads] */
   dsv4_dtype w_dtype;
   void *out;              /* [batch][heads][dim] */
-  dsv4_dtype out_dtype;
+  dsv4_dtype out_dtype;   /* F32, BF16 or FP8E4M3 (128-channel blocks, see dsv4_mqa_args) */
   int32_t *topk_idx;      /* optional [batch][topk]: the selected entries (C4) */
   uint32_t *d_status;
+  float *out_scales;      /* [batch][heads][dim/128] for FP8E4M3 output */
 } dsv4_step;
 
 size_t dsv4_hybrid_decode_workspace_size(const dsv4_layer *layer, int32_t batch);

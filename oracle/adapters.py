@@ -41,6 +41,8 @@ def layer_state(la) -> O.LayerState:
                                 la.scales.copy(), la.block_table.copy()),
         window=O.WindowRing(spec.swa_dtype, spec.W, spec.D, la.swa_rows.copy(),
                             la.swa_scales.copy()))
+    if getattr(la, "gamma_q", None) is not None:
+        st.gamma_q = la.gamma_q.astype(np.float64)
     if spec.kind == "c4":
         st.gamma_idx = la.gamma_idx.astype(np.float64)
         st.idx_state = O.CompressorState(spec.m, spec.d_I, spec.d_I, la.idx_state.copy())

@@ -110,7 +110,8 @@ class LayerSpec:
     q_dtype: str = "bf16"       # query
     q_idx_dtype: str = "fp8"    # indexer query
     w_dtype: str = "bf16"       # indexer head weights
-    out_dtype: str = "bf16"
+    out_dtype: str = "bf16"     # f32, bf16 or fp8 (128-channel blocks)
+    q_norm: bool = False        # the layer RMS-norms each query head before RoPE
 
     @property
     def per_page(self) -> int:
@@ -133,6 +134,7 @@ class LayerArrays:
     idx_scales: np.ndarray | None = None
     idx_block_table: np.ndarray | None = None
     idx_state: np.ndarray | None = None
+    gamma_q: np.ndarray | None = None  # [D] float32 query norm weight (q_norm layers)
 
     @property
     def max_entries(self) -> int:
@@ -193,6 +195,8 @@ def make_layer(spec: LayerSpec, B: int, context_entries: int, seed: int, *,
     la = LayerArrays(spec=spec, B=B, gamma=np.ones(spec.D, dtype=np.float32), pages=pages,
                      scales=scales, block_table=bt, swa_rows=swa_rows, swa_scales=swa_scales,
                      state=state)
+    if spec.q_norm:
+        la.gamma_q = (1.0 + 0.1 * normal_f32(rng, (spec.D,))).astype(np.float32)
     if spec.kind == "c4":
         la.gamma_idx = np.ones(spec.d_I, dtype=np.float32)
         la.idx_pages, la.idx_scales = synth_rows(rng, (num_pages, per_page, spec.d_I),

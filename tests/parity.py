@@ -116,6 +116,35 @@ def check_output(got, want, inputs: str, ctx: str = "", out_dtype: str = "f32"):
     return err.max(), rel
 
 
+def e4m3_step(v, scale) -> np.ndarray:
+    """Spacing of the e4m3 grid (times `scale`) at |v|: 2^(floor(log2(|v|/scale)) - 3) for
+    normal codes, 2^-9 below 2^-6 (the subnormal spacing)."""
+    a = np.abs(np.asarray(v, np.float64)) / np.asarray(scale, np.float64)
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -6)))
+    return np.exp2(e - 3) * np.asarray(scale, np.float64)
+
+
+def check_output_fp8(codes, scales, want, inputs: str, ctx: str = ""):
+    """An fp8 output (e4m3 codes [H, D] with one scale per 128-channel block, R22) against the
+    oracle's output rounded the same way (its own block scales): within the bound plus one
+    e4m3 step of the rounded value, and rel-L2 within the bound."""
+    codes = np.asarray(codes, np.uint8)
+    scales = np.asarray(scales, np.float32)
+    H, D = codes.shape
+    blk = O.OUT_BLOCK
+    got = O.e4m3_decode(codes) * np.repeat(scales.astype(np.float64), blk, axis=1)
+    _, wsc, want_q = O.store_output(np.asarray(want, np.float64), "fp8")
+    step = e4m3_step(want_q, np.repeat(wsc.astype(np.float64), blk, axis=1))
+    bound = F32_MAX_ABS if inputs == "f32" else LOWP_MAX_ABS
+    err = np.abs(got - want_q)
+    assert np.all(np.isfinite(got)), f"{ctx}: non-finite output"
+    assert np.all(err <= bound + step), f"{ctx}: max-abs {err.max():.3e} > {bound} (+ one e4m3 step)"
+    assert np.all(np.abs(scales.astype(np.float64) - wsc) <= 2e-2 * wsc), f"{ctx}: block scales"
+    rel = np.linalg.norm(got - want_q) / max(np.linalg.norm(want_q), 1e-30)
+    assert rel <= LOWP_REL_L2, f"{ctx}: rel-L2 {rel:.3e} > {LOWP_REL_L2}"
+    return err.max(), rel
+
+
 def decode_out(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 

@@ -13,7 +13,8 @@ import compressed_sparse_kv_dsv4_b200 as dsv4
 import oracle.dsv4_oracle as O
 import synthetic as W
 from oracle import adapters as OA
-from tests.parity import check_output, check_topk, codes_close, decode_out, input_class, require_gpu
+from tests.parity import (check_output, check_output_fp8, check_topk, codes_close, decode_out, input_class,
+                          require_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -294,14 +295,15 @@ def _mqa_case(spec, B, pos, n_entries, idx=None, seed=41, value_std=1.0, out_dty
     return decode_out(out), lse.cpu().numpy(), status.item(), ol, qd, st
 
 
-def _ref_attention(ol, qd, st, s, sel, spec):
+def _ref_attention(ol, qd, st, s, sel, spec, gamma_q=None):
     p = int(st.pos[s])
     parts = [ol.window.read(s, O.window_positions(p, spec.W))]
     if len(sel):
         parts.append(ol.main_cache.read(s, np.asarray(sel)))
     keys = np.concatenate(parts)
-    o = O.shared_kv_attention(qd[s], p, keys, 1 / np.sqrt(spec.D), spec.rope_dims, spec.rope_base)
-    qr = O.apply_rope(qd[s], p, spec.rope_dims, spec.rope_base)
+    q = qd[s] if gamma_q is None else O.query_norm(qd[s], gamma_q, spec.eps)
+    o = O.shared_kv_attention(q, p, keys, 1 / np.sqrt(spec.D), spec.rope_dims, spec.rope_base)
+    qr = O.apply_rope(q, p, spec.rope_dims, spec.rope_base)
     lg = qr @ keys.T / np.sqrt(spec.D)
     lse = lg.max(1) + np.log(np.exp(lg - lg.max(1, keepdims=True)).sum(1))
     return o, lse
@@ -379,3 +381,55 @@ def test_mqa_cuda_core_fp32():
         o, l = _ref_attention(ol, qd, st, s, sel, spec)
         check_output(out[s], o, "f32", f"seq {s}")
         assert np.max(np.abs(lse[s] - l)) < 1e-4
+
+
+@pytest.mark.parametrize("B", [3, 40])  # clusters of 4 CTAs (one 128-column block each) and of 2 (two)
+def test_mqa_tensor_core_query_norm_fp8_output(B):
+    """Query norm before RoPE and fp8 output in 128-channel blocks, fused in the attention's
+    query preparation and merge epilogue."""
+    spec = W.C4_SPEC
+    n_c = 3000
+    rng = np.random.default_rng(9)
+    idx = np.stack([rng.permutation(n_c)[:512] for _ in range(B)]).astype(np.int64)
+    la = W.make_layer(spec, B, n_c + 1, 43, outlier_frac=0.05)
+    st = W.make_step(spec, B, [131072 - 7 * i for i in range(B)], 44, q_std=3.0)
+    gq = (1.0 + 0.2 * rng.standard_normal(spec.D)).astype(np.float32)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    q = dsv4.to_device_codes(st.q, spec.q_dtype, "cuda")
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    (codes, scales) = dsv4.sparse_mqa_decode(
+        q, torch.from_numpy(st.pos).cuda(), dl.cache, dl.ring, q_dtype=spec.q_dtype, out_dtype="fp8",
+        idx=torch.from_numpy(idx.astype(np.int32)).cuda(), n_entries=torch.full((B,), n_c, dtype=torch.int32,
+                                                                                device="cuda"),
+        rope_dims=spec.rope_dims, d_status=status, q_norm_gamma=torch.from_numpy(gq).cuda(), q_norm_eps=spec.eps)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    ol = OA.layer_state(la)
+    qd = OA.decode_input(st.q, spec.q_dtype)
+    codes, scales = codes.cpu().numpy(), scales.cpu().numpy()
+    for s_ in range(B):
+        o, _ = _ref_attention(ol, qd, st, s_, idx[s_], spec, gamma_q=gq.astype(np.float64))
+        check_output_fp8(codes[s_], scales[s_], o, "lowp", f"seq {s_}")
+
+
+def test_mqa_cuda_core_query_norm_fp8_output():
+    spec = W.TINY_SPEC
+    B = 2
+    rng = np.random.default_rng(10)
+    idx = np.stack([rng.permutation(1024)[:64] for _ in range(B)]).astype(np.int64)
+    la = W.make_layer(spec, B, 1025, 45)
+    st = W.make_step(spec, B, [4096, 300], 46)
+    gq = (1.0 + 0.2 * rng.standard_normal(spec.D)).astype(np.float32)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    (codes, scales) = dsv4.sparse_mqa_decode(
+        torch.from_numpy(st.q).cuda(), torch.from_numpy(st.pos).cuda(), dl.cache, dl.ring, q_dtype="f32",
+        out_dtype="fp8", idx=torch.from_numpy(idx.astype(np.int32)).cuda(),
+        n_entries=torch.full((B,), 1024, dtype=torch.int32, device="cuda"), rope_dims=spec.rope_dims,
+        q_norm_gamma=torch.from_numpy(gq).cuda(), q_norm_eps=spec.eps)
+    torch.cuda.synchronize()
+    ol = OA.layer_state(la)
+    qd = OA.decode_input(st.q, spec.q_dtype)
+    codes, scales = codes.cpu().numpy(), scales.cpu().numpy()
+    for s_ in range(B):
+        o, _ = _ref_attention(ol, qd, st, s_, idx[s_], spec, gamma_q=gq.astype(np.float64))
+        check_output_fp8(codes[s_], scales[s_], o, "f32", f"seq {s_}")

@@ -31,7 +31,8 @@ import compressed_sparse_kv_dsv4_b200 as dsv4
 import oracle.dsv4_oracle as O
 import synthetic as W
 from oracle import adapters as OA
-from tests.parity import check_output, check_step_writes, check_topk, codes_close, decode_out, input_class, require_gpu
+from tests.parity import (check_output, check_output_fp8, check_step_writes, check_topk, codes_close, decode_out,
+                          input_class, require_gpu)
 
 pytestmark = pytest.mark.gpu
 
@@ -61,7 +62,7 @@ def _step_and_check(dl, ol, spec, st, seqs=None, attend=True, must_select=None):
     if not attend:
         return 0, differ
     res = O.decode_attend(ol, oin, seqs)
-    out = decode_out(ds.out)
+    out = ds.out.cpu().numpy() if spec.out_dtype == "fp8" else decode_out(ds.out)
     idx = ds.topk_idx.cpu().numpy() if ds.topk_idx is not None else None
     swaps = 0
     for s, (o, sel, scores) in res.items():
@@ -72,7 +73,10 @@ def _step_and_check(dl, ol, spec, st, seqs=None, attend=True, must_select=None):
                 if must_select[s] not in differ[s]:
                     assert must_select[s] in set(idx[s].tolist()), f"seq {s}: new entry {must_select[s]} not selected"
             swaps += check_topk(idx[s], scores, spec.k, n_c, f"seq {s}", excused=differ[s])
-        check_output(out[s], o, input_class(spec), f"seq {s}", out_dtype=spec.out_dtype)
+        if spec.out_dtype == "fp8":
+            check_output_fp8(out[s], ds.out_scales[s].cpu().numpy(), o, input_class(spec), f"seq {s}")
+        else:
+            check_output(out[s], o, input_class(spec), f"seq {s}", out_dtype=spec.out_dtype)
     return swaps, differ
 
 
@@ -192,3 +196,21 @@ def test_c4_first_tokens_window_only(out_dtype):
     for i in range(3):
         st = W.make_step(spec, B, [0 + i, 1 + i, 2 + i], seed=62 + i)
         _step_and_check(dl, ol, spec, st)
+
+
+@pytest.mark.parametrize("kind", ["c4", "c128"])
+def test_query_norm_and_fp8_output_step(kind):
+    """A decode step of a layer with a query norm weight and fp8 outputs (128-channel blocks):
+    C4 (indexer, top-k, sparse attention; 3 sequences at ~9K context, one completing a block)
+    and C128 (dense; 8 sequences at 65K context)."""
+    if kind == "c4":
+        spec = dataclasses.replace(W.C4_SPEC, q_norm=True, out_dtype="fp8")
+        la = W.make_layer(spec, 3, 9000 // 4 + 4, seed=81, outlier_frac=0.05)
+        st = W.make_step(spec, 3, [9003, 9000, 9130], seed=82, q_std=2.0)
+    else:
+        spec = dataclasses.replace(W.C128_SPEC, q_norm=True, out_dtype="fp8")
+        la = W.make_layer(spec, 8, 65536 // 128, seed=83, value_std=1 / np.sqrt(512))
+        st = W.make_step(spec, 8, 65536, seed=84, q_std=1.0)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    ol = OA.layer_state(la)
+    _step_and_check(dl, ol, spec, st)

@@ -40,7 +40,7 @@ def test_every_declared_function_is_exported(lib):
 
 
 def test_host_helpers(lib, golden_dir):
-    assert lib.dsv4_abi_version() == 1
+    assert lib.dsv4_abi_version() == 2
     assert lib.dsv4_status_string(A.OK) == b"ok"
     assert lib.dsv4_status_string(A.ERR_INVALID_ARG) == b"invalid argument"
     assert lib.dsv4_status_string(99) == b"unknown status"
@@ -107,7 +107,9 @@ def test_validation_rejects_bad_calls(lib):
     # attention: bad shapes / pointers / dtypes
     for bad, code in ((dict(batch=0), A.ERR_INVALID_ARG), (dict(q=None), A.ERR_INVALID_ARG),
                       (dict(q=FAKE + 4), A.ERR_INVALID_ARG), (dict(dim=500), A.ERR_INVALID_ARG),
-                      (dict(q_dtype=A.FP8), A.ERR_UNSUPPORTED), (dict(out_dtype=A.FP8), A.ERR_UNSUPPORTED),
+                      (dict(q_dtype=A.FP8), A.ERR_UNSUPPORTED), (dict(out_dtype=A.FP8), A.ERR_INVALID_ARG),
+                      (dict(out_dtype=7), A.ERR_UNSUPPORTED),
+                      (dict(q_norm_gamma=FAKE, q_norm_eps=-1.0), A.ERR_INVALID_ARG),
                       (dict(rope=A.Rope(63, 1e4)), A.ERR_INVALID_ARG), (dict(n_entries=None), A.ERR_INVALID_ARG),
                       (dict(cache=_cache(scales=None)), A.ERR_INVALID_ARG),
                       (dict(cache=_cache(m=3)), A.ERR_INVALID_ARG),
@@ -115,6 +117,9 @@ def test_validation_rejects_bad_calls(lib):
         a = _mqa(**bad)
         assert lib.dsv4_sparse_mqa_decode(C.byref(a), C.c_void_p(FAKE), 1 << 30, None) == code, bad
         assert lib.dsv4_mqa_workspace_size(C.byref(a)) == 0
+    # fp8 output with its block scales, and a query norm, are accepted
+    assert lib.dsv4_mqa_workspace_size(C.byref(_mqa(out_dtype=A.FP8, out_scales=FAKE))) > 0
+    assert lib.dsv4_mqa_workspace_size(C.byref(_mqa(q_norm_gamma=FAKE, q_norm_eps=1e-6))) > 0
     # a too-small workspace is rejected before any launch
     a = _mqa()
     need = lib.dsv4_mqa_workspace_size(C.byref(a))
