@@ -85,6 +85,7 @@ EXPORTS = {
     "dsv4_indexer_workspace_size": (C.c_size_t, [C.POINTER(IndexerArgs)]),
     "dsv4_indexer_topk": (C.c_int, [C.POINTER(IndexerArgs), p, C.c_size_t, p]),
     "dsv4_indexer_topk_noalloc": (C.c_int, [C.POINTER(IndexerArgs), p]),
+    "dsv4_indexer_scores": (C.c_int, [C.POINTER(IndexerArgs), p, C.c_int64, p]),
     "dsv4_mqa_workspace_size": (C.c_size_t, [C.POINTER(MqaArgs)]),
     "dsv4_sparse_mqa_decode": (C.c_int, [C.POINTER(MqaArgs), p, C.c_size_t, p]),
     "dsv4_hybrid_decode_workspace_size": (C.c_size_t, [C.POINTER(Layer), i32]),

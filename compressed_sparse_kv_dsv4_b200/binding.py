@@ -282,6 +282,21 @@ def indexer_topk(q_idx, w, keys: DeviceCache, n_entries, k: int, *, q_dtype: str
     return idx, scores
 
 
+def indexer_scores(q_idx, w, keys: DeviceCache, n_entries, *, q_dtype: str, w_dtype: str, q_scale=None, out=None,
+                   d_status=None, stream=None):
+    """Every visible entry's indexer score, [B, ld] float32 (ld = the cache capacity rounded up
+    to 4); entries past n_entries are left as `out` held them."""
+    B = q_idx.shape[0]
+    cap = keys.block_table.shape[1] * (A.PAGE_POSITIONS // keys.m)
+    ld = (cap + 3) // 4 * 4
+    if out is None:
+        out = torch.full((B, ld), float("nan"), dtype=torch.float32, device=q_idx.device)
+    a = indexer_args(q_idx, w, keys, n_entries, 1, q_dtype=q_dtype, w_dtype=w_dtype, q_scale=q_scale,
+                     d_status=d_status)
+    A.check("dsv4_indexer_scores", A.load().dsv4_indexer_scores(C.byref(a), _ptr(out), out.shape[1], _stream(stream)))
+    return out
+
+
 def indexer_topk_noalloc(q_idx, w, keys: DeviceCache, n_entries, k: int, *, idx, q_dtype: str, w_dtype: str,
                          scores=None, q_scale=None, pos=None, q_rope_dims: int = 0, rope_base: float = 10000.0,
                          d_status=None, stream=None):

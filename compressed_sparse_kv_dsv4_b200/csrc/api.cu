@@ -227,6 +227,22 @@ dsv4_status dsv4_indexer_topk(const dsv4_indexer_args *a, void *ws, size_t ws_by
   return to_status(launch_indexer_topk(p, ws, static_cast<cudaStream_t>(stream)));
 }
 
+dsv4_status dsv4_indexer_scores(const dsv4_indexer_args *a, float *scores, int64_t scores_ld, dsv4_stream stream) {
+  if (!a) return DSV4_ERR_INVALID_ARG;
+  dsv4_indexer_args b = *a;
+  int32_t dummy_idx = 0;
+  if (!b.idx) b.idx = &dummy_idx;  // (the selection's output is not used here)
+  IndexerLaunch p;
+  const dsv4_status s = indexer_launch_args(&b, &p);
+  if (s != DSV4_OK) return s;
+  if (!indexer_uses_tensor_cores(p)) return DSV4_ERR_UNSUPPORTED;
+  if (!scores || (reinterpret_cast<uintptr_t>(scores) & 15u) || scores_ld < indexer_score_capacity(p) ||
+      scores_ld % 4 != 0)
+    return DSV4_ERR_INVALID_ARG;
+  p.idx = nullptr;
+  return to_status(launch_indexer_scores(p, scores, scores_ld, static_cast<cudaStream_t>(stream)));
+}
+
 // ------------------------------------------------------------------------------------
 static dsv4_status mqa_launch_args(const dsv4_mqa_args *a, MqaLaunch *p) {
   if (!a) return DSV4_ERR_INVALID_ARG;

@@ -999,7 +999,7 @@ int tc_stages(int B) {
 }
 
 template <int H>
-cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st) {
+cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st, int64_t ld = 0) {
   TcParams tp{};
   if (!make_rows_map(&tp.tmap_k, p.k_pages, static_cast<uint64_t>(p.num_pages) * kPerPage, kPerPage))
     return cudaErrorInvalidValue;
@@ -1016,10 +1016,10 @@ cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st) {
   tp.n_entries = p.n_entries;
   tp.pos = p.pos;
   tp.scores = scores;
-  tp.ld = score_ld(p);
+  tp.ld = ld > 0 ? ld : score_ld(p);
   tp.d_status = p.d_status;
   tp.before_append = p.before_append ? 1 : 0;
-  tp.release = 1;
+  tp.release = p.idx != nullptr || p.release_next ? 1 : 0;  // the top-k kernel, or a kernel of the call, follows
   // six stages in flight where shared memory allows, else five
   const size_t tail = tc_tail_bytes(p.B);
   if (tc_stages<H>(p.B) == 6) {
@@ -1052,6 +1052,14 @@ size_t indexer_workspace_bytes(const IndexerLaunch &p) {
 
 cudaError_t launch_indexer_topk(const IndexerLaunch &p0, void *ws, cudaStream_t st) {
   return launch_indexer_part(p0, ws, st, 0);
+}
+
+int64_t indexer_score_capacity(const IndexerLaunch &p) { return capacity_of(p); }
+
+cudaError_t launch_indexer_scores(const IndexerLaunch &p, float *scores, int64_t ld, cudaStream_t st) {
+  IndexerLaunch q = p;
+  q.release_next = false;
+  return q.H == 32 ? launch_tc<32>(q, scores, st, ld) : launch_tc<64>(q, scores, st, ld);
 }
 
 cudaError_t launch_indexer_part(const IndexerLaunch &p0, void *ws, cudaStream_t st, int part) {

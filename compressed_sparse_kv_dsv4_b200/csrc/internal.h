@@ -139,6 +139,9 @@ struct IndexerLaunch {
 bool indexer_uses_tensor_cores(const IndexerLaunch &p);
 size_t indexer_workspace_bytes(const IndexerLaunch &p);
 cudaError_t launch_indexer_topk(const IndexerLaunch &p, void *ws, cudaStream_t st);
+// the scoring kernel alone (tensor-core path), into scores [B][ld], ld >= the capacity
+int64_t indexer_score_capacity(const IndexerLaunch &p);
+cudaError_t launch_indexer_scores(const IndexerLaunch &p, float *scores, int64_t ld, cudaStream_t st);
 // part 1: the scoring kernel only (tensor-core path); part 2: the top-k only; 0: both
 cudaError_t launch_indexer_part(const IndexerLaunch &p, void *ws, cudaStream_t st, int part);
 

@@ -224,6 +224,18 @@ dsv4_status dsv4_indexer_topk(const dsv4_indexer_args *args, void *workspace,
                               size_t workspace_bytes, dsv4_stream stream);
 
 /* ------------------------------------------------------------------------------------
+ * dsv4_indexer_scores: the lightning indexer's scores alone, without the selection (the first
+ * half of dsv4_indexer_topk, for a caller that selects by itself): scores[s * scores_ld + j] =
+ * s_j for every j < n_entries[s] (the same values dsv4_indexer_topk selects from; -inf where an
+ * entry's page is invalid); the rest of each row is left as it is. Same arguments as
+ * dsv4_indexer_topk (idx and the args' scores are not used). The tensor-core shapes only
+ * (DSV4_ERR_UNSUPPORTED otherwise). scores: device float32, 16-byte aligned; scores_ld a
+ * multiple of 4, at least keys.max_blocks * 256 / keys.m. No workspace.
+ */
+dsv4_status dsv4_indexer_scores(const dsv4_indexer_args *args, float *scores, int64_t scores_ld,
+                                dsv4_stream stream);
+
+/* ------------------------------------------------------------------------------------
  * dsv4_indexer_topk_noalloc: dsv4_indexer_topk on scratch the library owns. The pages have
  * no counterpart to this call: it is a convenience of the library, not a step of the method.
  * Same arguments, kernels and results as dsv4_indexer_topk; no workspace argument.

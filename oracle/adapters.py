@@ -21,6 +21,8 @@ def decode_input(codes, dtype: str, scales=None) -> np.ndarray:
         return O.bf16_decode(codes)
     if dtype == "fp8":
         return O.e4m3_decode(codes) * np.asarray(scales, np.float32).astype(np.float64)[..., None]
+    if dtype == "fp4":
+        return O.decode_rows(codes, scales, "fp4")
     raise ValueError(dtype)
 
 

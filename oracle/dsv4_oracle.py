@@ -68,6 +68,12 @@ Readings taken where both are silent (the plainest one the text supports):
       kernel): when a layer has a query norm weight, each query head is
       RMS-normed over its D dims with that weight and the layer's eps before its
       RoPE, like the window key of R4.
+  R23 fp4 indexer cache ([vLLM] "four moves": "fp8 attention cache + fp4
+      indexer cache"): an fp4 row is OCP e2m1 codes (1 sign, 2 exponent bits
+      with bias 1, 1 mantissa bit: magnitudes 0, 0.5, 1, 1.5, 2, 3, 4, 6), two
+      per byte with the even element in the low nibble, plus one float32 scale
+      amax/6 per row (1 if amax = 0); code = RNE_satfinite(x * (6/amax)), the
+      rule of R12 with 6 the largest e2m1 magnitude.
   R22 fp8 output ([vLLM] "vLLM side": the fused "inverse RoPE + fp8 quant"
       kernel): the output of each head, after its inverse RoPE, is stored as
       e4m3 codes in blocks of 128 channels, each block with one float32 scale
@@ -128,6 +134,61 @@ def e4m3_encode(x) -> np.ndarray:
     take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
     mag = np.where(take_hi, hi, lo).astype(np.uint8)
     return mag | np.where(np.signbit(x), 0x80, 0).astype(np.uint8)
+
+
+# OCP 4-bit floating point, E2M1: 1 sign bit, 2 exponent bits with bias 1, 1
+# mantissa bit, no infinities or NaN, largest finite 6 (reading R23).
+
+E2M1_MAX = 6.0
+
+
+def _e2m1_value(code: int) -> float:
+    sign = -1.0 if code & 0x8 else 1.0
+    exp = (code >> 1) & 0x3
+    man = code & 0x1
+    if exp == 0:  # subnormal: 0.m * 2^(1-bias)
+        return sign * (man / 2.0)
+    return sign * (1.0 + man / 2.0) * 2.0 ** (exp - 1)
+
+
+E2M1_VALUES = np.array([_e2m1_value(c) for c in range(16)], dtype=np.float64)
+_E2M1_POS = E2M1_VALUES[:8]  # codes 0..7: 0 .. 6, increasing
+
+
+def e2m1_decode(codes) -> np.ndarray:
+    """e2m1 codes (0..15) -> float64 values, from the format definition."""
+    return E2M1_VALUES[np.asarray(codes, dtype=np.uint8) & 0xF]
+
+
+def e2m1_encode(x) -> np.ndarray:
+    """float32 values -> e2m1 codes (0..15): round to nearest, ties to the even
+    mantissa, saturating at 6; a value rounding to zero keeps its sign (code 8)."""
+    x = np.asarray(x, dtype=np.float32).astype(np.float64)
+    if not np.all(np.isfinite(x)):
+        raise ValueError("e2m1_encode: non-finite input")
+    a = np.minimum(np.abs(x), E2M1_MAX)
+    hi = np.minimum(np.searchsorted(_E2M1_POS, a, side="left"), 7)
+    lo = np.maximum(hi - 1, 0)
+    d_hi = _E2M1_POS[hi] - a
+    d_lo = a - _E2M1_POS[lo]
+    take_hi = (d_hi < d_lo) | ((d_hi == d_lo) & (hi % 2 == 0))
+    mag = np.where(take_hi, hi, lo).astype(np.uint8)
+    return mag | np.where(np.signbit(x), 0x8, 0).astype(np.uint8)
+
+
+def fp4_pack(codes) -> np.ndarray:
+    """e2m1 codes [..., D] -> bytes [..., D/2], element 2i in the low nibble."""
+    c = np.asarray(codes, dtype=np.uint8)
+    return (c[..., 0::2] & 0xF) | ((c[..., 1::2] & 0xF) << 4)
+
+
+def fp4_unpack(packed) -> np.ndarray:
+    """bytes [..., D/2] -> e2m1 codes [..., D]."""
+    b = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(b.shape[:-1] + (2 * b.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = b & 0xF
+    out[..., 1::2] = b >> 4
+    return out
 
 
 def bf16_decode(bits) -> np.ndarray:
@@ -231,6 +292,16 @@ def store(x, dtype: str):
             inv = np.float32(np.float32(E4M3_MAX) / amax)
         codes = e4m3_encode((x32 * inv).astype(np.float32))
         return codes, scale, e4m3_decode(codes) * np.float64(scale)
+    if dtype == "fp4":  # reading R23: packed e2m1 codes, one scale amax/6
+        amax = np.float32(np.max(np.abs(x32)))
+        if amax == 0:
+            scale = np.float32(1.0)
+            inv = np.float32(1.0)
+        else:
+            scale = np.float32(amax / np.float32(E2M1_MAX))
+            inv = np.float32(np.float32(E2M1_MAX) / amax)
+        codes = e2m1_encode((x32 * inv).astype(np.float32))
+        return fp4_pack(codes), scale, e2m1_decode(codes) * np.float64(scale)
     raise ValueError(dtype)
 
 
@@ -242,6 +313,8 @@ def decode_rows(codes, scales, dtype: str) -> np.ndarray:
         return bf16_decode(codes)
     if dtype == "fp8":
         return e4m3_decode(codes) * np.asarray(scales, dtype=np.float32).astype(np.float64)[..., None]
+    if dtype == "fp4":
+        return e2m1_decode(fp4_unpack(codes)) * np.asarray(scales, dtype=np.float32).astype(np.float64)[..., None]
     raise ValueError(dtype)
 
 
@@ -249,7 +322,7 @@ def decode_rows(codes, scales, dtype: str) -> np.ndarray:
 # caches and state (the same byte layout the library uses)
 # ---------------------------------------------------------------------------
 
-CODE_DTYPE = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8}
+CODE_DTYPE = {"f32": np.float32, "bf16": np.uint16, "fp8": np.uint8, "fp4": np.uint8}
 
 
 @dataclass
@@ -262,7 +335,7 @@ class PagedCache:
     dtype: str
     m: int
     D: int
-    pages: np.ndarray        # [num_pages, 256 // m, D] codes
+    pages: np.ndarray        # [num_pages, 256 // m, D] codes ([.., D/2] bytes for fp4)
     scales: np.ndarray       # [num_pages, 256 // m] float32 (fp8; ones otherwise)
     block_table: np.ndarray  # [B, max_blocks] int32
 

@@ -240,6 +240,30 @@ def test_indexer_many_short_sequences_topk_in_entry_order():
         assert np.all(np.diff(idx[s][v]) > 0), f"seq {s}: output not in ascending entry order"
 
 
+def test_indexer_scores_alone_match_oracle():
+    """dsv4_indexer_scores: every visible entry's score (the tensor-core kernel alone), rows
+    past n_entries untouched."""
+    spec = W.C4_SPEC
+    n_list = [130, 4097, 0, 600]
+    B = len(n_list)
+    la = W.make_layer(spec, B, max(n_list) + 1, 24, outlier_frac=0.05)
+    st = W.make_step(spec, B, 0, 25)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    out = dsv4.indexer_scores(dsv4.to_device_codes(st.q_idx, "fp8", "cuda"), dsv4.to_device_codes(st.w, "bf16", "cuda"),
+                              dl.idx_cache, torch.tensor(n_list, dtype=torch.int32, device="cuda"), q_dtype="fp8",
+                              w_dtype="bf16", q_scale=torch.from_numpy(st.q_idx_scale).cuda())
+    torch.cuda.synchronize()
+    got = out.cpu().numpy()
+    ol = OA.layer_state(la)
+    qd = OA.decode_input(st.q_idx, spec.q_idx_dtype, st.q_idx_scale)
+    wd = OA.decode_input(st.w, spec.w_dtype)
+    for s_, n in enumerate(n_list):
+        assert np.all(np.isnan(got[s_, n:])), f"seq {s_}: entries past n_entries were written"
+        if n:
+            ref = O.indexer_scores(qd[s_], wd[s_], ol.idx_cache.read(s_, np.arange(n)))
+            assert np.all(np.abs(got[s_, :n] - ref) <= 1e-5 * np.abs(ref).max()), f"seq {s_}"
+
+
 def test_indexer_full_tie_takes_lowest_indices():
     idx, scores, ol, qd, wd = _indexer_case([3000, 700], 512, all_negative=True)
     for s in range(2):

@@ -126,6 +126,14 @@ def test_validation_rejects_bad_calls(lib):
     assert need > 0
     assert lib.dsv4_sparse_mqa_decode(C.byref(a), C.c_void_p(FAKE), need - 1, None) == A.ERR_INVALID_ARG
     assert lib.dsv4_sparse_mqa_decode(C.byref(a), C.c_void_p(FAKE + 16), need, None) == A.ERR_INVALID_ARG
+    # indexer scores alone: the tensor-core shapes, an aligned output with a wide enough stride
+    ia = _indexer()
+    cap = ia.keys.max_blocks * (256 // ia.keys.m)
+    assert lib.dsv4_indexer_scores(None, C.c_void_p(FAKE), cap, None) == A.ERR_INVALID_ARG
+    assert lib.dsv4_indexer_scores(C.byref(ia), None, cap, None) == A.ERR_INVALID_ARG
+    assert lib.dsv4_indexer_scores(C.byref(ia), C.c_void_p(FAKE + 4), cap, None) == A.ERR_INVALID_ARG
+    assert lib.dsv4_indexer_scores(C.byref(ia), C.c_void_p(FAKE), cap - 4, None) == A.ERR_INVALID_ARG
+    assert lib.dsv4_indexer_scores(C.byref(_indexer(q_dtype=A.F32)), C.c_void_p(FAKE), cap, None) == A.ERR_UNSUPPORTED
     # indexer
     for bad, code in ((dict(k=0), A.ERR_INVALID_ARG), (dict(idx=None), A.ERR_INVALID_ARG),
                       (dict(dim=64), A.ERR_INVALID_ARG), (dict(q_dtype=A.BF16), A.ERR_UNSUPPORTED),

@@ -382,3 +382,48 @@ def test_fp8_output_blocks_hand_example():
     inv = np.float32(np.float32(448.0) / np.float32(1.0))
     lib = torch.from_numpy(np.float32(o[0, :128]).astype(np.float32) * inv).to(torch.float8_e4m3fn)
     assert np.array_equal(codes[0, :128], lib.view(torch.uint8).numpy())
+
+
+# ----------------------------------------------------------------- fp4 indexer cache (R23)
+def test_e2m1_codes_from_the_format_definition():
+    """All 16 e2m1 codes: the OCP E2M1 table (sign, 2 exponent bits with bias 1, 1 mantissa
+    bit), written out by hand."""
+    table = [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert list(O.E2M1_VALUES[:8]) == table
+    assert list(O.E2M1_VALUES[8:]) == [-v for v in table]
+    assert np.signbit(O.E2M1_VALUES[8])
+
+
+def test_e2m1_encode_is_nearest_with_ties_to_even():
+    """Against brute force: the nearest of the 8 magnitudes, an exact tie going to the code
+    with an even mantissa bit; saturation at 6; the sign kept, also for values rounding to 0."""
+    x = np.concatenate([RNG.uniform(-8, 8, 20000), np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25,
+                                                              -5.0, 7.0, -100.0, 1e-9, -1e-9, 0.0])]).astype(np.float32)
+    got = O.e2m1_encode(x)
+    mags = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    for v, c in zip(x.astype(np.float64), got):
+        a = min(abs(v), 6.0)
+        d = np.abs(mags - a)
+        best = np.flatnonzero(d == d.min())
+        want = best[0] if len(best) == 1 else [b for b in best if b % 2 == 0][0]
+        assert (c & 7) == want and bool(c & 8) == bool(np.signbit(v)), (v, c)
+    # the hand-picked ties
+    assert list(O.e2m1_encode(np.float32([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]))) == [0, 2, 2, 4, 4, 6, 6]
+
+
+def test_fp4_rows_pack_and_scale():
+    x = RNG.standard_normal(128) * 2.0
+    packed, scale, dec = O.store(x, "fp4")
+    assert packed.shape == (64,) and packed.dtype == np.uint8
+    amax = np.float32(np.max(np.abs(np.float32(x))))
+    assert scale == np.float32(amax / np.float32(6.0))
+    codes = O.fp4_unpack(packed)
+    assert np.array_equal(O.fp4_pack(codes), packed)
+    assert codes[np.argmax(np.abs(x))] & 7 == 7  # the largest value maps to 6
+    assert np.array_equal(dec, O.decode_rows(packed[None], np.array([scale]), "fp4")[0])
+    # even elements in the low nibble
+    p2 = O.fp4_pack(np.array([3, 12], np.uint8))
+    assert p2[0] == 0xC3
+    # e2m1 keeps 1 mantissa bit: relative error <= 1/4 above the subnormal range
+    big = np.abs(x) >= float(scale)
+    assert np.all(np.abs(dec[big] - x[big]) <= 0.25 * np.abs(x[big]) + 1e-12)
