@@ -39,7 +39,7 @@ UNIT = "tokens/s"
 SPEC_ROWS = dict(D=512, H=64, k=512, W=128, H_I=64, d_I=128)
 
 
-def algorithmic_bytes_per_seq(n_c: int, out_bytes: int = 2) -> dict:
+def algorithmic_bytes_per_seq(n_c: int, out_bytes: int = 2, idx_row_bytes: int = SPEC_ROWS["d_I"]) -> dict:
     """Bytes one sequence's decode step must move (fp8 caches with a 4-byte row scale).
 
     indexer: every visible indexer key row (128 B + scale); attention: the k selected
@@ -49,9 +49,9 @@ def algorithmic_bytes_per_seq(n_c: int, out_bytes: int = 2) -> dict:
     slots (float32) and the window row written; the indexer query, its scales and weights.
     """
     D, H, k, W, H_I, d_I = (SPEC_ROWS[x] for x in ("D", "H", "k", "W", "H_I", "d_I"))
-    idx = n_c * (d_I + 4)
+    idx = n_c * (idx_row_bytes + 4)  # idx_row_bytes: d_I for fp8 keys, d_I / 2 for fp4
     attn = (k + W) * (D + 4) + H * D * 2 + H * D * out_bytes
-    upd = 2 * D * 2 + 2 * d_I * 2 + 2 * D * 4 + 2 * d_I * 4 + (D + 4)
+    upd = 2 * D * 2 + 2 * d_I * 2 + 2 * D * 4 + 2 * d_I * 4 + (D + 4)  # appended cache rows: under 1/m per step
     qidx = H_I * d_I + H_I * 4 + H_I * 2
     return dict(indexer=idx + qidx, attention=attn, updates=upd, total=idx + qidx + attn + upd)
 
@@ -370,6 +370,59 @@ def leg_stack_1m(lib, dev, stream, flush, hbm_peak: float, steps: int = 16) -> d
     return res
 
 
+def leg_c4_fp4_indexer(lib, dev, stream, flush, hbm_peak: float, steps: int = 50) -> dict:
+    """The benchmark's C4 step (32 sequences, 131072-token context) with an fp4 (e2m1)
+    indexer-key cache: 64 bytes + a float32 scale per entry instead of 128 + 4. One step =
+    one dsv4_hybrid_decode call; the scoring kernel is also timed alone."""
+    import torch
+
+    import compressed_sparse_kv_dsv4_b200 as dsv4
+    from compressed_sparse_kv_dsv4_b200 import _abi as A
+    from compressed_sparse_kv_dsv4_b200.binding import indexer_args
+    import synthetic as W
+
+    spec = W.C4_FP4_SPEC
+    la, sets = W.c4_sparse(seed=7, B=B_PER_GPU, context=CONTEXT, steps=1, spec=spec)
+    dl = dsv4.DeviceLayer.from_arrays(la, dev)
+    ds = dsv4.DeviceStep.from_arrays(spec, sets[0], dev)
+    total = steps + 3
+    pos = torch.tensor([[CONTEXT + (i % POS_CYCLE)] * B_PER_GPU for i in range(total)], dtype=torch.int32,
+                       device=dev)
+    ws = dl.workspace(B_PER_GPU)
+    L = dl.struct()
+    Ss = []
+    for i in range(total):
+        S = ds.struct()
+        S.pos = pos[i].data_ptr()
+        Ss.append(S)
+    sh = C.c_void_p(stream.cuda_stream)
+    n0 = lib.dsv4_launch_count()
+    ms = event_mean_ms(stream, lambda i: A.check("dsv4_hybrid_decode", lib.dsv4_hybrid_decode(
+        C.byref(L), C.byref(Ss[i]), C.c_void_p(ws.data_ptr()), ws.numel(), sh)), steps, flush, warm=3)
+    launches = (lib.dsv4_launch_count() - n0) // total
+    status = int(ds.d_status.item())
+    n_c = CONTEXT // spec.m
+    n_ent = torch.full((B_PER_GPU,), n_c, dtype=torch.int32, device=dev)
+    ia = indexer_args(ds.q_idx, ds.w, dl.idx_cache, n_ent, spec.k, q_dtype="fp8", w_dtype="bf16",
+                      q_scale=ds.q_idx_scale, d_status=ds.d_status)
+    sc_ld = (dl.idx_cache.block_table.shape[1] * (A.PAGE_POSITIONS // spec.m) + 3) // 4 * 4
+    sc_buf = torch.empty((B_PER_GPU, sc_ld), dtype=torch.float32, device=dev)
+    sc_ms = event_mean_ms(stream, lambda j: A.check("dsv4_indexer_scores", lib.dsv4_indexer_scores(
+        C.byref(ia), C.c_void_p(sc_buf.data_ptr()), sc_ld, sh)), steps, flush)
+    byts = algorithmic_bytes_per_seq(n_c, out_bytes=2, idx_row_bytes=spec.d_I // 2)
+    step_b, ix_b = byts["total"] * B_PER_GPU, byts["indexer"] * B_PER_GPU
+    res = {"workload": "c4_sparse_131k_fp4_indexer", "batch": B_PER_GPU, "context": CONTEXT,
+           "indexer_cache": "e2m1, 64 B + fp32 scale per entry", "ms_per_step": round(ms, 5),
+           "tokens_per_s": round(B_PER_GPU / (ms * 1e-3), 1), "step_algorithmic_bytes": step_b,
+           "step_frac": round(step_b / ms / 1e6 / hbm_peak, 4),
+           "indexer_scores_ms": round(sc_ms, 5), "indexer_algorithmic_bytes": ix_b,
+           "indexer_gbs": round(ix_b / sc_ms / 1e6, 1), "indexer_frac": round(ix_b / sc_ms / 1e6 / hbm_peak, 4),
+           "launches_per_step": launches, "device_status": status, "l2": "flushed between steps (256 MiB write)"}
+    del dl, ds, ws, sc_buf
+    torch.cuda.empty_cache()
+    return res
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_ours(args):
     import torch
@@ -539,6 +592,7 @@ def run_ours(args):
     }
     if world == 1 and not args.no_extra:
         line["compress_prefill"] = leg_compress_prefill(lib, dev, stream, flush, hbm_peak)
+        line["c4_fp4_indexer"] = leg_c4_fp4_indexer(lib, dev, stream, flush, hbm_peak)
         if not args.skip_1m:
             line["stack_1m"] = leg_stack_1m(lib, dev, stream, flush, hbm_peak)
     if world == 1 and not args.no_cpu_baseline:

@@ -7,7 +7,7 @@ import os
 
 from .build import LIB
 
-F32, BF16, FP8 = 0, 1, 2
+F32, BF16, FP8, FP4 = 0, 1, 2, 3
 LAYER_C4, LAYER_C128 = 0, 1
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_CUDA, ERR_SCRATCH_LIMIT = 0, 1, 2, 3, 4
 NOALLOC_SCRATCH_BYTES = 16 << 20
@@ -15,7 +15,7 @@ DEV_BAD_INDEX, DEV_BAD_PAGE, DEV_TIMEOUT, DEV_BAD_LENGTH = 1, 2, 4, 8
 PAGE_POSITIONS = 256
 OUT_BLOCK = 128  # channels per fp8 output block
 
-DTYPE_CODE = {"f32": F32, "bf16": BF16, "fp8": FP8}
+DTYPE_CODE = {"f32": F32, "bf16": BF16, "fp8": FP8, "fp4": FP4}
 
 p = C.c_void_p
 i32 = C.c_int32

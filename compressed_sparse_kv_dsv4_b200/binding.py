@@ -15,8 +15,8 @@ import torch
 
 from . import _abi as A
 
-DT = {"f32": A.F32, "bf16": A.BF16, "fp8": A.FP8}
-TORCH_CODE_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.uint8}
+DT = {"f32": A.F32, "bf16": A.BF16, "fp8": A.FP8, "fp4": A.FP4}
+TORCH_CODE_DTYPE = {"f32": torch.float32, "bf16": torch.bfloat16, "fp8": torch.uint8, "fp4": torch.uint8}
 
 
 def _ptr(t) -> int | None:
@@ -37,7 +37,7 @@ def to_device_codes(a: np.ndarray, dtype: str, device) -> torch.Tensor:
     a = np.ascontiguousarray(a)
     if dtype == "bf16":
         t = torch.from_numpy(a.view(np.int16)).view(torch.bfloat16)
-    elif dtype == "fp8":
+    elif dtype in ("fp8", "fp4"):  # e4m3 codes, or e2m1 codes packed two per byte
         t = torch.from_numpy(a.view(np.uint8))
     else:
         t = torch.from_numpy(a.astype(np.float32, copy=False))
@@ -48,7 +48,7 @@ def to_numpy_codes(t: torch.Tensor, dtype: str) -> np.ndarray:
     t = t.detach().cpu().contiguous()
     if dtype == "bf16":
         return t.view(torch.int16).numpy().view(np.uint16)
-    if dtype == "fp8":
+    if dtype in ("fp8", "fp4"):
         return t.view(torch.uint8).numpy()
     return t.float().numpy()
 
@@ -61,9 +61,13 @@ class DeviceCache:
     m: int
     dtype: str
 
+    @property
+    def dim(self) -> int:
+        return self.pages.shape[2] * (2 if self.dtype == "fp4" else 1)  # fp4 rows: dim/2 bytes
+
     def struct(self) -> A.PagedCache:
         return A.PagedCache(_ptr(self.pages), _ptr(self.scales), _ptr(self.block_table), self.pages.shape[0],
-                            self.block_table.shape[1], self.pages.shape[2], self.m, DT[self.dtype])
+                            self.block_table.shape[1], self.dim, self.m, DT[self.dtype])
 
 
 @dataclass

@@ -41,7 +41,10 @@ namespace {
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool valid_dtype(dsv4_dtype d) { return d == DSV4_F32 || d == DSV4_BF16 || d == DSV4_FP8E4M3; }
+// caches may also hold fp4 rows (indexer keys)
+bool valid_cache_dtype(dsv4_dtype d) { return valid_dtype(d) || d == DSV4_FP4E2M1; }
 size_t dsize(dsv4_dtype d) { return d == DSV4_F32 ? 4 : (d == DSV4_BF16 ? 2 : 1); }
+size_t row_bytes(dsv4_dtype d, int dim) { return d == DSV4_FP4E2M1 ? static_cast<size_t>(dim) / 2 : dim * dsize(d); }
 bool pow2(int x) { return x > 0 && (x & (x - 1)) == 0; }
 
 dsv4_status to_status(cudaError_t e) {
@@ -57,9 +60,11 @@ bool valid_rope(const dsv4_rope &r, int dim) {
 // a paged cache: pointers, dims, alignment
 bool valid_cache(const dsv4_paged_cache &c, bool need_scales_if_fp8 = true) {
   if (!c.pages || !c.block_table || c.num_pages <= 0 || c.max_blocks <= 0 || c.dim <= 0) return false;
-  if (!pow2(c.m) || c.m > DSV4_PAGE_POSITIONS || !valid_dtype(c.dtype)) return false;
-  if (!aligned16(c.pages) || (c.dim * dsize(c.dtype)) % 16 != 0) return false;
-  if (c.dtype == DSV4_FP8E4M3 && need_scales_if_fp8 && (!c.scales || !aligned16(c.scales))) return false;
+  if (!pow2(c.m) || c.m > DSV4_PAGE_POSITIONS || !valid_cache_dtype(c.dtype)) return false;
+  if (c.dtype == DSV4_FP4E2M1 && c.dim % 2 != 0) return false;
+  if (!aligned16(c.pages) || row_bytes(c.dtype, c.dim) % 16 != 0) return false;
+  if ((c.dtype == DSV4_FP8E4M3 || c.dtype == DSV4_FP4E2M1) && need_scales_if_fp8 && (!c.scales || !aligned16(c.scales)))
+    return false;
   return true;
 }
 
@@ -251,6 +256,7 @@ static dsv4_status mqa_launch_args(const dsv4_mqa_args *a, MqaLaunch *p) {
   if (!a->q || !a->pos || !a->out) return DSV4_ERR_INVALID_ARG;
   if (!valid_cache(a->cache) || !valid_ring(a->ring)) return DSV4_ERR_INVALID_ARG;
   if (a->cache.dim != a->dim || a->ring.dim != a->dim || a->cache.dtype != a->ring.dtype) return DSV4_ERR_INVALID_ARG;
+  if (a->cache.dtype == DSV4_FP4E2M1) return DSV4_ERR_UNSUPPORTED;  // fp4 is for indexer keys only
   if (a->idx && a->k <= 0) return DSV4_ERR_INVALID_ARG;
   if (!a->idx && !a->n_entries) return DSV4_ERR_INVALID_ARG;
   if (!valid_rope(a->rope, a->dim)) return DSV4_ERR_INVALID_ARG;
@@ -328,7 +334,7 @@ dsv4_status hybrid_plan(const dsv4_layer *L, const dsv4_step *S, int32_t batch, 
     return DSV4_ERR_INVALID_ARG;
   if (L->state.m != L->cache.m || L->state.dim != L->dim || L->cache.dim != L->dim || L->ring.dim != L->dim)
     return DSV4_ERR_INVALID_ARG;
-  if (L->cache.dtype != L->ring.dtype) return DSV4_ERR_UNSUPPORTED;
+  if (L->cache.dtype != L->ring.dtype || L->cache.dtype == DSV4_FP4E2M1) return DSV4_ERR_UNSUPPORTED;
   if (!valid_rope(L->rope, L->dim) || !(L->eps >= 0.f)) return DSV4_ERR_INVALID_ARG;
   if (!valid_pool_dim(L->dim)) return DSV4_ERR_UNSUPPORTED;
   if (c4) {

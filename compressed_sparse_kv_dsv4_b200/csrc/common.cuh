@@ -190,13 +190,40 @@ __device__ __forceinline__ void load_row_f(const void *base, dsv4_dtype dt, size
   }
 }
 
+// OCP e2m1 (1 sign, 2 exponent bits with bias 1, 1 mantissa bit): code -> value (exact)
+__device__ __forceinline__ float e2m1_to_float(uint32_t code) {
+  const uint32_t e = (code >> 1) & 3u, m = code & 1u;
+  // exponent 0: 0.m (0 or 0.5); otherwise 1.m * 2^(e - 1)
+  const float mag = e == 0 ? 0.5f * static_cast<float>(m) : __int_as_float(static_cast<int>((e + 126u) << 23 | m << 22));
+  return (code & 8u) ? -mag : mag;
+}
+
+// float -> e2m1 code: round to nearest, an exact tie to the even mantissa, saturating at 6; the
+// sign is kept (a value rounding to zero gives code 8 when negative). Between the
+// representable magnitudes 0, .5, 1, 1.5, 2, 3, 4, 6 the midpoints are .25, .75, 1.25, 1.75,
+// 2.5, 3.5, 5; at each the even code (mantissa 0: 0, 1, 2, 4) is the lower one for .25, 1.25,
+// 2.5, 5 and the upper one for .75, 1.75, 3.5.
+__device__ __forceinline__ uint32_t float_to_e2m1(float x) {
+  const float a = fabsf(x);
+  const uint32_t mag = (a > 0.25f) + (a >= 0.75f) + (a > 1.25f) + (a >= 1.75f) + (a > 2.5f) + (a >= 3.5f) + (a > 5.0f);
+  return mag | (signbit(x) ? 8u : 0u);
+}
+
 __device__ __forceinline__ float load_one_f(const void *base, dsv4_dtype dt, size_t off) {
   if (dt == DSV4_F32) return static_cast<const float *>(base)[off];
   if (dt == DSV4_BF16) return bf16_bits_to_float(static_cast<const uint16_t *>(base)[off]);
+  if (dt == DSV4_FP4E2M1) {  // element off: byte off / 2, the low nibble for even off
+    const uint8_t b = static_cast<const uint8_t *>(base)[off >> 1];
+    return e2m1_to_float((off & 1) ? (b >> 4) : (b & 15u));
+  }
   uint8_t c = static_cast<const uint8_t *>(base)[off];
   return e4m3x2_to_float2(c).x;
 }
 
+// bytes of n consecutive values of a row in `dt` (n even for fp4)
+__device__ __forceinline__ size_t dtype_bytes(dsv4_dtype dt, size_t n) {
+  return dt == DSV4_F32 ? 4 * n : (dt == DSV4_BF16 ? 2 * n : (dt == DSV4_FP4E2M1 ? n / 2 : n));
+}
 __device__ __forceinline__ size_t dtype_size(dsv4_dtype dt) { return dt == DSV4_F32 ? 4 : (dt == DSV4_BF16 ? 2 : 1); }
 
 // --------------------------------------------------------------------------------------
@@ -349,6 +376,13 @@ __device__ __forceinline__ uint64_t sw128_desc(uint32_t saddr, uint32_t lbo, uin
 // Instruction descriptors: fp32 accumulate; a_mn/b_mn = 1 for MN-major operands.
 __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+// kind::f8f6f4 with A in e2m1 (format 5; in shared memory as 16 values in the first 8 bytes of
+// each 16-byte chunk, the layout TMA's 16U4_ALIGN16B type writes) and B in e4m3
+__host__ __device__ constexpr uint32_t idesc_e2m1_e4m3(int M, int N) {
+  return (1u << 4) | (5u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 

@@ -107,7 +107,7 @@ __device__ __forceinline__ void *cache_row(void *pages, float *scales, const int
   }
   const size_t r = static_cast<size_t>(page) * per_page + static_cast<size_t>(j % per_page);
   *scale_ptr = scales ? scales + r : nullptr;
-  return static_cast<char *>(pages) + r * D * dtype_size(dt);
+  return static_cast<char *>(pages) + dtype_bytes(dt, r * D);
 }
 
 // items of sequence s: one per completed block, at least one (the state-tail write)
@@ -490,6 +490,20 @@ __device__ void compress_chunk(const CompressView &p, const PrefillShape &sh, fl
       *reinterpret_cast<uint4 *>(static_cast<uint16_t *>(row) + cg * 8) =
           make_uint4(pack_bf16x2(e[0], e[1]), pack_bf16x2(e[2], e[3]), pack_bf16x2(e[4], e[5]),
                      pack_bf16x2(e[6], e[7]));
+  } else if (p.cache_dt == DSV4_FP4E2M1) {  // e2m1 codes, two per byte, one scale amax/6
+    float am = 0.f;
+#pragma unroll
+    for (int c = 0; c < 8; ++c) am = fmaxf(am, fabsf(e[c]));
+    am = group_reduce(am, sh.R, red, true);
+    const float scale = am > 0.f ? __fdiv_rn(am, 6.0f) : 1.0f;
+    const float inv = am > 0.f ? __fdiv_rn(6.0f, am) : 1.0f;
+    if (row) {
+      uint32_t w = 0;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) w |= float_to_e2m1(__fmul_rn(e[c], inv)) << (4 * c);
+      *reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(row) + cg * 4) = w;
+      if (cg == 0 && sp) *sp = scale;
+    }
   } else {
     float am = 0.f;
 #pragma unroll

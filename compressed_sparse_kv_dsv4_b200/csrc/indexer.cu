@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(256) indexer_simt_kernel(const IndexerLaunch p
     report(p.d_status, DSV4_DEV_BAD_PAGE);
   } else {
     const size_t row = static_cast<size_t>(page) * per_page + static_cast<size_t>(j % per_page);
-    const float ks = p.k_dt == DSV4_FP8E4M3 ? p.k_scales[row] : 1.0f;
+    const float ks = (p.k_dt == DSV4_FP8E4M3 || p.k_dt == DSV4_FP4E2M1) ? p.k_scales[row] : 1.0f;
     float s = 0.f;
     for (int h = 0; h < H; ++h) {
       float dot = 0.f;
@@ -145,6 +145,7 @@ struct TcParams {
   int64_t ld;
   uint32_t *d_status;
   int before_append;  // score only the entries visible before this step's append (floor(pos / m))
+  int keys_fp4;       // keys are e2m1 (64 bytes per row in global memory) instead of e4m3
   int release;  // release the next kernel early (always: the top-k kernel follows)
 };
 
@@ -350,7 +351,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
         if (ok && k >= kStages && !mbar_wait(&S.empty[s], static_cast<uint32_t>((k / kStages - 1) & 1), &S.abort_flag))
           ok = 0;
         if (ok) {
-          mbar_arrive_expect_tx(&S.full[s], static_cast<uint32_t>(nt) * kTile * kRowBytes);
+          // (fp4 keys: the transaction counts the packed bytes read, half the tile)
+          mbar_arrive_expect_tx(&S.full[s], static_cast<uint32_t>(nt) * kTile * (p.keys_fp4 ? kRowBytes / 2 : kRowBytes));
           for (int t = 0; t < nt; ++t)
 #pragma unroll
             for (int h = 0; h < 2; ++h)
@@ -372,7 +374,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   } else if (warp == 1) {
     // ---------------- MMA issuer: stage k goes to accumulator set k % 2 (read by group k % 2)
     if (lane == 0) {
-      constexpr uint32_t idesc = idesc_e4m3(kTile, H);
+      const uint32_t idesc = p.keys_fp4 ? idesc_e2m1_e4m3(kTile, H) : idesc_e4m3(kTile, H);
       StageIter it;
       it.init(prefix, p.B, t0, t1);
       int sb, nt, seg = -1;
@@ -557,6 +559,7 @@ struct TopkOut {
 // c_h * ReLU(q_h . k) over the heads, their sum times the key's scale.
 struct AppendedKey {
   int enabled;
+  int fp4;               // keys in e2m1 (64 bytes per row) instead of e4m3
   const uint8_t *q;      // [B][H][128] e4m3 codes
   const float *q_scale;  // [B][H] or null (1)
   const void *w;         // [B][H]
@@ -577,19 +580,34 @@ __device__ float appended_score(const AppendedKey &ap, int b, int64_t j, float *
   const size_t row = valid ? static_cast<size_t>(page) * kPerPage + static_cast<size_t>(j % kPerPage) : 0;
   float acc = 0.f;
   if (h < ap.H && valid) {
-    const uint2 kq = *reinterpret_cast<const uint2 *>(ap.k_pages + row * kRowBytes + 8 * sub);
     const uint2 qq = *reinterpret_cast<const uint2 *>(ap.q + (static_cast<size_t>(b) * ap.H + h) * kRowBytes + 8 * sub);
-    const uint32_t kw[2] = {kq.x, kq.y}, qw[2] = {qq.x, qq.y};
+    const uint32_t qw[2] = {qq.x, qq.y};
+    float kv[8];
+    if (ap.fp4) {  // dims 8 sub .. +7: one 32-bit word of 8 nibbles
+      const uint32_t kw = *reinterpret_cast<const uint32_t *>(ap.k_pages + row * (kRowBytes / 2) + 4 * sub);
+#pragma unroll
+      for (int c = 0; c < 8; ++c) kv[c] = e2m1_to_float((kw >> (4 * c)) & 15u);
+    } else {
+      const uint2 kq = *reinterpret_cast<const uint2 *>(ap.k_pages + row * kRowBytes + 8 * sub);
+      const uint32_t kw[2] = {kq.x, kq.y};
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const float2 k0 = e4m3x2_to_float2(static_cast<uint16_t>(kw[u] & 0xFFFF));
+        const float2 k1 = e4m3x2_to_float2(static_cast<uint16_t>(kw[u] >> 16));
+        kv[4 * u] = k0.x;
+        kv[4 * u + 1] = k0.y;
+        kv[4 * u + 2] = k1.x;
+        kv[4 * u + 3] = k1.y;
+      }
+    }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const float2 k0 = e4m3x2_to_float2(static_cast<uint16_t>(kw[u] & 0xFFFF));
-      const float2 k1 = e4m3x2_to_float2(static_cast<uint16_t>(kw[u] >> 16));
       const float2 q0 = e4m3x2_to_float2(static_cast<uint16_t>(qw[u] & 0xFFFF));
       const float2 q1 = e4m3x2_to_float2(static_cast<uint16_t>(qw[u] >> 16));
-      acc = fmaf(q0.x, k0.x, acc);
-      acc = fmaf(q0.y, k0.y, acc);
-      acc = fmaf(q1.x, k1.x, acc);
-      acc = fmaf(q1.y, k1.y, acc);
+      acc = fmaf(q0.x, kv[4 * u], acc);
+      acc = fmaf(q0.y, kv[4 * u + 1], acc);
+      acc = fmaf(q1.x, kv[4 * u + 2], acc);
+      acc = fmaf(q1.y, kv[4 * u + 3], acc);
     }
   }
 #pragma unroll
@@ -948,16 +966,20 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
   return fn;
 }
 
-bool make_rows_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows) {
+// Rows of 128 values: e4m3 (128 bytes each), or e2m1 (fp4: 64 packed bytes each, landing in
+// shared memory as 128-byte rows with each 8 bytes of values followed by 8 bytes of gap, the
+// operand layout of the f8f6f4 MMA's e2m1 type). 128B swizzle either way.
+bool make_rows_map(CUtensorMap *map, const void *base, uint64_t rows, uint32_t box_rows, bool fp4 = false) {
   auto fn = get_encode_fn();
   if (!fn) return false;
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kRowBytes), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(kRowBytes)};
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(kRowBytes), static_cast<cuuint64_t>(rows)};  // values
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(fp4 ? kRowBytes / 2 : kRowBytes)};          // bytes
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(kRowBytes), box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  return fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  return fn(map, fp4 ? CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B : CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+            const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
 }
 
 int tc_grid() { return sm_count(); }
@@ -1001,8 +1023,10 @@ int tc_stages(int B) {
 template <int H>
 cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st, int64_t ld = 0) {
   TcParams tp{};
-  if (!make_rows_map(&tp.tmap_k, p.k_pages, static_cast<uint64_t>(p.num_pages) * kPerPage, kPerPage))
+  const bool fp4 = p.k_dt == DSV4_FP4E2M1;
+  if (!make_rows_map(&tp.tmap_k, p.k_pages, static_cast<uint64_t>(p.num_pages) * kPerPage, kPerPage, fp4))
     return cudaErrorInvalidValue;
+  tp.keys_fp4 = fp4 ? 1 : 0;
   if (!make_rows_map(&tp.tmap_q, p.q, static_cast<uint64_t>(p.B) * H, H)) return cudaErrorInvalidValue;
   tp.k_scales = p.k_scales;
   tp.block_table = p.block_table;
@@ -1037,7 +1061,9 @@ cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st, in
 }  // namespace
 
 bool indexer_uses_tensor_cores(const IndexerLaunch &p) {
-  return p.k_dt == DSV4_FP8E4M3 && p.q_dt == DSV4_FP8E4M3 && p.Dq == kRowBytes &&
+  const bool keys_ok = p.k_dt == DSV4_FP8E4M3 ||
+                       (p.k_dt == DSV4_FP4E2M1 && (reinterpret_cast<uintptr_t>(p.k_pages) & 31u) == 0);
+  return keys_ok && p.q_dt == DSV4_FP8E4M3 && p.Dq == kRowBytes &&
          (p.H == 32 || p.H == 64) && p.m == 4 && p.k >= 1 && p.k <= 2048 && p.q_rope_dims == 0 &&
          p.B <= 512 && static_cast<int64_t>(p.max_blocks) * (DSV4_PAGE_POSITIONS / p.m) <= kTkMaxCluster * kTkSlice;
 }
@@ -1081,6 +1107,7 @@ cudaError_t launch_indexer_part(const IndexerLaunch &p0, void *ws, cudaStream_t 
     AppendedKey ap{};
     if (p.before_append && !p.n_entries) {
       ap.enabled = 1;
+      ap.fp4 = p.k_dt == DSV4_FP4E2M1 ? 1 : 0;
       ap.q = static_cast<const uint8_t *>(p.q);
       ap.q_scale = p.q_scale;
       ap.w = p.w;

@@ -67,7 +67,11 @@ typedef enum {
   DSV4_ERR_SCRATCH_LIMIT = 4 /* the request needs more than the library's static scratch */
 } dsv4_status;
 
-typedef enum { DSV4_F32 = 0, DSV4_BF16 = 1, DSV4_FP8E4M3 = 2 } dsv4_dtype;
+/* DSV4_FP4E2M1 ("four moves": "fp4 indexer cache"): OCP e2m1 codes, two per byte (the even
+ * element in the low nibble), with one float32 scale amax/6 per row (value = e2m1 * scale).
+ * Indexer-key caches only (the keys of dsv4_indexer_topk, a C4 layer's idx_cache, and the cache
+ * dsv4_compress writes); a row of dim values is dim/2 bytes. */
+typedef enum { DSV4_F32 = 0, DSV4_BF16 = 1, DSV4_FP8E4M3 = 2, DSV4_FP4E2M1 = 3 } dsv4_dtype;
 
 typedef enum { DSV4_LAYER_C4 = 0, DSV4_LAYER_C128 = 1 } dsv4_layer_kind;
 
@@ -88,7 +92,8 @@ typedef enum { DSV4_LAYER_C4 = 0, DSV4_LAYER_C128 = 1 } dsv4_layer_kind;
  * codes; rows are contiguous). For DSV4_FP8E4M3, `scales` [num_pages][256/m] holds one
  * float32 per row (value = code * scale); it is ignored (may be NULL) otherwise.
  * m must be a power of two in [1, 256]. `pages` must be 16-byte aligned and dim*size(dtype)
- * a multiple of 16.
+ * a multiple of 16. For DSV4_FP4E2M1 rows are dim/2 bytes with one float32 scale each (scales
+ * required); dim/2 must be a multiple of 16.
  */
 typedef struct {
   void *pages;
@@ -190,11 +195,13 @@ dsv4_status dsv4_swa_insert(const dsv4_swa_insert_args *args, dsv4_stream stream
  * NULL it receives the matching s_j (-inf for padding).
  *   q_idx [batch][heads][dim] in q_dtype (DSV4_F32 or DSV4_FP8E4M3); q_scale [batch][heads]
  *   float32 (fp8 queries; NULL = 1); w [batch][heads] in w_dtype (F32 or BF16);
- *   keys: paged cache with keys.dim == dim, dtype F32 or FP8E4M3;
+ *   keys: paged cache with keys.dim == dim, dtype F32, FP8E4M3 or FP4E2M1;
  *   n_entries [batch] device int32 (<= keys.max_blocks * 256/keys.m);
  *   pos [batch] device int32 (used only when q_rope_dims > 0).
- * fp8 queries and keys with dim 128, heads 32 or 64, m == 4, no query RoPE and batch <= 512
- * run on the tensor cores (tcgen05, fed by TMA); other shapes run on a CUDA-core kernel.
+ * fp8 queries and fp8 or fp4 keys with dim 128, heads 32 or 64, m == 4, no query RoPE and
+ * batch <= 512 run on the tensor cores (tcgen05 kind::f8f6f4, e4m3 or e2m1 keys against e4m3
+ * queries, fed by TMA; fp4 pages must be 32-byte aligned); other shapes run on a CUDA-core
+ * kernel.
  * Both give the same entries. On the tensor-core path a second kernel selects each
  * sequence's top k from the streamed scores (one thread-block cluster per sequence) and writes
  * idx in ascending entry order.

@@ -27,6 +27,10 @@ import torch
 PAGE_POSITIONS = 256
 FP8_GAIN = 112.0          # synthetic e4m3 rows: codes of N(0,1)*112 (clipped), scale 1/112
 FP8_LIMIT = 448.0
+# synthetic e2m1 rows: magnitude codes 0..7 (values 0 .5 1 1.5 2 3 4 6) with about the frequencies
+# of N(0,1)*2 rounded to that grid, scale 1/2 (times the row's gain)
+FP4_CODE_PROBS = [0.10, 0.19, 0.18, 0.16, 0.13, 0.14, 0.07, 0.03]
+FP4_GAIN = 2.0
 
 
 def rng_for(seed: int) -> np.random.Generator:
@@ -78,6 +82,13 @@ def synth_rows(rng, shape, dtype: str, std: float = 1.0, row_gain=None):
     if dtype == "fp8":
         codes = fp8_codes(x * np.float32(FP8_GAIN))
         scales = (gain * np.float32(std / FP8_GAIN)).astype(np.float32)
+        return codes, scales
+    if dtype == "fp4":  # e2m1 codes drawn directly (magnitude codes 0..7, random sign), packed
+        mag = rng.choice(8, size=shape, p=FP4_CODE_PROBS).astype(np.uint8)
+        sign = (rng.random(shape) < 0.5).astype(np.uint8) << 3
+        c = mag | sign
+        codes = (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+        scales = (gain * np.float32(std / FP4_GAIN)).astype(np.float32)
         return codes, scales
     x *= np.float32(std)
     x *= gain[..., None]
@@ -306,6 +317,8 @@ C4_SPEC = LayerSpec(kind="c4", m=4, H=64, D=512, W=128, k=512, H_I=64, d_I=128,
                     idx_rope_dims=64, cache_dtype="fp8", swa_dtype="fp8", idx_dtype="fp8",
                     kv_dtype="bf16", q_dtype="bf16", q_idx_dtype="fp8", w_dtype="bf16",
                     out_dtype="bf16")
+# the same layer with an fp4 (e2m1) indexer-key cache
+C4_FP4_SPEC = replace(C4_SPEC, idx_dtype="fp4")
 
 
 def c128_dense_bf16(seed: int = 1, B: int = 8, context: int = 65536, steps: int = 1):

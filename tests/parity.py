@@ -169,6 +169,15 @@ def codes_close(gpu_codes, ref_codes, gpu_scales, ref_scales, dtype, ctx, max_fr
         return
     gs, rs = np.asarray(gpu_scales, np.float64), np.asarray(ref_scales, np.float64)
     assert np.all(np.abs(gs - rs) <= 1e-6 * rs), f"{ctx}: scales"
+    if dtype == "fp4":  # e2m1 codes two per byte: sign bit 3, magnitude codes 0..7 in value order
+        g = O.fp4_unpack(np.asarray(gpu_codes)).astype(np.int32)
+        r = O.fp4_unpack(np.asarray(ref_codes)).astype(np.int32)
+        same_sign = (g & 0x8) == (r & 0x8)
+        step = np.abs((g & 0x7) - (r & 0x7))
+        zero = ((g & 0x7) == 0) & ((r & 0x7) <= 1) | ((r & 0x7) == 0) & ((g & 0x7) <= 1)
+        assert np.all((same_sign & (step <= 1)) | zero), f"{ctx}: fp4 codes more than one step apart"
+        assert np.mean(g != r) <= max_frac, f"{ctx}: too many fp4 rounding differences"
+        return
     g = np.asarray(gpu_codes).astype(np.int32)
     r = np.asarray(ref_codes).astype(np.int32)
     same_sign = (g & 0x80) == (r & 0x80)

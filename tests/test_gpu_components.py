@@ -25,7 +25,8 @@ def _gpu():
 
 
 # ---------------------------------------------------------------------------- compressor
-@pytest.mark.parametrize("m,cache_dtype,D", [(4, "bf16", 512), (128, "fp8", 512), (4, "fp8", 128), (4, "f32", 32)])
+@pytest.mark.parametrize("m,cache_dtype,D", [(4, "bf16", 512), (128, "fp8", 512), (4, "fp8", 128), (4, "f32", 32),
+                                               (4, "fp4", 128)])
 def test_compress_prefill_matches_oracle(m, cache_dtype, D):
     rng = W.rng_for(11)
     lens = np.array([37, 300, 129], dtype=np.int32)
@@ -214,6 +215,21 @@ def test_indexer_tensor_core_topk_matches_oracle(k):
         assert np.all(np.abs(got - want) <= 1e-5 * np.abs(want).max()), f"seq {s}: scores"
 
 
+def test_indexer_tensor_core_fp4_keys_topk_matches_oracle():
+    """e2m1 keys (two per byte, one float32 scale per row) against fp8 queries, on the tensor
+    cores: scores and the top-k set equal the oracle's on the same codes."""
+    n_list = [130, 1000, 4097, 0, 600, 20000]
+    idx, scores, ol, qd, wd = _indexer_case(n_list, 512, seed=27, spec=W.C4_FP4_SPEC)
+    for s, n in enumerate(n_list):
+        if n == 0:
+            assert np.all(idx[s] == -1)
+            continue
+        ref = O.indexer_scores(qd[s], wd[s], ol.idx_cache.read(s, np.arange(n)))
+        check_topk(idx[s], ref, 512, n, f"seq {s}")
+        v = idx[s] >= 0
+        assert np.all(np.abs(scores[s][v] - ref[idx[s][v]]) <= 1e-5 * np.abs(ref).max()), f"seq {s}: scores"
+
+
 def test_indexer_tensor_core_long_sequences_topk_matches_oracle():
     """Sequences of 46K-70K entries: top-k clusters of more CTAs, slices of 24 keys per
     thread, an empty sequence beside them."""
@@ -240,10 +256,11 @@ def test_indexer_many_short_sequences_topk_in_entry_order():
         assert np.all(np.diff(idx[s][v]) > 0), f"seq {s}: output not in ascending entry order"
 
 
-def test_indexer_scores_alone_match_oracle():
+@pytest.mark.parametrize("idx_dtype", ["fp8", "fp4"])
+def test_indexer_scores_alone_match_oracle(idx_dtype):
     """dsv4_indexer_scores: every visible entry's score (the tensor-core kernel alone), rows
     past n_entries untouched."""
-    spec = W.C4_SPEC
+    spec = W.C4_FP4_SPEC if idx_dtype == "fp4" else W.C4_SPEC
     n_list = [130, 4097, 0, 600]
     B = len(n_list)
     la = W.make_layer(spec, B, max(n_list) + 1, 24, outlier_frac=0.05)

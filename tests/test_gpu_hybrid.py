@@ -214,3 +214,21 @@ def test_query_norm_and_fp8_output_step(kind):
     dl = dsv4.DeviceLayer.from_arrays(la)
     ol = OA.layer_state(la)
     _step_and_check(dl, ol, spec, st)
+
+
+def test_c4_fp4_indexer_cache_steps():
+    """The C4 step with an fp4 (e2m1) indexer cache: 6 sequences at 9K-40K context, two
+    consecutive steps; at the second, sequences 0..2 complete a block and their new indexer
+    entry (encoded to e2m1 by the step's own prologue, scored by the top-k kernel from the
+    packed codes) is built to rank among their top k. Queries are drawn as in the benchmark
+    workload (std 1), the scale the output bound assumes."""
+    spec = W.C4_FP4_SPEC
+    B = 6
+    pos0 = np.array([9002, 12006, 40002, 9000, 17001, 33333], np.int64)
+    la = W.make_layer(spec, B, int(pos0.max()) // 4 + 8, seed=91, outlier_frac=0.05)
+    dl = dsv4.DeviceLayer.from_arrays(la)
+    ol = OA.layer_state(la)
+    for i in range(2):
+        st = W.make_step(spec, B, (pos0 + i).tolist(), seed=92 + i)
+        must = {s: _rank_new_index_entry(spec, st, s, ol) for s in range(3)} if i == 1 else None
+        _step_and_check(dl, ol, spec, st, must_select=must)

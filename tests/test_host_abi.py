@@ -39,6 +39,19 @@ def test_every_declared_function_is_exported(lib):
         assert n in A.EXPORTS, f"{n} has no binding"
 
 
+def test_package_exports_every_binding_call():
+    """Each public function and class of the binding is reachable from the package."""
+    import inspect
+
+    from compressed_sparse_kv_dsv4_b200 import binding
+
+    names = [n for n, v in vars(binding).items() if not n.startswith("_") and (inspect.isfunction(v) or
+             inspect.isclass(v)) and getattr(v, "__module__", "") == binding.__name__]
+    assert "indexer_scores" in names
+    missing = [n for n in names if not hasattr(dsv4, n)]
+    assert not missing, missing
+
+
 def test_host_helpers(lib, golden_dir):
     assert lib.dsv4_abi_version() == 2
     assert lib.dsv4_status_string(A.OK) == b"ok"
@@ -141,6 +154,10 @@ def test_validation_rejects_bad_calls(lib):
                       (dict(q_rope_dims=16), A.ERR_INVALID_ARG), (dict(k=4096), A.ERR_UNSUPPORTED)):
         a = _indexer(**bad)
         assert lib.dsv4_indexer_topk(C.byref(a), C.c_void_p(FAKE), 1 << 30, None) == code, bad
+    # fp4 (e2m1) keys: accepted for the indexer with their scales, never as an attention cache
+    assert lib.dsv4_indexer_workspace_size(C.byref(_indexer(keys=_cache(dim=128, dtype=A.FP4)))) > 0
+    assert lib.dsv4_indexer_workspace_size(C.byref(_indexer(keys=_cache(dim=128, dtype=A.FP4, scales=None)))) == 0
+    assert lib.dsv4_mqa_workspace_size(C.byref(_mqa(cache=_cache(dtype=A.FP4)))) == 0
     a = _indexer()
     need = lib.dsv4_indexer_workspace_size(C.byref(a))
     assert need >= 2 * 512 * 4  # at least one float score per cache entry of each sequence
