@@ -4,15 +4,15 @@
 //   s_j = sum_h w_h * ReLU(q_h . k_j)       for every visible C4 entry j
 //   keep the k largest s_j (ties to the lower j)
 //
-// Tensor-core path (fp8 keys, 128-dim, the C4 layers): a persistent kernel, one CTA per
-// SM, over the flattened (sequence, 128-entry tile) space, in stages of up to two tiles of
-// one sequence. Warp 0 streams key pages with TMA (8 KB boxes, 128B swizzle) into a ring of
-// 5 or 6 stages, with the block-table entries fetched a batch of 8 stages ahead, and hands
-// each stage's page rows to the epilogue; warp 1 issues tcgen05.mma kind::f8f6f4 (M = 128
-// entries, N = H heads, K = 128) into two TMEM accumulator sets; two groups of four warps
-// take alternate stages, load their keys' scales, read their accumulators back
-// (tcgen05.ld), apply ReLU, the per-head weights w_h * scale_q[h] and the per-entry key
-// scale, and store every score (4 bytes per entry, coalesced). A second kernel selects the
+// Tensor-core path (fp8 or fp4 keys, 128-dim, the C4 layers): a persistent kernel, one CTA
+// per SM, over the flattened (sequence, 128-entry tile) space, in stages of up to four tiles
+// of one sequence. Warp 0 streams key pages with TMA (one 64-row box per page and lane,
+// 128B swizzle) into a ring of 2 or 3 stages of 64 KB, with the block-table entries fetched
+// a batch of 4 stages ahead, and hands each stage's page rows to the epilogue; warp 1 issues
+// tcgen05.mma kind::f8f6f4 (M = 128 entries, N = H heads, K = 128) into two TMEM accumulator
+// sets; two groups of four warps take alternate stages, load their keys' scales, read their
+// accumulators back (tcgen05.ld), apply ReLU, the per-head weights w_h * scale_q[h] and the
+// per-entry key scale, and store every score (4 bytes per entry, coalesced). A second kernel selects the
 // top k of each sequence from the scores (a cluster radix select over registers), writing
 // them in ascending entry order.
 //
@@ -150,17 +150,20 @@ struct TcParams {
 };
 
 // The tensor-core path serves C4 layers: 64 entries per page, a 128-entry tile = 2 pages,
-// a pipeline stage = up to 2 tiles of one sequence (32 KB of keys).
+// a pipeline stage = up to 4 tiles of one sequence (64 KB of keys in shared memory). Larger
+// stages halve the producer's per-stage bookkeeping per byte, which had set its pace.
 constexpr int kPerPage = 64;
-constexpr int kStageTiles = 2;
-constexpr int kStagePages = kStageTiles * kTile / kPerPage;  // 4
+constexpr int kStageTiles = 4;
+constexpr int kStagePages = kStageTiles * kTile / kPerPage;
+constexpr int kStagesHi = 12 / kStageTiles;  // 192 KB of key stages in flight, or one stage less
+constexpr int kStagesLo = kStagesHi - 1;
 constexpr int kSlots = 8;        // ring of the stages' page rows, one slot per stage
-constexpr int kBatchStages = 32 / kStagePages;  // stages whose page ids one warp load covers (8)
+constexpr int kBatchStages = 32 / kStagePages;  // stages whose page ids one warp load covers (4)
 constexpr int kGroups = 2;       // epilogue warp groups, alternating stages
 constexpr int kGroupThreads = 128;
 constexpr int kIxThreads = 64 + kGroups * kGroupThreads;
 
-template <int H, int kStages>  // H in {32, 64}; kStages key stages of 32 KB in flight
+template <int H, int kStages>  // H in {32, 64}; kStages key stages of 64 KB in flight
 struct alignas(1024) TcSmem {
   uint8_t stage[kStages][kStageTiles][kTile * kRowBytes];  // key tiles (rows = entries)
   uint8_t q[2][H * kRowBytes];
@@ -181,7 +184,7 @@ __device__ __forceinline__ int find_seq(const long long *prefix, int B, long lon
   return lo;
 }
 
-// Walks a CTA's tile range [t0, t1) as stages of up to 2 tiles that never cross a sequence.
+// Walks a CTA's tile range [t0, t1) as stages of up to kStageTiles tiles that never cross a sequence.
 struct StageIter {
   long long g, t1;
   int b;
@@ -210,10 +213,19 @@ struct StageIter {
   }
 };
 
-// Block-table entries of the next kBatchStages stages, one per lane (lane = 4 * stage +
-// page): the loads of a whole batch are in flight together, a batch ahead of their use.
-__device__ __forceinline__ int load_page_batch(const TcParams &p, const long long *prefix, const int64_t *nvis,
-                                               StageIter &ahead, int lane) {
+// Block-table entries of the next kBatchStages stages, one per lane (lane = kStagePages *
+// stage + page): the loads of a whole batch are in flight together, a batch ahead of their use.
+// Returns the raw entry (the load is not waited for here: the address is always valid and
+// nothing reads the value until the batch is used) and whether the lane's slot has a page.
+struct PageBatch {
+  int raw;
+  bool has;
+  // the entry, or -1 (no page); the first read of `raw`, so the wait for its load is here
+  __device__ __forceinline__ int get() const { return has ? raw : -1; }
+};
+
+__device__ __forceinline__ PageBatch load_page_batch(const TcParams &p, const long long *prefix, const int64_t *nvis,
+                                                     StageIter &ahead, int lane) {
   int sb_l = -1;
   int64_t first_l = 0;
 #pragma unroll 1
@@ -222,15 +234,17 @@ __device__ __forceinline__ int load_page_batch(const TcParams &p, const long lon
     long long lt0;
     bool ns, se;
     if (!ahead.next(prefix, sb, lt0, nt, ns, se)) break;
-    if ((lane >> 2) == i && (lane & 3) < nt * 2) {
+    if (lane / kStagePages == i && lane % kStagePages < nt * (kTile / kPerPage)) {
       sb_l = sb;
-      first_l = lt0 * kTile + static_cast<int64_t>(lane & 3) * kPerPage;
+      first_l = lt0 * kTile + static_cast<int64_t>(lane % kStagePages) * kPerPage;
     }
   }
-  // the raw table entry; no page (-1) when the slot has no tile or starts past the visible
-  // entries. It is validated where it is used, so the load is not waited for here.
-  return sb_l >= 0 && first_l < nvis[sb_l] ? p.block_table[static_cast<size_t>(sb_l) * p.max_blocks + first_l / kPerPage]
-                                           : -1;
+  // no page when the slot has no tile or starts past the visible entries; the entry is
+  // validated where it is used
+  PageBatch r;
+  r.has = sb_l >= 0 && first_l < nvis[sb_l];
+  r.raw = p.block_table[r.has ? static_cast<size_t>(sb_l) * p.max_blocks + first_l / kPerPage : 0];
+  return r;
 }
 
 template <int H, int kStages>
@@ -246,7 +260,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   // ---- setup: barriers, TMEM, tile prefix over sequences
   if (tid == 0) {
     for (int i = 0; i < kStages; ++i) { mbar_init(&S.full[i], 1); mbar_init(&S.empty[i], 1); }
-    for (int i = 0; i < kSlots; ++i) { mbar_init(&S.sfull[i], 1); mbar_init(&S.sempty[i], kGroupThreads / 32); }
+    for (int i = 0; i < kSlots; ++i) { mbar_init(&S.sfull[i], kStagePages); mbar_init(&S.sempty[i], kGroupThreads / 32); }
     for (int i = 0; i < kGroups; ++i) { mbar_init(&S.tfull[i], 1); mbar_init(&S.tempty[i], kGroupThreads / 32); }
     for (int i = 0; i < 2; ++i) { mbar_init(&S.qfull[i], 1); mbar_init(&S.qempty[i], 1); }
     S.abort_flag = 0;
@@ -262,6 +276,8 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
     nvis[b] = visible_entries(p.n_entries, p.pos, p.m, b, capacity, p.d_status, blockIdx.x == 0,
                               p.before_append ? 0 : 1);
   __syncthreads();
+  StageIter it, ahead;                // the producer's walk over its stages (warp 0)
+  PageBatch batch_cur{}, batch_next{};  // and its first two batches of page ids
   if (warp == 0) {  // tiles per sequence, scanned by one warp
     long long carry = 0;
     for (int b0 = 0; b0 < p.B; b0 += 32) {
@@ -277,6 +293,14 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
       carry += __shfl_sync(0xFFFFFFFFu, v, 31);
     }
     if (lane == 0) prefix[p.B] = carry;
+    __syncwarp();
+    // The block table is written by none of the library's kernels (the only ones that may
+    // still run when this one starts early), so its first two batches load before the wait.
+    const long long G = gridDim.x;
+    it.init(prefix, p.B, (carry * blockIdx.x) / G, (carry * (blockIdx.x + 1)) / G);
+    ahead = it;
+    batch_cur = load_page_batch(p, prefix, nvis, ahead, lane);
+    batch_next = load_page_batch(p, prefix, nvis, ahead, lane);
   }
   // Keys and scales may be written by the kernel before: every read waits for it. (In a
   // decode step this kernel runs first, beside the step's own updates, which touch no entry it
@@ -292,52 +316,42 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
   const long long t0 = (T * blockIdx.x) / G, t1 = (T * (blockIdx.x + 1)) / G;
 
   if (warp == 0) {
-    // ---------------- producer. Lane 0 issues the key TMA of stage k (one box per 64-row
-    // page, completing as transaction bytes on the stage's barrier; an invalid page, or one
-    // past the visible entries, takes a zero-filled out-of-range box) and stores the stage's
-    // page rows in a small ring for the epilogue, which loads the keys' scales itself.
+    // ---------------- producer. Per stage, lanes 0..7 take one 64-row page each: its page
+    // row goes to a small ring for the epilogue (which loads the keys' scales itself), and
+    // its key box is issued as one TMA (an invalid page, or one past the visible entries,
+    // takes a zero-filled out-of-range box), completing as transaction bytes on the stage's
+    // barrier. Ring positions and phases are kept as counters: no division in the loop.
     const int oob_row = p.num_pages * kPerPage;
-    StageIter it, ahead;
-    it.init(prefix, p.B, t0, t1);
-    ahead = it;
-    int batch_cur = load_page_batch(p, prefix, nvis, ahead, lane);
-    int batch_next = load_page_batch(p, prefix, nvis, ahead, lane);
     int seg = -1;
-    long long k = 0;
+    int k = 0, bs = 0;              // stage count; stage within the page batch
+    int s = 0, slot = 0;            // key ring stage and page-row slot
+    uint32_t s_lap = 0, slot_lap = 0;
     int sb, nt;
     long long lt0;
     bool new_seg, seg_end;
     while (it.next(prefix, sb, lt0, nt, new_seg, seg_end)) {
-      const int bs = static_cast<int>(k % kBatchStages);
-      if (bs == 0 && k > 0) {
+      if (bs == kBatchStages) {
+        bs = 0;
         batch_cur = batch_next;
         batch_next = load_page_batch(p, prefix, nvis, ahead, lane);
       }
-      const int slot = static_cast<int>(k % kSlots);
-      // this stage's pages (lanes 0..3), validated: an entry outside the pool is reported and
+      // this lane's page (lanes 0..3), validated: an entry outside the pool is reported and
       // treated as no page
-      int pid = __shfl_sync(0xFFFFFFFFu, batch_cur, (bs * kStagePages + lane) & 31);
+      int pid = __shfl_sync(0xFFFFFFFFu, batch_cur.get(), (bs * kStagePages + lane) & 31);
       if (lane < kStagePages && pid != -1 && (pid < 0 || pid >= p.num_pages)) {
         report(p.d_status, DSV4_DEV_BAD_PAGE);
         pid = -1;
       }
-      if (lane >= kStagePages) pid = -1;
-      int rows[kStagePages];
-#pragma unroll
-      for (int i = 0; i < kStagePages; ++i) {
-        const int v = __shfl_sync(0xFFFFFFFFu, pid, i);
-        rows[i] = v >= 0 ? v * kPerPage : oob_row;
-      }
+      const int row = pid >= 0 ? pid * kPerPage : oob_row;
       int ok = 1;
-      if (lane == 0) {
-        if (k >= kSlots && !mbar_wait(&S.sempty[slot], static_cast<uint32_t>((k / kSlots - 1) & 1), &S.abort_flag))
-          ok = 0;
-        if (ok) {  // the pages' rows; the epilogue threads load their keys' scales themselves
-          // (as four 256-byte bulk copies per stage they held up the producer's issue)
-#pragma unroll
-          for (int i = 0; i < kStagePages; ++i) S.spage[slot][i] = rows[i];
+      if (lane < kStagePages) {
+        if (k >= kSlots && !mbar_wait(&S.sempty[slot], (slot_lap - 1) & 1, &S.abort_flag)) ok = 0;
+        if (ok) {
+          S.spage[slot][lane] = row;
           mbar_arrive(&S.sfull[slot]);
         }
+      }
+      if (lane == 0) {
         if (ok && new_seg) {
           ++seg;
           const int qs = seg & 1;
@@ -347,28 +361,27 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
             tma_load_2d(S.q[qs], &p.tmap_q, &S.qfull[qs], 0, sb * H);
           }
         }
-        const int s = static_cast<int>(k % kStages);
-        if (ok && k >= kStages && !mbar_wait(&S.empty[s], static_cast<uint32_t>((k / kStages - 1) & 1), &S.abort_flag))
-          ok = 0;
-        if (ok) {
-          // (fp4 keys: the transaction counts the packed bytes read, half the tile)
-          mbar_arrive_expect_tx(&S.full[s], static_cast<uint32_t>(nt) * kTile * (p.keys_fp4 ? kRowBytes / 2 : kRowBytes));
-          for (int t = 0; t < nt; ++t)
-#pragma unroll
-            for (int h = 0; h < 2; ++h)
-              tma_load_2d(S.stage[s][t] + h * kPerPage * kRowBytes, &p.tmap_k, &S.full[s], 0, rows[t * 2 + h]);
-        }
+        if (ok && k >= kStages && !mbar_wait(&S.empty[s], (s_lap - 1) & 1, &S.abort_flag)) ok = 0;
+        // (fp4 keys: the transaction counts the packed bytes read, half the tile)
+        if (ok) mbar_arrive_expect_tx(&S.full[s], static_cast<uint32_t>(nt) * kTile * (p.keys_fp4 ? kRowBytes / 2 : kRowBytes));
       }
-      ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+      ok = __all_sync(0xFFFFFFFFu, ok);
       if (!ok) break;
+      if (lane < nt * (kTile / kPerPage))  // lane i: page i % 2 of tile i / 2
+        tma_load_2d(S.stage[s][lane >> 1] + (lane & 1) * kPerPage * kRowBytes, &p.tmap_k, &S.full[s], 0, row);
       ++k;
+      ++bs;
+      if (++s == kStages) { s = 0; ++s_lap; }
+      if (++slot == kSlots) { slot = 0; ++slot_lap; }
     }
     if (lane == 0 && S.abort_flag) {
-      // let key loads already in flight land before the CTA leaves
-      const long long from = k > kStages ? k - kStages : 0;
-      for (long long n = from; n < k; ++n) {
+      // let key loads already in flight land before the CTA leaves: the stages issued, the
+      // last kStages of them (stage k - n sits at ring position s - n)
+      const int from = k > kStages ? kStages : k;
+      for (int n = from; n >= 1; --n) {
+        const int q = k - n;
         volatile int dummy = 0;
-        mbar_wait(&S.full[n % kStages], static_cast<uint32_t>((n / kStages) & 1), &dummy);
+        mbar_wait(&S.full[q % kStages], static_cast<uint32_t>((q / kStages) & 1), &dummy);
       }
     }
   } else if (warp == 1) {
@@ -378,16 +391,17 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
       StageIter it;
       it.init(prefix, p.B, t0, t1);
       int sb, nt, seg = -1;
-      long long lt0, k = 0;
+      long long lt0;
+      int k = 0, s = 0;
+      uint32_t s_lap = 0;
       bool new_seg, seg_end;
       while (it.next(prefix, sb, lt0, nt, new_seg, seg_end)) {
         if (new_seg) {
           ++seg;
           if (!mbar_wait(&S.qfull[seg & 1], (seg >> 1) & 1, &S.abort_flag)) break;
         }
-        const int s = static_cast<int>(k % kStages);
-        if (!mbar_wait(&S.full[s], static_cast<uint32_t>((k / kStages) & 1), &S.abort_flag)) break;
-        const int a = static_cast<int>(k % kGroups);
+        if (!mbar_wait(&S.full[s], s_lap & 1, &S.abort_flag)) break;
+        const int a = k & (kGroups - 1);
         if (k >= kGroups && !mbar_wait(&S.tempty[a], static_cast<uint32_t>((k / kGroups - 1) & 1), &S.abort_flag)) break;
         tc_fence_after();
         const uint64_t bq = sw128_desc(smem_u32(S.q[seg & 1]), 16, 1024);
@@ -401,6 +415,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
         mma_commit(&S.tfull[a]);
         if (seg_end) mma_commit(&S.qempty[seg & 1]);
         ++k;
+        if (++s == kStages) { s = 0; ++s_lap; }
       }
     }
   } else {
@@ -1017,7 +1032,7 @@ size_t tc_tail_bytes(int B) { return 1024 + (2 * static_cast<size_t>(B) + 1) * 8
 
 template <int H>
 int tc_stages(int B) {
-  return sizeof(TcSmem<H, 6>) + tc_tail_bytes(B) <= 227 * 1024 ? 6 : 5;
+  return sizeof(TcSmem<H, kStagesHi>) + tc_tail_bytes(B) <= 227 * 1024 ? kStagesHi : kStagesLo;
 }
 
 template <int H>
@@ -1046,16 +1061,16 @@ cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st, in
   tp.release = p.idx != nullptr || p.release_next ? 1 : 0;  // the top-k kernel, or a kernel of the call, follows
   // six stages in flight where shared memory allows, else five
   const size_t tail = tc_tail_bytes(p.B);
-  if (tc_stages<H>(p.B) == 6) {
-    const size_t smem = sizeof(TcSmem<H, 6>) + tail;
-    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (tc_stages<H>(p.B) == kStagesHi) {
+    const size_t smem = sizeof(TcSmem<H, kStagesHi>) + tail;
+    cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H, kStagesHi>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    return launch_pdl(indexer_tc_kernel<H, 6>, dim3(tc_grid()), dim3(kIxThreads), smem, st, 1, tp);
+    return launch_pdl(indexer_tc_kernel<H, kStagesHi>, dim3(tc_grid()), dim3(kIxThreads), smem, st, 1, tp);
   }
-  const size_t smem = sizeof(TcSmem<H, 5>) + tail;
-  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H, 5>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const size_t smem = sizeof(TcSmem<H, kStagesLo>) + tail;
+  cudaError_t e = cudaFuncSetAttribute(indexer_tc_kernel<H, kStagesLo>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(indexer_tc_kernel<H, 5>, dim3(tc_grid()), dim3(kIxThreads), smem, st, 1, tp);
+  return launch_pdl(indexer_tc_kernel<H, kStagesLo>, dim3(tc_grid()), dim3(kIxThreads), smem, st, 1, tp);
 }
 
 }  // namespace
