@@ -74,6 +74,11 @@ Readings taken where both are silent (the plainest one the text supports):
       per byte with the even element in the low nibble, plus one float32 scale
       amax/6 per row (1 if amax = 0); code = RNE_satfinite(x * (6/amax)), the
       rule of R12 with 6 the largest e2m1 magnitude.
+  R24 projection in front of the compressor ([vLLM] "vLLM side" fuses the
+      compressor with its cache insert; SGLang's "Flash Compressor"): kv_t and
+      gate_t are the products of token t's hidden state with the compressor's
+      projection weights (kv rows, then gate rows), each rounded once to bf16,
+      the compressor's input type (nearest, ties to even, from the exact value).
   R22 fp8 output ([vLLM] "vLLM side": the fused "inverse RoPE + fp8 quant"
       kernel): the output of each head, after its inverse RoPE, is stored as
       e4m3 codes in blocks of 128 channels, each block with one float32 scale
@@ -409,6 +414,25 @@ def compress_tokens(state: CompressorState, cache: PagedCache, s: int, start_pos
             blk = state.buf[s].astype(np.float64)
             entry = compress_block(blk[:, :d], blk[:, d:], t // m, m, gamma, eps, rope_dims, rope_base)
             cache.write(s, t // m, entry)
+
+
+def bf16_round_exact(x) -> np.ndarray:
+    """float64 -> the nearest bf16 value (8 significant bits), ties to even, as float64:
+    one rounding from the given value (no intermediate float32)."""
+    x = np.asarray(x, dtype=np.float64)
+    m, e = np.frexp(x)  # x = m * 2^e, 0.5 <= |m| < 1
+    return np.ldexp(np.round(np.ldexp(m, 8)), e - 8)  # np.round: half to even
+
+
+def project(hidden, w, dim: int):
+    """R24: kv = bf16(hidden . w[:dim]^T), gate = bf16(hidden . w[dim:]^T), each element
+    rounded once from its exact (float64) dot product. hidden [T, Hd], w [2 dim, Hd] as
+    values; returns (kv, gate) as bf16 bits [T, dim]."""
+    h = np.asarray(hidden, dtype=np.float64)
+    wt = np.asarray(w, dtype=np.float64)
+    out = bf16_round_exact(h @ wt.T)
+    bits = bf16_encode(out.astype(np.float32))  # exact: every value is a bf16 value
+    return bits[:, :dim], bits[:, dim:]
 
 
 def compress(kv, gate, cu_seqlens, start_pos, state: CompressorState, cache: PagedCache,

@@ -427,3 +427,53 @@ def test_fp4_rows_pack_and_scale():
     # e2m1 keeps 1 mantissa bit: relative error <= 1/4 above the subnormal range
     big = np.abs(x) >= float(scale)
     assert np.all(np.abs(dec[big] - x[big]) <= 0.25 * np.abs(x[big]) + 1e-12)
+
+
+# ----------------------------------------------------------------- projection (R24)
+def _bf16_neighbours(v: float):
+    """The two bf16 values around v (v itself twice when v is one), from the bit patterns."""
+    f = np.float32(v)
+    u = int(np.array([f]).view(np.uint32)[0])
+    lo_bits = u & 0xFFFF0000
+    lo = float(np.array([lo_bits], np.uint32).view(np.float32)[0])
+    hi = float(np.array([lo_bits + 0x10000], np.uint32).view(np.float32)[0])
+    return (lo, hi) if abs(lo) <= abs(v) else (hi, lo)
+
+
+def test_bf16_round_exact_is_nearest_ties_to_even():
+    # hand ties: halfway between 1 and 1 + 2^-7 goes to 1 (even), halfway above goes up
+    got = O.bf16_round_exact(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -(1 + 2.0 ** -8), 3.0, 0.0]))
+    assert list(got) == [1.0, 1 + 2.0 ** -6, -1.0, 3.0, 0.0]
+    # random values against the two neighbouring bf16 values, chosen by distance (float64 values
+    # that float32 would round first are included: the rounding is from the exact value)
+    xs = np.concatenate([RNG.standard_normal(3000) * 10.0 ** RNG.integers(-3, 4, 3000),
+                         1 + (2 * RNG.integers(0, 64, 200) + 1) * 2.0 ** -8 + 2.0 ** -40])
+    for v, r in zip(xs, O.bf16_round_exact(xs)):
+        a, b = sorted(_bf16_neighbours(v), key=abs)
+        da, db = abs(v - a), abs(v - b)
+        assert r == (a if da < db else b if db < da else r), (v, r, a, b)
+        assert r in (a, b)
+
+
+def test_projection_brute_force_and_closed_forms():
+    # brute force: every output element as an explicit sum over the hidden dim
+    T, Hd, D = 3, 5, 2
+    h = RNG.standard_normal((T, Hd))
+    w = RNG.standard_normal((2 * D, Hd))
+    kv, gate = O.project(h, w, D)
+    for t in range(T):
+        for c in range(2 * D):
+            acc = 0.0
+            for i in range(Hd):
+                acc += h[t, i] * w[c, i]
+            want = O.bf16_round_exact(acc)
+            got = O.bf16_decode(kv[t, c] if c < D else gate[t, c - D])
+            assert got == want, (t, c)
+    # identity weights: kv is the hidden state, gate twice it, each rounded to bf16
+    h2 = RNG.standard_normal((4, 8))
+    kv2, gate2 = O.project(h2, np.vstack([np.eye(8), 2 * np.eye(8)]), 8)
+    assert np.array_equal(O.bf16_decode(kv2), O.bf16_round_exact(h2))
+    assert np.array_equal(O.bf16_decode(gate2), O.bf16_round_exact(2 * h2))
+    # scaling the hidden state by a power of two scales the output exactly
+    kv3, _ = O.project(4.0 * h2, np.vstack([np.eye(8), np.eye(8)]), 8)
+    assert np.array_equal(O.bf16_decode(kv3), 4.0 * O.bf16_decode(kv2))
