@@ -5,6 +5,7 @@ this package is its thin Python binding over torch CUDA tensors.
 """
 
 from .binding import (DeviceCache, DeviceLayer, DeviceRing, DeviceState, DeviceStep, compress,  # noqa: F401
+                      compress_project,
                       hybrid_decode, indexer_args, indexer_scores, indexer_topk, indexer_topk_noalloc,
                       layer_state_bytes, mqa_args, mqa_workspace_size, sparse_mqa_decode, swa_insert,
                       to_device_codes, to_numpy_codes)

@@ -44,6 +44,10 @@ class CompressArgs(C.Structure):
                 ("state", CompressorState), ("cache", PagedCache), ("d_status", p)]
 
 
+class CompressProjectArgs(C.Structure):
+    _fields_ = [("c", CompressArgs), ("hidden", p), ("w", p), ("hidden_dim", i32)]
+
+
 class SwaInsertArgs(C.Structure):
     _fields_ = [("batch", i32), ("total_tokens", i32), ("kv", p), ("kv_dtype", C.c_int), ("cu_seqlens", p),
                 ("start_pos", p), ("gamma", p), ("eps", C.c_float), ("rope", Rope), ("ring", WindowRing),
@@ -81,6 +85,8 @@ class Step(C.Structure):
 
 EXPORTS = {
     "dsv4_compress": (C.c_int, [C.POINTER(CompressArgs), p]),
+    "dsv4_compress_project_workspace_size": (C.c_size_t, [C.POINTER(CompressProjectArgs)]),
+    "dsv4_compress_project": (C.c_int, [C.POINTER(CompressProjectArgs), p, C.c_size_t, p]),
     "dsv4_swa_insert": (C.c_int, [C.POINTER(SwaInsertArgs), p]),
     "dsv4_indexer_workspace_size": (C.c_size_t, [C.POINTER(IndexerArgs)]),
     "dsv4_indexer_topk": (C.c_int, [C.POINTER(IndexerArgs), p, C.c_size_t, p]),

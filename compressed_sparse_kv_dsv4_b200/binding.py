@@ -249,6 +249,31 @@ def compress(kv, gate, cu_seqlens, start_pos, state: DeviceState, cache: DeviceC
     A.check("dsv4_compress", lib.dsv4_compress(C.byref(a), _stream(stream)))
 
 
+def compress_project(hidden, w, cu_seqlens, start_pos, state: DeviceState, cache: DeviceCache, gamma, *,
+                     eps: float = 1e-6, rope_dims: int = 64, rope_base: float = 10000.0, d_status=None,
+                     workspace=None, stream=None):
+    """dsv4_compress_project: kv, gate = bf16(hidden [T, Hd] . w [2D, Hd]^T) on the tensor cores,
+    then the compressor. Returns (kv, gate): views [T, D] bf16 of the workspace, which hold
+    the projection after the call."""
+    lib = A.load()
+    T, Hd = hidden.shape
+    D = state.dim
+    c = A.CompressArgs(batch=cu_seqlens.shape[0] - 1, total_tokens=T, kv=None, gate=None, kv_dtype=A.BF16,
+                       cu_seqlens=_ptr(cu_seqlens), start_pos=_ptr(start_pos), gamma=_ptr(gamma), eps=eps,
+                       rope=A.Rope(rope_dims, rope_base), state=state.struct(), cache=cache.struct(),
+                       d_status=_ptr(d_status))
+    a = A.CompressProjectArgs(c=c, hidden=_ptr(hidden), w=_ptr(w), hidden_dim=Hd)
+    need = lib.dsv4_compress_project_workspace_size(C.byref(a))
+    if need == 0:
+        A.check("dsv4_compress_project_workspace_size", A.ERR_INVALID_ARG)
+    ws = workspace if workspace is not None else torch.empty(need, dtype=torch.uint8, device=hidden.device)
+    A.check("dsv4_compress_project", lib.dsv4_compress_project(C.byref(a), _ptr(ws), ws.numel(), _stream(stream)))
+    off = (T * D * 2 + 255) // 256 * 256
+    kv = ws[:T * D * 2].view(torch.bfloat16).view(T, D)
+    gate = ws[off:off + T * D * 2].view(torch.bfloat16).view(T, D)
+    return kv, gate
+
+
 def swa_insert(kv, cu_seqlens, start_pos, ring: DeviceRing, gamma, *, kv_dtype: str, eps: float = 1e-6,
                rope_dims: int = 64, rope_base: float = 10000.0, d_status=None, stream=None):
     lib = A.load()

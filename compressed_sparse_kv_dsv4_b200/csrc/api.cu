@@ -84,6 +84,32 @@ bool valid_pool_dim(int d) { return pow2(d) && d >= 32 && d <= 2048; }
 
 }  // namespace
 
+namespace {
+// the checks of dsv4_compress that do not look at kv, gate and kv_dtype
+dsv4_status check_compress_common(const dsv4_compress_args *a) {
+  if (a->batch <= 0 || a->batch > 16384 || a->total_tokens < 0) return DSV4_ERR_INVALID_ARG;
+  if (!a->cu_seqlens || !a->start_pos || !a->gamma) return DSV4_ERR_INVALID_ARG;
+  if (!valid_state(a->state) || !valid_cache(a->cache)) return DSV4_ERR_INVALID_ARG;
+  if (a->state.m != a->cache.m || a->state.dim != a->cache.dim) return DSV4_ERR_INVALID_ARG;
+  if (!valid_rope(a->rope, a->state.dim) || !(a->eps >= 0.f)) return DSV4_ERR_INVALID_ARG;
+  if (!valid_pool_dim(a->state.dim)) return DSV4_ERR_UNSUPPORTED;
+  return DSV4_OK;
+}
+
+// the projection's own rules (beside those of dsv4_compress); DSV4_OK or the error
+dsv4_status check_project(const dsv4_compress_project_args *a) {
+  if (!a) return DSV4_ERR_INVALID_ARG;
+  const dsv4_status c = check_compress_common(&a->c);
+  if (c != DSV4_OK) return c;
+  if (a->c.total_tokens > 0 && (!a->hidden || !a->w)) return DSV4_ERR_INVALID_ARG;
+  if (!aligned16(a->hidden) || !aligned16(a->w)) return DSV4_ERR_INVALID_ARG;
+  if (a->hidden_dim <= 0) return DSV4_ERR_INVALID_ARG;
+  if (a->c.state.gate_dim != a->c.state.dim) return DSV4_ERR_UNSUPPORTED;
+  if (a->hidden_dim % 64 != 0 || a->c.state.dim % 128 != 0) return DSV4_ERR_UNSUPPORTED;
+  return DSV4_OK;
+}
+}  // namespace
+
 extern "C" {
 
 const char *dsv4_status_string(dsv4_status s) {
@@ -111,14 +137,10 @@ uint64_t dsv4_layer_state_bytes(uint64_t context, int32_t m, int32_t entry_width
 // ------------------------------------------------------------------------------------
 dsv4_status dsv4_compress(const dsv4_compress_args *a, dsv4_stream stream) {
   if (!a) return DSV4_ERR_INVALID_ARG;
-  if (a->batch <= 0 || a->batch > 16384 || a->total_tokens < 0) return DSV4_ERR_INVALID_ARG;
-  if (!a->cu_seqlens || !a->start_pos || !a->gamma) return DSV4_ERR_INVALID_ARG;
+  const dsv4_status c = check_compress_common(a);
+  if (c != DSV4_OK) return c;
   if (a->total_tokens > 0 && (!a->kv || !a->gate)) return DSV4_ERR_INVALID_ARG;
-  if (!valid_state(a->state) || !valid_cache(a->cache)) return DSV4_ERR_INVALID_ARG;
-  if (a->state.m != a->cache.m || a->state.dim != a->cache.dim) return DSV4_ERR_INVALID_ARG;
-  if (!valid_rope(a->rope, a->state.dim) || !(a->eps >= 0.f)) return DSV4_ERR_INVALID_ARG;
   if (a->kv_dtype != DSV4_F32 && a->kv_dtype != DSV4_BF16) return DSV4_ERR_UNSUPPORTED;
-  if (!valid_pool_dim(a->state.dim)) return DSV4_ERR_UNSUPPORTED;
   if (!aligned16(a->kv) || !aligned16(a->gate)) return DSV4_ERR_INVALID_ARG;
   if (a->total_tokens == 0) return DSV4_OK;
   CompressLaunch p{};
@@ -145,6 +167,38 @@ dsv4_status dsv4_compress(const dsv4_compress_args *a, dsv4_stream stream) {
   p.cache_dt = a->cache.dtype;
   p.d_status = a->d_status;
   return to_status(launch_compress(p, static_cast<cudaStream_t>(stream)));
+}
+
+size_t dsv4_compress_project_workspace_size(const dsv4_compress_project_args *a) {
+  if (check_project(a) != DSV4_OK) return 0;
+  return 2 * project_out_bytes(a->c.total_tokens, a->c.state.dim) + 256;
+}
+
+dsv4_status dsv4_compress_project(const dsv4_compress_project_args *a, void *ws, size_t ws_bytes,
+                                  dsv4_stream stream) {
+  const dsv4_status c = check_project(a);
+  if (c != DSV4_OK) return c;
+  if (a->c.total_tokens == 0) return DSV4_OK;
+  if (!ws || reinterpret_cast<uintptr_t>(ws) % 256 != 0 || ws_bytes < dsv4_compress_project_workspace_size(a))
+    return DSV4_ERR_INVALID_ARG;
+  const int T = a->c.total_tokens, D = a->c.state.dim;
+  ProjectLaunch pj{};
+  pj.hidden = a->hidden;
+  pj.w = a->w;
+  pj.kv = static_cast<uint16_t *>(ws);
+  pj.gate = reinterpret_cast<uint16_t *>(static_cast<char *>(ws) + project_out_bytes(T, D));
+  pj.T = T;
+  pj.D = D;
+  pj.Hd = a->hidden_dim;
+  pj.d_status = a->c.d_status;
+  const cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_project(pj, st);
+  if (e != cudaSuccess) return to_status(e);
+  dsv4_compress_args cc = a->c;
+  cc.kv = pj.kv;
+  cc.gate = pj.gate;
+  cc.kv_dtype = DSV4_BF16;
+  return dsv4_compress(&cc, stream);
 }
 
 dsv4_status dsv4_swa_insert(const dsv4_swa_insert_args *a, dsv4_stream stream) {

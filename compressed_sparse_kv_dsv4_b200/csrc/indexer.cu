@@ -969,18 +969,6 @@ __global__ void __launch_bounds__(kSelThreads) topk_select_kernel(const unsigned
 // ------------------------------------------------------------------------------------
 // host side
 
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
-    void *ptr = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
-  return fn;
-}
-
 // Rows of 128 values: e4m3 (128 bytes each), or e2m1 (fp4: 64 packed bytes each, landing in
 // shared memory as 128-byte rows with each 8 bytes of values followed by 8 bytes of gap, the
 // operand layout of the f8f6f4 MMA's e2m1 type). 128B swizzle either way.
@@ -1074,6 +1062,18 @@ cudaError_t launch_tc(const IndexerLaunch &p, float *scores, cudaStream_t st, in
 }
 
 }  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
 
 bool indexer_uses_tensor_cores(const IndexerLaunch &p) {
   const bool keys_ok = p.k_dt == DSV4_FP8E4M3 ||

@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 #include <stdint.h>
@@ -14,6 +15,9 @@ namespace dsv4 {
 
 // number of SMs of the current device (cached per device)
 int sm_count();
+
+// the driver's cuTensorMapEncodeTiled (null if the driver does not provide it)
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn();
 
 // RoPE's angle step of pair 1, base^(-2/rope_dims), in float64 on the host; pair i turns by
 // pos * theta1^i. The launchers fill the rope_theta1 fields below from it.
@@ -45,6 +49,20 @@ struct CompressLaunch {
   uint32_t *d_status;
 };
 cudaError_t launch_compress(const CompressLaunch &p, cudaStream_t st);
+
+// The compressor's input projection: kv [T][D] and gate [T][D] (bf16) = bf16(hidden . w^T),
+// hidden [T][Hd] and w [2D][Hd] bf16 (kv rows, then gate rows). Hd % 64 == 0, D % 128 == 0.
+struct ProjectLaunch {
+  const void *hidden;
+  const void *w;
+  uint16_t *kv;
+  uint16_t *gate;
+  int T, D, Hd;
+  uint32_t *d_status;
+};
+// bytes of one projected [T][D] bf16 array in the workspace (256-byte aligned)
+size_t project_out_bytes(int T, int D);
+cudaError_t launch_project(const ProjectLaunch &p, cudaStream_t st);
 
 struct SwaLaunch {
   int B;

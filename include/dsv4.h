@@ -55,7 +55,7 @@
 extern "C" {
 #endif
 
-#define DSV4_ABI_VERSION 2
+#define DSV4_ABI_VERSION 3
 
 typedef void *dsv4_stream; /* a cudaStream_t; NULL = the legacy default stream */
 
@@ -161,6 +161,36 @@ typedef struct {
 } dsv4_compress_args;
 
 dsv4_status dsv4_compress(const dsv4_compress_args *args, dsv4_stream stream);
+
+/* ------------------------------------------------------------------------------------
+ * dsv4_compress_project: dsv4_compress with the compressor's input projection in front
+ * (the projection GEMM of the fused compressor: vLLM "compressor + RMSNorm + RoPE + cache
+ * insert", SGLang "Flash Compressor"). The kv and gate of token t are its hidden state times
+ * the projection weights, each rounded once to bf16 (reading R24):
+ *   kv[t][c]   = bf16( sum_i hidden[t][i] * w[c][i] )          c < dim
+ *   gate[t][c] = bf16( sum_i hidden[t][i] * w[dim + c][i] )    (one gate per channel)
+ * computed on the tensor cores (bf16 operands, fp32 accumulation, one rounding to bf16),
+ * then compressed exactly as dsv4_compress with kv_dtype = DSV4_BF16.
+ *   c             the compressor arguments; c.kv, c.gate and c.kv_dtype are ignored;
+ *                 c.state.gate_dim must equal c.state.dim, and dim must be a multiple of 128.
+ *   hidden        [c.total_tokens][hidden_dim] bf16, 16-byte aligned (caller-owned).
+ *   w             [2 * dim][hidden_dim] bf16, 16-byte aligned: the kv rows, then the gate rows.
+ *   hidden_dim    a positive multiple of 64.
+ * Workspace: dsv4_compress_project_workspace_size() bytes, 256-byte aligned, caller-owned.
+ * After the call it holds the projected kv [total_tokens][dim] bf16 at offset 0 and gate
+ * [total_tokens][dim] bf16 at offset round_up(total_tokens * dim * 2, 256).
+ * Errors as dsv4_compress; DSV4_ERR_UNSUPPORTED for a dim or hidden_dim outside the rules.
+ */
+typedef struct {
+  dsv4_compress_args c;
+  const void *hidden;
+  const void *w;
+  int32_t hidden_dim;
+} dsv4_compress_project_args;
+
+size_t dsv4_compress_project_workspace_size(const dsv4_compress_project_args *args);
+dsv4_status dsv4_compress_project(const dsv4_compress_project_args *args, void *workspace, size_t workspace_bytes,
+                                  dsv4_stream stream);
 
 /* ------------------------------------------------------------------------------------
  * dsv4_swa_insert: window keys of new tokens (vLLM "Q-norm + KV RoPE + K insert", the K

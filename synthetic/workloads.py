@@ -369,6 +369,40 @@ def compressor_prefill(seed: int = 3, B: int = 8, tokens_per_seq: int = 4096, D:
     return PrefillWorkload(cu, sp, kv4, g4, kv128, g128, layers[0], layers[1])
 
 
+@dataclass
+class ProjectionWorkload:
+    cu_seqlens: np.ndarray   # [B+1] int32
+    start_pos: np.ndarray    # [B] int32
+    hidden: np.ndarray       # [T, Hd] bf16 bits, ~ N(0, 1)
+    w4: np.ndarray           # [2D, Hd] bf16 bits, ~ N(0, 1/Hd): the C4 compressor's kv rows, then gate rows
+    w128: np.ndarray         # the C128 compressor's
+    layer4: LayerArrays      # C4 caches + state
+    layer128: LayerArrays
+
+
+def projection_prefill(seed: int = 5, B: int = 8, tokens_per_seq: int = 4096, hidden_dim: int = 4096,
+                       D: int = 512, start_pos=None, lens=None, cache_dtype: str = "bf16") -> ProjectionWorkload:
+    """Hidden states of new tokens and the projection weights of two compressors (m = 4 and
+    m = 128): hidden ~ N(0,1), weights ~ N(0, 1/hidden_dim), so kv and gate come out ~ N(0,1)
+    like the compressor prefill's inputs. `lens` (per sequence) overrides tokens_per_seq."""
+    rng = rng_for(seed)
+    lens = np.full(B, tokens_per_seq, np.int64) if lens is None else np.asarray(lens, np.int64)
+    B = lens.shape[0]
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    T = int(cu[-1])
+    sp = np.zeros(B, np.int32) if start_pos is None else np.asarray(start_pos, np.int32)
+    hidden = bf16_bits(normal_f32(rng, (T, hidden_dim)))
+    w4 = bf16_bits(normal_f32(rng, (2 * D, hidden_dim), 1.0 / np.sqrt(hidden_dim)))
+    w128 = bf16_bits(normal_f32(rng, (2 * D, hidden_dim), 1.0 / np.sqrt(hidden_dim)))
+    layers = []
+    for m in (4, 128):
+        spec = LayerSpec(kind="c128", m=m, H=64, D=D, cache_dtype=cache_dtype, swa_dtype="bf16")
+        ctx = int((sp + lens).max())
+        la = make_layer(spec, B, ctx // m + 1, seed * 100 + m, spare_blocks=1)
+        layers.append(la)
+    return ProjectionWorkload(cu, sp, hidden, w4, w128, layers[0], layers[1])
+
+
 def stack_1m(seed: int = 4, B: int = 4, context: int = 1 << 20, steps: int = 16):
     """Two C4 (fp8) and two C128 (bf16) layers at 1M context; per-layer inputs
     for `steps` consecutive decode steps."""

@@ -53,7 +53,7 @@ def test_package_exports_every_binding_call():
 
 
 def test_host_helpers(lib, golden_dir):
-    assert lib.dsv4_abi_version() == 2
+    assert lib.dsv4_abi_version() == 3
     assert lib.dsv4_status_string(A.OK) == b"ok"
     assert lib.dsv4_status_string(A.ERR_INVALID_ARG) == b"invalid argument"
     assert lib.dsv4_status_string(99) == b"unknown status"
@@ -190,6 +190,39 @@ def test_compress_and_window_validation(lib):
     w2 = A.SwaInsertArgs.from_buffer_copy(w)
     w2.total_tokens = 0
     assert lib.dsv4_swa_insert(C.byref(w2), None) == A.OK
+
+
+def test_compress_project_validation_and_workspace(lib):
+    """dsv4_compress_project: the compressor's checks, plus hidden_dim % 64, dim % 128 and one
+    gate per channel; the workspace holds the projected kv and gate (bf16, 256-byte aligned)."""
+    state = A.CompressorState(FAKE, 4, 512, 512)
+    c = A.CompressArgs(batch=2, total_tokens=1000, kv=None, gate=None, kv_dtype=A.F32, cu_seqlens=FAKE,
+                       start_pos=FAKE, gamma=FAKE, eps=1e-6, rope=A.Rope(64, 1e4), state=state, cache=_cache(),
+                       d_status=None)
+    a = A.CompressProjectArgs(c=c, hidden=FAKE, w=FAKE, hidden_dim=4096)
+    need = lib.dsv4_compress_project_workspace_size(C.byref(a))
+    per = (1000 * 512 * 2 + 255) // 256 * 256
+    assert 2 * per <= need <= 2 * per + 256
+    assert lib.dsv4_compress_project(None, None, 0, None) == A.ERR_INVALID_ARG
+    for field, val, code in (("hidden_dim", 100, A.ERR_UNSUPPORTED), ("hidden_dim", 0, A.ERR_INVALID_ARG),
+                             ("hidden", None, A.ERR_INVALID_ARG), ("w", FAKE + 8, A.ERR_INVALID_ARG)):
+        b = A.CompressProjectArgs.from_buffer_copy(a)
+        setattr(b, field, val)
+        assert lib.dsv4_compress_project(C.byref(b), C.c_void_p(FAKE), need, None) == code, field
+        assert lib.dsv4_compress_project_workspace_size(C.byref(b)) == 0
+    b = A.CompressProjectArgs.from_buffer_copy(a)
+    b.c.state = A.CompressorState(FAKE, 4, 512, 1)  # one gate per token: not what the projection makes
+    assert lib.dsv4_compress_project(C.byref(b), C.c_void_p(FAKE), need, None) == A.ERR_UNSUPPORTED
+    b = A.CompressProjectArgs.from_buffer_copy(a)
+    b.c.state = A.CompressorState(FAKE, 4, 192, 192)
+    b.c.cache = _cache(dim=192)
+    assert lib.dsv4_compress_project(C.byref(b), C.c_void_p(FAKE), 1 << 30, None) == A.ERR_UNSUPPORTED
+    # a short or misaligned workspace is refused before any launch
+    assert lib.dsv4_compress_project(C.byref(a), C.c_void_p(FAKE), need - 1, None) == A.ERR_INVALID_ARG
+    assert lib.dsv4_compress_project(C.byref(a), C.c_void_p(FAKE + 16), need, None) == A.ERR_INVALID_ARG
+    b = A.CompressProjectArgs.from_buffer_copy(a)
+    b.c.total_tokens = 0  # nothing to do
+    assert lib.dsv4_compress_project(C.byref(b), None, 0, None) == A.OK
 
 
 def test_hybrid_validation_and_workspace(lib):
