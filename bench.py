@@ -321,6 +321,56 @@ def leg_compress_prefill(lib, dev, stream, flush, hbm_peak: float, iters: int = 
     return out
 
 
+def leg_compress_project(lib, dev, stream, flush, peaks: dict, iters: int = 10) -> dict:
+    """The compressor prefill with its projection: 8 x 4096 tokens of bf16 hidden states
+    (hidden 4096) projected on the tensor cores into kv and gate (D = 512) for a C4 and a C128
+    compressor, each then compressed (dsv4_compress_project, one call per compressor).
+    FLOPs counted: the projections only, 2 T hidden 2D per compressor."""
+    import torch
+
+    import compressed_sparse_kv_dsv4_b200 as dsv4
+    from compressed_sparse_kv_dsv4_b200 import _abi as A
+    import synthetic as W
+
+    wl = W.projection_prefill()
+    B, T = wl.start_pos.shape[0], int(wl.cu_seqlens[-1])
+    Hd, D = wl.hidden.shape[1], wl.layer4.spec.D
+    cu = torch.from_numpy(wl.cu_seqlens).to(dev)
+    sp = torch.from_numpy(wl.start_pos).to(dev)
+    hid = dsv4.to_device_codes(wl.hidden, "bf16", dev)
+    calls = []
+    for la, w in ((wl.layer4, wl.w4), (wl.layer128, wl.w128)):
+        spec = la.spec
+        dl = dsv4.DeviceLayer.from_arrays(la, dev)
+        wd = dsv4.to_device_codes(w, "bf16", dev)
+        c = A.CompressArgs(batch=B, total_tokens=T, kv=None, gate=None, kv_dtype=A.BF16, cu_seqlens=cu.data_ptr(),
+                           start_pos=sp.data_ptr(), gamma=dl.gamma.data_ptr(), eps=spec.eps,
+                           rope=A.Rope(spec.rope_dims, spec.rope_base), state=dl.state.struct(),
+                           cache=dl.cache.struct(), d_status=None)
+        a = A.CompressProjectArgs(c=c, hidden=hid.data_ptr(), w=wd.data_ptr(), hidden_dim=Hd)
+        ws = torch.empty(lib.dsv4_compress_project_workspace_size(C.byref(a)), dtype=torch.uint8, device=dev)
+        calls.append((spec.m, a, ws, (dl, wd)))
+    sh = C.c_void_p(stream.cuda_stream)
+    flops = 2.0 * T * Hd * 2 * D  # per compressor
+    bf16_peak = float(peaks.get("bf16_tflops", 1590.0))
+    out = {"workload": "compressor_prefill_projected_8x4096", "tokens": T, "hidden": Hd, "kv_dim": D,
+           "cache": "bf16", "flops_per_compressor": flops, "peak_tflops": bf16_peak,
+           "peak_source": "measured" if "bf16_tflops" in peaks else "fallback"}
+    total = 0.0
+    for m, a, ws, _keep in calls:
+        ms = event_mean_ms(stream, lambda j, a=a, ws=ws: A.check("dsv4_compress_project", lib.dsv4_compress_project(
+            C.byref(a), C.c_void_p(ws.data_ptr()), ws.numel(), sh)), iters, flush)
+        tf = flops / (ms * 1e-3) / 1e12
+        out[f"c{m}"] = {"ms": round(ms, 5), "tflops": round(tf, 1), "frac": round(tf / bf16_peak, 4)}
+        total += ms
+    out["both"] = {"ms": round(total, 5), "tflops": round(2 * flops / (total * 1e-3) / 1e12, 1),
+                   "frac": round(2 * flops / (total * 1e-3) / 1e12 / bf16_peak, 4),
+                   "tokens_per_s": round(T / (total * 1e-3), 1)}
+    del calls, hid
+    torch.cuda.empty_cache()
+    return out
+
+
 def leg_stack_1m(lib, dev, stream, flush, hbm_peak: float, steps: int = 16) -> dict:
     """The 1M-context mixed stack: two C4 layers (262144 fp8 entries, top-512) and two C128
     layers (8192 bf16 entries), 4 sequences; one step = the four layers' dsv4_hybrid_decode
@@ -593,6 +643,7 @@ def run_ours(args):
     if world == 1 and not args.no_extra:
         line["compress_prefill"] = leg_compress_prefill(lib, dev, stream, flush, hbm_peak)
         line["c4_fp4_indexer"] = leg_c4_fp4_indexer(lib, dev, stream, flush, hbm_peak)
+        line["compress_project"] = leg_compress_project(lib, dev, stream, flush, peaks)
         if not args.skip_1m:
             line["stack_1m"] = leg_stack_1m(lib, dev, stream, flush, hbm_peak)
     if world == 1 and not args.no_cpu_baseline:
