@@ -183,7 +183,8 @@ def _indexer_case(n_list, k, H=64, seed=21, spec=W.C4_SPEC, all_negative=False):
     st = W.make_step(spec, B, 0, seed + 1)
     if all_negative:  # every q.k < 0: all scores are exactly zero
         st.q_idx = st.q_idx & 0x7F
-        la.idx_pages = la.idx_pages | 0x80
+        # the sign bit of every key element: bit 7 of an e4m3 code, bit 3 of each e2m1 nibble
+        la.idx_pages = la.idx_pages | (0x88 if spec.idx_dtype == "fp4" else 0x80)
     dl = dsv4.DeviceLayer.from_arrays(la)
     q = dsv4.to_device_codes(st.q_idx, spec.q_idx_dtype, "cuda")
     w = dsv4.to_device_codes(st.w, spec.w_dtype, "cuda")
@@ -281,8 +282,10 @@ def test_indexer_scores_alone_match_oracle(idx_dtype):
             assert np.all(np.abs(got[s_, :n] - ref) <= 1e-5 * np.abs(ref).max()), f"seq {s_}"
 
 
-def test_indexer_full_tie_takes_lowest_indices():
-    idx, scores, ol, qd, wd = _indexer_case([3000, 700], 512, all_negative=True)
+@pytest.mark.parametrize("idx_dtype", ["fp8", "fp4"])
+def test_indexer_full_tie_takes_lowest_indices(idx_dtype):
+    spec = W.C4_FP4_SPEC if idx_dtype == "fp4" else W.C4_SPEC
+    idx, scores, ol, qd, wd = _indexer_case([3000, 700], 512, all_negative=True, spec=spec)
     for s in range(2):
         assert sorted(idx[s].tolist()) == list(range(512))
         assert np.all(scores[s] == 0.0)

@@ -178,17 +178,18 @@ def test_stack_1m_sixteen_steps(out_dtype):
             _step_and_check(dls[li], ols[li], spec, step_sets[li][i], attend=attend, must_select=must)
 
 
-@pytest.mark.parametrize("out_dtype", OUT_DTYPES)
-def test_c4_first_tokens_window_only(out_dtype):
+@pytest.mark.parametrize("out_dtype,idx_dtype", [("f32", "fp8"), ("bf16", "fp8"), ("bf16", "fp4")])
+def test_c4_first_tokens_window_only(out_dtype, idx_dtype):
     """Positions 0, 1, 2 (then one step further): no complete block in any sequence at the
     first step, so the indexer has no tile; the output is the window-only softmax over the
     positions 0..p, the newest of which the step itself inserted.
 
-    The window and the main cache are bf16 here (the indexer stays fp8, on the tensor cores):
+    The window and the main cache are bf16 here (the indexer stays fp8 or fp4, on the tensor cores):
     with one to three keys the output is nearly the new key itself, and an fp8 code that the
     two sides round one step apart (allowed for rows each side builds itself) would move it
     by up to 1/16 of the element, more than the output bound; one bf16 step stays within it."""
-    spec = _with_out(dataclasses.replace(W.C4_SPEC, cache_dtype="bf16", swa_dtype="bf16"), out_dtype)
+    spec = _with_out(dataclasses.replace(W.C4_SPEC, cache_dtype="bf16", swa_dtype="bf16", idx_dtype=idx_dtype),
+                     out_dtype)
     B = 3
     la = W.make_layer(spec, B, 4, seed=61, outlier_frac=0.05)
     dl = dsv4.DeviceLayer.from_arrays(la)

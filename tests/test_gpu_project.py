@@ -58,12 +58,16 @@ def _rows_close_e2e(g_codes, g_scale, r_codes, r_scale, dtype, ctx):
     weights), and the RMSNorm scales that by 1/rms: every decoded value agrees within one
     rounding step of the cache dtype plus 2^-6 of itself plus 2^-3 of the row's rms, and at most
     10 % of them (the channels a changed input reached) need more than the first two terms.
-    An fp8 row's scale (amax/448) agrees within 2^-5."""
+    An fp8 or fp4 row's scale (amax/448, amax/6) agrees within 2^-5."""
     g = O.decode_rows(np.asarray(g_codes)[None], np.array([g_scale], np.float32), dtype)[0]
     r = O.decode_rows(np.asarray(r_codes)[None], np.array([r_scale], np.float32), dtype)[0]
     if dtype == "fp8":
         assert abs(float(g_scale) - float(r_scale)) <= 2.0 ** -5 * float(r_scale), f"{ctx}: scale"
         step = np.exp2(np.floor(np.log2(np.maximum(np.abs(r) / float(r_scale), 2.0 ** -6))) - 3) * float(r_scale)
+    elif dtype == "fp4":  # e2m1 magnitudes 0 .5 1 1.5 2 3 4 6: steps of 1/2, 1, 2 (times the scale)
+        assert abs(float(g_scale) - float(r_scale)) <= 2.0 ** -5 * float(r_scale), f"{ctx}: scale"
+        a = np.abs(r) / float(r_scale)
+        step = np.where(a < 2, 0.5, np.where(a < 4, 1.0, 2.0)) * float(r_scale)
     else:
         step = np.exp2(np.floor(np.log2(np.maximum(np.abs(r), 2.0 ** -126))) - 7)
     rms = float(np.sqrt(np.mean(r * r)))
@@ -122,7 +126,7 @@ def _run(wl, which, seqs=None):
     return gkv, ggate
 
 
-@pytest.mark.parametrize("m,D,cache_dtype", [(4, 128, "fp8"), (4, 512, "bf16"), (128, 512, "fp8")])
+@pytest.mark.parametrize("m,D,cache_dtype", [(4, 128, "fp8"), (4, 128, "fp4"), (4, 512, "bf16"), (128, 512, "fp8")])
 def test_compress_project_matches_oracle(m, D, cache_dtype):
     """Three sequences of 37, 300 and 129 tokens (several 128-token tiles, ragged tails, a
     sequence starting mid-block), hidden_dim 320 (five 64-wide slices)."""
