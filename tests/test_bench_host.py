@@ -25,3 +25,24 @@ def test_packed_step_inputs_are_views_of_one_buffer_with_the_same_bytes():
     assert raw <= host.numel() <= raw + 255 * len(bench.STEP_INPUTS)
     # the rest of the step (outputs, positions, status) is the same
     assert packed.out is ds.out and packed.pos is ds.pos and packed.d_status is ds.d_status
+
+
+def test_algorithmic_byte_counts():
+    """The byte counts behind the bench's fractions, against the per-sequence figures worked
+    out by hand: C3 (32768 fp8 indexer keys of 128 B + a 4 B scale; 640 attended rows of
+    512 B + 4 B; bf16 query and output; the step's updates), its fp4 variant (64 B keys), the
+    dense C128 step and the compressor prefill."""
+    import bench
+
+    b = bench.algorithmic_bytes_per_seq(32768)
+    assert b["indexer"] == 32768 * 132 + 64 * 128 + 64 * 4 + 64 * 2 == 4_333_952
+    assert b["attention"] == 640 * 516 + 64 * 512 * 2 * 2 == 461_312
+    assert b["total"] == 4_803_460
+    assert bench.c4_step_bytes_per_seq(32768) * 32 == 153_710_720
+    f4 = bench.algorithmic_bytes_per_seq(32768, idx_row_bytes=64)
+    assert f4["indexer"] == 32768 * 68 + 64 * 128 + 64 * 4 + 64 * 2
+    assert f4["total"] - b["total"] == f4["indexer"] - b["indexer"]
+    # dense C128: every entry and the window rows in bf16, q and o, the updates
+    assert bench.c128_bytes_per_seq(512) == (512 + 128) * 1024 + 2 * 64 * 512 * 2 + (2 * 512 * 2 + 2 * 512 * 4 + 1024)
+    # compressor prefill: 8 x 4096 bf16 tokens (kv + gate), 1024 entries per sequence at m = 4
+    assert bench.prefill_bytes(32768, 8, 4) == 32768 * 2048 + 8 * 1024 * 1024 + 8 * 4 * 4096
