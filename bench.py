@@ -63,6 +63,15 @@ def c128_bytes_per_seq(n_c: int, D: int = 512, H: int = 64, W: int = 128) -> int
     return (n_c + W) * 2 * D + 2 * H * D * 2 + (2 * D * 2 + 2 * D * 4 + 2 * D)
 
 
+def c4_step_flops_per_seq(n_c: int) -> dict:
+    """Tensor-core FLOPs of one sequence's C4 step: the indexer's q . k for every visible entry
+    (2 H_I d_I each) and the attention's two products over the k + W keys (4 H D each)."""
+    D, H, k, W, H_I, d_I = (SPEC_ROWS[x] for x in ("D", "H", "k", "W", "H_I", "d_I"))
+    idx = 2 * H_I * d_I * n_c
+    attn = 4 * H * (k + W) * D
+    return dict(indexer=idx, attention=attn, total=idx + attn)
+
+
 def c4_step_bytes_per_seq(n_c: int) -> int:
     return algorithmic_bytes_per_seq(n_c)["total"]
 
@@ -622,6 +631,8 @@ def run_ours(args):
 
     byts = algorithmic_bytes_per_seq(n_c, out_bytes=4 if spec.out_dtype == "f32" else 2)
     step_bytes = byts["total"] * B_PER_GPU
+    fl = c4_step_flops_per_seq(n_c)
+    step_flops, ix_flops = fl["total"] * B_PER_GPU, fl["indexer"] * B_PER_GPU
     ix_bytes = byts["indexer"] * B_PER_GPU
     peaks = {}
     try:
@@ -648,6 +659,9 @@ def run_ours(args):
         "hbm": {"step_algorithmic_bytes": step_bytes, "achieved_gbs": round(step_gbs, 1),
                 "pct_of_8tbs": round(100 * step_gbs / 8000.0, 1),
                 "pct_of_measured_copy": round(100 * step_gbs / hbm_peak, 1)},
+        "tflops": {"step": round(step_flops / (ms * 1e-3) / 1e12, 1),
+                   "indexer_alone": round(ix_flops / (sc_ms * 1e-3) / 1e12, 1),
+                   "step_flops": step_flops, "note": "fp8 indexer and fp16 attention MMAs; HBM-bound"},
         "roofline": {"kernel": "indexer_tc_kernel (dsv4_indexer_scores)", "bound": "hbm",
                      "achieved": round(sc_gbs, 1), "peak": hbm_peak, "peak_source": peak_src, "unit": "GB/s",
                      "frac": round(sc_gbs / hbm_peak, 4), "traffic": traffic, "algorithmic_bytes_per_launch": ix_bytes,

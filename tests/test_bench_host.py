@@ -46,3 +46,13 @@ def test_algorithmic_byte_counts():
     assert bench.c128_bytes_per_seq(512) == (512 + 128) * 1024 + 2 * 64 * 512 * 2 + (2 * 512 * 2 + 2 * 512 * 4 + 1024)
     # compressor prefill: 8 x 4096 bf16 tokens (kv + gate), 1024 entries per sequence at m = 4
     assert bench.prefill_bytes(32768, 8, 4) == 32768 * 2048 + 8 * 1024 * 1024 + 8 * 4 * 4096
+
+
+def test_step_flop_counts():
+    """The C3 step's tensor-core FLOPs: 17.2 GFLOP of indexer products and 2.7 GFLOP of attention
+    for 32 sequences."""
+    import bench
+
+    f = bench.c4_step_flops_per_seq(32768)
+    assert f["indexer"] * 32 == 2 * 64 * 128 * 32768 * 32 == 17_179_869_184
+    assert f["attention"] * 32 == 4 * 64 * 640 * 512 * 32 == 2_684_354_560
