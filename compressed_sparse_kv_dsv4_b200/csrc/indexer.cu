@@ -335,7 +335,7 @@ __global__ void __launch_bounds__(kIxThreads, 1) indexer_tc_kernel(const __grid_
         batch_cur = batch_next;
         batch_next = load_page_batch(p, prefix, nvis, ahead, lane);
       }
-      // this lane's page (lanes 0..3), validated: an entry outside the pool is reported and
+      // this lane's page (lanes 0..7), validated: an entry outside the pool is reported and
       // treated as no page
       int pid = __shfl_sync(0xFFFFFFFFu, batch_cur.get(), (bs * kStagePages + lane) & 31);
       if (lane < kStagePages && pid != -1 && (pid < 0 || pid >= p.num_pages)) {
