@@ -477,3 +477,15 @@ def test_projection_brute_force_and_closed_forms():
     # scaling the hidden state by a power of two scales the output exactly
     kv3, _ = O.project(4.0 * h2, np.vstack([np.eye(8), np.eye(8)]), 8)
     assert np.array_equal(O.bf16_decode(kv3), 4.0 * O.bf16_decode(kv2))
+
+
+def test_e2m1_encode_matches_library_cast():
+    """The e2m1 encoder against ml_dtypes' float4_e2m1fn cast (round to nearest even,
+    saturating at 6) on random values inside and beyond the range, and signed zeros."""
+    ml_dtypes = pytest.importorskip("ml_dtypes")
+    x = np.concatenate([RNG.uniform(-7.5, 7.5, 50000), RNG.standard_normal(20000) * 3,
+                        np.array([0.0, -0.0, 6.0, -6.0, 6.5, -9.0, 0.2, -0.2])]).astype(np.float32)
+    ours = O.e2m1_decode(O.e2m1_encode(x))
+    lib = x.astype(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    assert np.array_equal(ours, lib)
+    assert np.array_equal(np.signbit(ours[ours == 0]), np.signbit(lib[lib == 0]))
