@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(kPThreads, 1) project_kernel(const __grid_cons
           }
         }
       }
-      if (!ok) {  // let the copies in flight land before the CTA leaves
+      if (!ok || S.abort_flag) {  // a role gave up: let the copies in flight land before the CTA leaves
         const int from = issued > kPStages ? kPStages : issued;
         for (int n = from; n >= 1; --n) {
           const int q = issued - n;
